@@ -1,0 +1,151 @@
+"""Plain fp64 CPU oracle for exact softmax attention, forward and backward.
+
+TEST INFRASTRUCTURE ONLY.  Nothing on the product path imports this module:
+only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may call it.  It shares no code with the CUDA library.
+
+What it computes (the plain definition that the tiled method reaches exactly,
+up to floating-point reassociation -- "Attention and KV Compression",
+section "What it does and does not change"; "FlashAttention -- how 100K-token
+attention fits in memory", section "Why 'exact' matters"):
+
+    S = scale * Q K^T                  (N x N, materialised per head)
+    S_ij = -inf  for j > i             (causal mask, if requested)
+    P = softmax(S) row-wise            (p_i = e^{s_i} / sum_j e^{s_j}, FlashAttention
+                                        page, section "But softmax needs the whole row")
+    O = P V
+    LSE_i = m_i + ln sum_j exp(S_ij - m_i),   m_i = max_j S_ij
+
+The backward is the explicit chain rule through the same materialised
+matrices (the quantities the tiled backward recomputes tile by tile --
+"Attention and KV Compression", section "Recomputation in the backward pass"):
+
+    dV = P^T dO
+    dP = dO V^T
+    D_i = sum_j P_ij dP_ij
+    dS = P o (dP - D)
+    dQ = scale * dS K
+    dK = scale * dS^T Q
+
+All arithmetic is float64 (numpy); matrix products use numpy's matmul as a
+library primitive.  Inputs are arrays of shape (BH, N, d) (any float dtype,
+upcast to float64 here); heads are processed one at a time so that only one
+N x N matrix per head is resident.
+
+Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
+(worked online-softmax example, row sums, blockwise-vs-one-shot equality,
+closed forms, finite differences, an autograd cross-check).
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "head_scores",
+    "row_softmax",
+    "attn_fwd",
+    "attn_fwd_rows",
+    "attn_bwd",
+]
+
+
+def head_scores(q: np.ndarray, k: np.ndarray, scale: float, causal: bool,
+                rows: np.ndarray | None = None) -> np.ndarray:
+    """Scaled scores of one head, with the causal mask written in as -inf.
+
+    ``rows`` selects a subset of query rows (their global indices); the mask
+    uses those global indices.  The mask form (key j visible to query i iff
+    j <= i, queries and keys indexed from the same origin) is the plain
+    reading of the "mask" step of standard attention (FlashAttention flagship
+    page, Beat 01).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    if rows is None:
+        rows = np.arange(q.shape[0])
+    else:
+        rows = np.asarray(rows, dtype=np.int64)
+        q = q[rows]
+    s = float(scale) * (q @ k.T)
+    if causal:
+        cols = np.arange(k.shape[0])
+        s[cols[None, :] > rows[:, None]] = -np.inf
+    return s
+
+
+def row_softmax(s: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """Row-wise softmax and log-sum-exp of a score matrix.
+
+    p_ij = exp(s_ij - m_i) / sum_j exp(s_ij - m_i) with m_i the row maximum;
+    LSE_i = m_i + ln sum_j exp(s_ij - m_i).  Returns (P, LSE).
+    """
+    m = np.max(s, axis=1, keepdims=True)
+    e = np.exp(s - m)
+    l = np.sum(e, axis=1, keepdims=True)
+    p = e / l
+    lse = (m + np.log(l))[:, 0]
+    return p, lse
+
+
+def _as3(x: np.ndarray) -> np.ndarray:
+    x = np.asarray(x, dtype=np.float64)
+    if x.ndim == 2:
+        x = x[None]
+    if x.ndim != 3:
+        raise ValueError("expected (BH, N, d) or (N, d)")
+    return x
+
+
+def attn_fwd(Q, K, V, scale: float, causal: bool, return_probs: bool = False):
+    """Forward: O (BH, N, d) and LSE (BH, N); optionally P (BH, N, N)."""
+    Q, K, V = _as3(Q), _as3(K), _as3(V)
+    bh, n, d = Q.shape
+    O = np.empty((bh, n, d), dtype=np.float64)
+    LSE = np.empty((bh, n), dtype=np.float64)
+    Ps = np.empty((bh, n, n), dtype=np.float64) if return_probs else None
+    for h in range(bh):
+        s = head_scores(Q[h], K[h], scale, causal)
+        p, lse = row_softmax(s)
+        del s
+        O[h] = p @ V[h]
+        LSE[h] = lse
+        if return_probs:
+            Ps[h] = p
+    if return_probs:
+        return O, LSE, Ps
+    return O, LSE
+
+
+def attn_fwd_rows(q, k, v, scale: float, causal: bool, rows):
+    """Forward for selected query rows of ONE head: O_rows (r, d), LSE_rows (r,).
+
+    Row i of the result depends only on row i of S, so this is the same
+    definition evaluated on a subset of rows (used where N is too large to
+    materialise the full N x N matrix in host memory).
+    """
+    v = np.asarray(v, dtype=np.float64)
+    s = head_scores(q, k, scale, causal, rows=rows)
+    p, lse = row_softmax(s)
+    return p @ v, lse
+
+
+def attn_bwd(Q, K, V, dO, scale: float, causal: bool):
+    """Backward: dQ, dK, dV (each (BH, N, d)) from the explicit chain rule."""
+    Q, K, V, dO = _as3(Q), _as3(K), _as3(V), _as3(dO)
+    bh, n, d = Q.shape
+    dQ = np.empty((bh, n, d), dtype=np.float64)
+    dK = np.empty((bh, n, d), dtype=np.float64)
+    dV = np.empty((bh, n, d), dtype=np.float64)
+    for h in range(bh):
+        s = head_scores(Q[h], K[h], scale, causal)
+        p, _ = row_softmax(s)
+        del s
+        dV[h] = p.T @ dO[h]
+        dp = dO[h] @ V[h].T
+        D = np.sum(p * dp, axis=1, keepdims=True)
+        ds = p * (dp - D)
+        del dp, p
+        dQ[h] = float(scale) * (ds @ K[h])
+        dK[h] = float(scale) * (ds.T @ Q[h])
+    return dQ, dK, dV

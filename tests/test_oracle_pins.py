@@ -1,0 +1,408 @@
+"""Pins for the fp64 oracle: checks against what the pages and mathematics fix.
+
+None of these re-types the oracle's formulas.  Each pin comes from somewhere
+else: the worked example printed on the pages, an invariant (rows of P sum to
+one, permutation equivariance), an independent blockwise online-softmax
+routine written here from the pages' description, closed forms of special
+cases, central finite differences, or a library autograd.  Together they are
+chosen so that a dropped term, a wrong sign or index, or a transposed operand
+anywhere in the oracle fails at least one of them (``test_planted_mistakes``
+checks that claim by planting such mistakes).
+"""
+
+import math
+import os
+
+import numpy as np
+import pytest
+
+from oracle import attn_oracle as orc
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _read_golden(name):
+    out = {}
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, val = (t.strip() for t in line.split("=", 1))
+            out[key] = [float(x) for x in val.split()]
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Independent blockwise online softmax (test-only), written from the pages'
+# description: "Attention and KV Compression", section "Tiling and online
+# softmax"; FlashAttention page, sections "FlashAttention idea" and
+# "Online softmax intuition".  Plain Python loops, fp64.
+# ---------------------------------------------------------------------------
+
+def blockwise_attention(q, k, v, scale, causal, br, bc, trace=None):
+    n, d = q.shape
+    out = np.zeros((n, d))
+    lse = np.zeros(n)
+    for i0 in range(0, n, br):
+        for r in range(i0, min(i0 + br, n)):
+            m_run = -math.inf
+            l_run = 0.0
+            acc = [0.0] * d
+            for j0 in range(0, n, bc):
+                cols = range(j0, min(j0 + bc, n))
+                s = []
+                for c in cols:
+                    if causal and c > r:
+                        s.append(-math.inf)
+                    else:
+                        s.append(scale * sum(q[r, t] * k[c, t] for t in range(d)))
+                blk_max = max(s)
+                m_new = max(m_run, blk_max)
+                if m_new == -math.inf:
+                    continue
+                alpha = 0.0 if m_run == -math.inf else math.exp(m_run - m_new)
+                if trace is not None and m_run != -math.inf:
+                    trace.append((r, m_run, m_new, alpha))
+                l_run *= alpha
+                acc = [a * alpha for a in acc]
+                for c, sc in zip(cols, s):
+                    p = math.exp(sc - m_new)
+                    l_run += p
+                    for t in range(d):
+                        acc[t] += p * v[c, t]
+                m_run = m_new
+            out[r] = [a / l_run for a in acc]
+            lse[r] = m_run + math.log(l_run)
+    return out, lse
+
+
+def _rand(shape, seed):
+    return np.random.default_rng(seed).standard_normal(shape)
+
+
+# ---------------------------------------------------------------------------
+# The worked example printed on the pages
+# ---------------------------------------------------------------------------
+
+def test_worked_example_rescale_and_exactness():
+    g = _read_golden("online_softmax_worked_example.txt")
+    s1, s2 = g["block1_scores"], g["block2_scores"]
+    scores = s1 + s2
+    n = len(scores)
+    # One query whose scores against the keys are exactly the printed ones:
+    # q = e_0, k_j = scores[j] e_0, scale 1.  V = identity, so O row 0 = P row 0.
+    d = n
+    q = np.zeros((n, d)); q[0, 0] = 1.0
+    k = np.zeros((n, d)); k[:, 0] = scores
+    v = np.eye(n)
+    trace = []
+    o_blk, lse_blk = blockwise_attention(q, k, v, 1.0, False, br=1, bc=len(s1), trace=trace)
+    # The pages: block max 3, then the max moves to 4 and the accumulator is
+    # rescaled by e^(3-4) = e^(-1).
+    row0 = [t for t in trace if t[0] == 0]
+    assert len(row0) == 1
+    _, m_old, m_new, alpha = row0[0]
+    assert m_old == g["block1_max"][0]
+    assert m_new == g["new_max"][0]
+    assert alpha == pytest.approx(math.exp(g["rescale_exponent"][0]), rel=0, abs=1e-16)
+    # ... and blockwise equals the one-shot global softmax (the oracle).
+    O, LSE, P = orc.attn_fwd(q, k, v, 1.0, False, return_probs=True)
+    np.testing.assert_allclose(O[0, 0], o_blk[0], rtol=1e-14, atol=1e-16)
+    np.testing.assert_allclose(LSE[0, 0], lse_blk[0], rtol=1e-14)
+    np.testing.assert_allclose(O[0, 0], P[0, 0], rtol=0, atol=1e-15)
+    # Ratios of probabilities are e^(score difference); probabilities sum to 1.
+    p = P[0, 0]
+    for a in range(n):
+        for b in range(n):
+            assert p[a] / p[b] == pytest.approx(math.exp(scores[a] - scores[b]), rel=1e-13)
+    assert p.sum() == pytest.approx(1.0, abs=1e-15)
+    # LSE of the row is ln of the sum of exponentials (math.fsum of math.exp).
+    assert LSE[0, 0] == pytest.approx(math.log(math.fsum(math.exp(x) for x in scores)), rel=1e-15)
+
+
+# ---------------------------------------------------------------------------
+# Invariants
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_rows_of_p_sum_to_one(causal):
+    q, k, v = _rand((3, 37, 8), 1), _rand((3, 37, 8), 2), _rand((3, 37, 8), 3)
+    _, _, P = orc.attn_fwd(q, k, v, 0.7, causal, return_probs=True)
+    np.testing.assert_allclose(P.sum(axis=-1), 1.0, rtol=0, atol=1e-14)
+    assert (P >= 0).all()
+    if causal:
+        iu = np.triu_indices(37, 1)
+        assert (P[:, iu[0], iu[1]] == 0).all()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("n,d", [(1, 1), (2, 3), (5, 2), (7, 4), (9, 3)])
+def test_blockwise_equals_one_shot_every_split(causal, n, d):
+    q, k, v = _rand((n, d), 10 + n), _rand((n, d), 20 + n), _rand((n, d), 30 + n)
+    O, LSE = orc.attn_fwd(q, k, v, 0.9, causal)
+    for br in range(1, n + 1):
+        for bc in range(1, n + 1):
+            o_blk, lse_blk = blockwise_attention(q, k, v, 0.9, causal, br, bc)
+            np.testing.assert_allclose(o_blk, O[0], rtol=1e-12, atol=1e-13)
+            np.testing.assert_allclose(lse_blk, LSE[0], rtol=1e-12, atol=1e-13)
+
+
+def test_permutation_equivariance_noncausal():
+    rng = np.random.default_rng(5)
+    q, k, v = _rand((11, 6), 6), _rand((11, 6), 7), _rand((11, 6), 8)
+    O, LSE = orc.attn_fwd(q, k, v, 0.5, False)
+    pk = rng.permutation(11)
+    O2, LSE2 = orc.attn_fwd(q, k[pk], v[pk], 0.5, False)
+    np.testing.assert_allclose(O2, O, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(LSE2, LSE, rtol=1e-13)
+    pq = rng.permutation(11)
+    O3, LSE3 = orc.attn_fwd(q[pq], k, v, 0.5, False)
+    np.testing.assert_allclose(O3[0], O[0][pq], rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(LSE3[0], LSE[0][pq], rtol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# Closed forms
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_equal_scores_give_mean_of_visible_values(causal):
+    n, d = 13, 5
+    q = _rand((n, d), 40)
+    k = np.tile(_rand((1, d), 41), (n, 1))     # every key identical
+    v = _rand((n, d), 42)
+    O, LSE = orc.attn_fwd(q, k, v, 0.3, causal)
+    for i in range(n):
+        vis = i + 1 if causal else n
+        np.testing.assert_allclose(O[0, i], v[:vis].mean(axis=0), rtol=1e-13, atol=1e-14)
+        s = 0.3 * float(q[i] @ k[0])
+        assert LSE[0, i] == pytest.approx(s + math.log(vis), rel=1e-13, abs=1e-13)
+
+
+def test_causal_first_row_is_first_value():
+    q, k, v = _rand((9, 4), 50), _rand((9, 4), 51), _rand((9, 4), 52)
+    O, LSE = orc.attn_fwd(q, k, v, 0.8, True)
+    np.testing.assert_allclose(O[0, 0], v[0], rtol=0, atol=1e-15)
+    assert LSE[0, 0] == pytest.approx(0.8 * float(q[0] @ k[0]), rel=1e-14)
+
+
+def test_single_key_returns_value():
+    q, k, v = _rand((1, 7), 53), _rand((1, 7), 54), _rand((1, 7), 55)
+    for causal in (False, True):
+        O, LSE = orc.attn_fwd(q, k, v, 1.3, causal)
+        np.testing.assert_allclose(O[0], v, rtol=0, atol=1e-15)
+        assert LSE[0, 0] == pytest.approx(1.3 * float(q[0] @ k[0]), rel=1e-14)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_zero_scale_is_uniform_average(causal):
+    n = 10
+    q, k, v = _rand((n, 3), 56), _rand((n, 3), 57), _rand((n, 3), 58)
+    O, LSE = orc.attn_fwd(q, k, v, 0.0, causal)
+    for i in range(n):
+        vis = i + 1 if causal else n
+        np.testing.assert_allclose(O[0, i], v[:vis].mean(axis=0), rtol=1e-13, atol=1e-14)
+        assert LSE[0, i] == pytest.approx(math.log(vis), rel=1e-14)
+
+
+def test_constant_values_give_constant_output():
+    q, k = _rand((12, 4), 60), _rand((12, 4), 61)
+    v = np.tile(np.array([[1.5, -2.0, 0.25, 3.0]]), (12, 1))
+    for causal in (False, True):
+        O, _ = orc.attn_fwd(q, k, v, 0.6, causal)
+        np.testing.assert_allclose(O[0], v, rtol=1e-14, atol=1e-14)
+
+
+def test_dominant_key_selects_its_value():
+    n, d = 6, 3
+    q = np.zeros((n, d)); q[:, 0] = 1.0
+    k = np.zeros((n, d)); k[4, 0] = 60.0       # score 60 vs 0 elsewhere
+    v = _rand((n, d), 62)
+    O, LSE = orc.attn_fwd(q, k, v, 1.0, False)
+    # weight of key 4 is 1/(1 + 5 e^-60); error < 5 e^-60 * max|v|
+    np.testing.assert_allclose(O[0], np.tile(v[4], (n, 1)), rtol=0, atol=1e-24)
+    np.testing.assert_allclose(LSE[0], 60.0 + math.log1p(5 * math.exp(-60.0)), rtol=1e-15)
+
+
+def test_rows_variant_matches_full():
+    q, k, v = _rand((40, 8), 63), _rand((40, 8), 64), _rand((40, 8), 65)
+    rows = np.array([0, 3, 17, 39, 22])
+    for causal in (False, True):
+        O, LSE = orc.attn_fwd(q, k, v, 0.35, causal)
+        o_r, l_r = orc.attn_fwd_rows(q, k, v, 0.35, causal, rows)
+        np.testing.assert_allclose(o_r, O[0][rows], rtol=1e-14, atol=1e-15)
+        np.testing.assert_allclose(l_r, LSE[0][rows], rtol=1e-14)
+
+
+# ---------------------------------------------------------------------------
+# Backward: finite differences and a library autograd
+# ---------------------------------------------------------------------------
+
+def _loss(q, k, v, g, scale, causal):
+    O, _ = orc.attn_fwd(q, k, v, scale, causal)
+    return float(np.sum(O[0] * g))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("n,d", [(1, 2), (2, 3), (3, 4), (5, 2), (8, 3)])
+def test_backward_matches_central_differences(causal, n, d):
+    scale = 0.45
+    q, k, v, g = (_rand((n, d), 70 + i + 10 * n + 100 * d) for i in range(4))
+    dQ, dK, dV = orc.attn_bwd(q, k, v, g, scale, causal)
+    h = 1e-6
+    for name, x, grad in (("q", q, dQ[0]), ("k", k, dK[0]), ("v", v, dV[0])):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(*x.shape):
+            xp = x.copy(); xp[idx] += h
+            xm = x.copy(); xm[idx] -= h
+            args_p = {"q": q, "k": k, "v": v}; args_p[name] = xp
+            args_m = {"q": q, "k": k, "v": v}; args_m[name] = xm
+            fp = _loss(args_p["q"], args_p["k"], args_p["v"], g, scale, causal)
+            fm = _loss(args_m["q"], args_m["k"], args_m["v"], g, scale, causal)
+            num[idx] = (fp - fm) / (2 * h)
+        tol = 1e-7 * max(1.0, float(np.max(np.abs(num))))
+        np.testing.assert_allclose(grad, num, rtol=0, atol=tol, err_msg=name)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_matches_torch_autograd_fp64(causal):
+    torch = pytest.importorskip("torch")
+    bh, n, d, scale = 3, 33, 16, 0.25
+    Q, K, V, G = (_rand((bh, n, d), 90 + i) for i in range(4))
+    dQ, dK, dV = orc.attn_bwd(Q, K, V, G, scale, causal)
+    O, LSE = orc.attn_fwd(Q, K, V, scale, causal)
+    tq, tk, tv = (torch.tensor(x, dtype=torch.float64, requires_grad=True) for x in (Q, K, V))
+    s = scale * tq @ tk.transpose(-1, -2)
+    if causal:
+        s = s.masked_fill(torch.ones(n, n, dtype=torch.bool).triu(1), float("-inf"))
+    o = torch.softmax(s, dim=-1) @ tv
+    o.backward(torch.tensor(G))
+    np.testing.assert_allclose(O, o.detach().numpy(), rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(LSE, torch.logsumexp(s, dim=-1).detach().numpy(), rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(dQ, tq.grad.numpy(), rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(dK, tk.grad.numpy(), rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(dV, tv.grad.numpy(), rtol=1e-11, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# The pins catch plausible mistakes: plant each one in the oracle (on the CPU)
+# and check that at least one pin then fails.
+# ---------------------------------------------------------------------------
+
+def _pins_hold(mod):
+    """Run a compact subset of the pins above against ``mod``; True if all hold."""
+    try:
+        rng = np.random.default_rng(123)
+        n, d = 6, 3
+        q, k, v, g = (rng.standard_normal((n, d)) for _ in range(4))
+        for causal in (False, True):
+            O, LSE = mod.attn_fwd(q, k, v, 0.7, causal)
+            for br, bc in ((1, 1), (2, 3), (4, 2)):
+                ob, lb = blockwise_attention(q, k, v, 0.7, causal, br, bc)
+                if not (np.allclose(ob, O[0], rtol=1e-10, atol=1e-12)
+                        and np.allclose(lb, LSE[0], rtol=1e-10, atol=1e-12)):
+                    return False
+            dQ, dK, dV = mod.attn_bwd(q, k, v, g, 0.7, causal)
+            h = 1e-6
+            for name, x, grad in (("q", q, dQ[0]), ("k", k, dK[0]), ("v", v, dV[0])):
+                for idx in [(0, 0), (n - 1, d - 1), (2, 1)]:
+                    a = {"q": q.copy(), "k": k.copy(), "v": v.copy()}
+                    b = {"q": q.copy(), "k": k.copy(), "v": v.copy()}
+                    a[name][idx] += h
+                    b[name][idx] -= h
+                    fa = float(np.sum(mod.attn_fwd(a["q"], a["k"], a["v"], 0.7, causal)[0][0] * g))
+                    fb = float(np.sum(mod.attn_fwd(b["q"], b["k"], b["v"], 0.7, causal)[0][0] * g))
+                    if abs((fa - fb) / (2 * h) - grad[idx]) > 1e-6:
+                        return False
+        return True
+    except Exception:
+        return False
+
+
+def test_pins_hold_for_the_oracle():
+    assert _pins_hold(orc)
+
+
+_MUTANTS = {
+    "scores_transposed": lambda m: setattr(
+        m, "head_scores", _wrap_scores(lambda s: s.T.copy())),
+    "mask_off_by_one": lambda m: setattr(
+        m, "head_scores", _shifted_mask_scores),
+    "no_normalisation": lambda m: setattr(
+        m, "row_softmax", lambda s: (np.exp(s - s.max(1, keepdims=True)), orc.row_softmax(s)[1])),
+    "lse_without_max": lambda m: setattr(
+        m, "row_softmax", lambda s: (orc.row_softmax(s)[0], np.log(np.sum(np.exp(s - s.max(1, keepdims=True)), 1)))),
+    "scale_squared": lambda m: setattr(
+        m, "head_scores", lambda q, k, scale, causal, rows=None: orc.head_scores(q, k, scale * scale, causal, rows)),
+}
+
+
+def _wrap_scores(f):
+    def hs(q, k, scale, causal, rows=None):
+        s = orc.head_scores(q, k, scale, False, rows)
+        s = f(s)
+        if causal:
+            n = s.shape[1]
+            r = np.arange(s.shape[0]) if rows is None else np.asarray(rows)
+            s[np.arange(n)[None, :] > r[:, None]] = -np.inf
+        return s
+    return hs
+
+
+def _shifted_mask_scores(q, k, scale, causal, rows=None):
+    s = orc.head_scores(q, k, scale, False, rows)
+    if causal:
+        n = s.shape[1]
+        r = np.arange(s.shape[0]) if rows is None else np.asarray(rows)
+        s[np.arange(n)[None, :] >= r[:, None]] = -np.inf
+        s[0, 0] = scale * float(np.asarray(q)[0] @ np.asarray(k)[0])
+    return s
+
+
+def _bwd_mutant(kind):
+    def bwd(Q, K, V, dO, scale, causal):
+        Q, K, V, dO = orc._as3(Q), orc._as3(K), orc._as3(V), orc._as3(dO)
+        outs = [np.empty_like(Q) for _ in range(3)]
+        for h in range(Q.shape[0]):
+            p, _ = orc.row_softmax(orc.head_scores(Q[h], K[h], scale, causal))
+            dp = dO[h] @ V[h].T
+            D = np.sum(p * dp, axis=1, keepdims=True)
+            if kind == "ds_sign":
+                ds = p * (dp + D)
+            elif kind == "ds_no_D":
+                ds = p * dp
+            else:
+                ds = p * (dp - D)
+            dv = p.T @ dO[h] if kind != "dv_untransposed" else p @ dO[h]
+            dq = scale * (ds @ K[h]) if kind != "dq_no_scale" else ds @ K[h]
+            dk = scale * (ds.T @ Q[h]) if kind != "dk_untransposed" else scale * (ds @ Q[h])
+            outs[0][h], outs[1][h], outs[2][h] = dq, dk, dv
+        return tuple(outs)
+    return bwd
+
+
+for _k in ("ds_sign", "ds_no_D", "dv_untransposed", "dq_no_scale", "dk_untransposed"):
+    _MUTANTS["bwd_" + _k] = (lambda kind: (lambda m: setattr(m, "attn_bwd", _bwd_mutant(kind))))(_k)
+
+
+@pytest.mark.parametrize("mutant", sorted(_MUTANTS))
+def test_planted_mistakes_are_caught(mutant, monkeypatch):
+    import importlib
+    import types
+    mod = types.ModuleType("oracle_mutant")
+    src = importlib.import_module("oracle.attn_oracle")
+    for name in dir(src):
+        setattr(mod, name, getattr(src, name))
+    # The mutant's functions look up helpers through ``mod``: rebind the
+    # entry points so that they call the (possibly replaced) helpers.
+    def attn_fwd(Q, K, V, scale, causal, return_probs=False):
+        Q, K, V = orc._as3(Q), orc._as3(K), orc._as3(V)
+        O = np.empty_like(Q); L = np.empty(Q.shape[:2])
+        for h in range(Q.shape[0]):
+            p, lse = mod.row_softmax(mod.head_scores(Q[h], K[h], scale, causal))
+            O[h] = p @ V[h]; L[h] = lse
+        return O, L
+    mod.attn_fwd = attn_fwd
+    _MUTANTS[mutant](mod)
+    assert not _pins_hold(mod), f"planted mistake {mutant!r} was not caught by any pin"

@@ -1,0 +1,426 @@
+#!/usr/bin/env python
+"""Benchmark: exact attention forward + backward on B200, one JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one pass of the whole hot path over one batch: attn_fwd, then the
+backward (attn_bwd_preprocess, attn_bwd_dkdv, attn_bwd_dq), on the long-batch
+workload B=8, H=32, N=16384, d=128, causal, bf16 (the configuration whose
+target is forward >= 60 % and forward+backward >= 45 % of dense BF16 peak).
+Inputs are 1 GiB per tensor (larger than the 126 MB L2), so no L2 flush is
+needed between steps.
+
+Metric: attention TFLOP/s of forward+backward, counted as 4 N^2 d per head for
+the forward (halved under the causal mask) and 2.5x that for the backward.
+Multi-GPU (torchrun, one rank per GPU): every rank runs its own batch of the
+same workload (weak scaling, no collective on the data path); ``value`` is the
+FLOPs of all ranks over the slowest rank's time.
+
+``--impl reference`` times the fp64 CPU oracle on a bounded sample (the exact
+causal prefix sub-problem of one head: its first rows/keys), on rank 0 only.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "long_batch"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+METRIC = "attention TFLOP/s fwd and fwd+bwd at 1 B200; % of dense BF16 tensor peak"
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def csrc_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "exact_io_aware_58_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f)
+    ent = rec.get(WORKLOAD, {}).get(kernel)
+    if not ent or ent.get("csrc_hash") != csrc_hash():
+        return None
+    return ent.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        self.out = os.path.join("/tmp", f"bench_clocks_{os.getpid()}.csv")
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.out, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        try:
+            for line in open(self.out):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 7:
+                    continue
+                try:
+                    sm.append(float(parts[0]))
+                    mx.append(float(parts[1]))
+                except ValueError:
+                    continue
+                for nm, v in zip(names, parts[3:7]):
+                    if v.lower().startswith("active"):
+                        reasons.add(nm)
+            os.unlink(self.out)
+        except Exception:
+            pass
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def flops_fwd_per_rank(w) -> float:
+    return w.flops_fwd(True)
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from exact_io_aware_58_b200 import attn
+    from exact_io_aware_58_b200.inputs import WORKLOADS, workload_inputs
+
+    w = WORKLOADS[WORKLOAD]
+    causal = True
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    attn.load_library()
+    stream = torch.cuda.current_stream()
+
+    inp = workload_inputs(w, seed=1234 + rank, device=dev)
+    q, k, v, do = inp["Q"], inp["K"], inp["V"], inp["dO"]
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = attn.alloc_workspace(w.B, w.H, w.N, w.d, dev)
+    scale = w.scale
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        attn.attn_fwd(q, k, v, o, lse, causal, scale, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        attn.attn_bwd_preprocess(o, do, lse, ws, stream)
+        if ev is not None:
+            ev[2].record(stream)
+        attn.attn_bwd_dkdv(q, k, v, do, dk, dv, causal, scale, ws, stream)
+        if ev is not None:
+            ev[3].record(stream)
+        attn.attn_bwd_dq(q, k, v, do, dq, causal, scale, ws, stream)
+        if ev is not None:
+            ev[4].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    st = attn.attn_check_status(stream)
+    if st != attn.ATTN_OK:
+        raise RuntimeError(f"device status after warm-up: {attn.attn_status_string(st)}")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank)
+    time.sleep(0.3)
+    t0.record(stream)
+    for s in range(args.steps):
+        step(evs[s])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    if world > 1:
+        dist.barrier()
+    st = attn.attn_check_status(stream)
+    if st != attn.ATTN_OK:
+        raise RuntimeError(f"device status after timed region: {attn.attn_status_string(st)}")
+
+    total_ms = t0.elapsed_time(t1)
+    per_kernel = {"attn_fwd": 0.0, "bwd_pre": 0.0, "bwd_dkdv": 0.0, "bwd_dq": 0.0}
+    for e in evs:
+        per_kernel["attn_fwd"] += e[0].elapsed_time(e[1])
+        per_kernel["bwd_pre"] += e[1].elapsed_time(e[2])
+        per_kernel["bwd_dkdv"] += e[2].elapsed_time(e[3])
+        per_kernel["bwd_dq"] += e[3].elapsed_time(e[4])
+    per_kernel = {kname: t / args.steps for kname, t in per_kernel.items()}
+    t_fwd = per_kernel["attn_fwd"]
+    t_bwd = per_kernel["bwd_pre"] + per_kernel["bwd_dkdv"] + per_kernel["bwd_dq"]
+
+    # max over ranks of the timed-region duration and of the per-kernel means
+    vals = torch.tensor([total_ms, t_fwd, t_bwd] + list(per_kernel.values()), dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    total_ms, t_fwd, t_bwd = float(vals[0]), float(vals[1]), float(vals[2])
+    per_kernel = dict(zip(per_kernel.keys(), [float(x) for x in vals[3:]]))
+    ms_per_step = total_ms / args.steps
+
+    f_fwd = flops_fwd_per_rank(w)
+    value = 3.5 * f_fwd * world / (ms_per_step * 1e-3) / 1e12
+    fwd_tflops = f_fwd * world / (t_fwd * 1e-3) / 1e12
+    fwdbwd_kernel_tflops = 3.5 * f_fwd * world / ((t_fwd + t_bwd) * 1e-3) / 1e12
+
+    peaks, peaks_src = load_peaks()
+    burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+
+    # roofline of the dominant kernel: algorithmic FLOPs per launch (GEMMs on
+    # the causal half of the score matrix: fwd 2, dK/dV 4, dQ 3) over its
+    # CUDA-event mean duration.
+    alg = {"attn_fwd": f_fwd, "bwd_dkdv": 2.0 * f_fwd, "bwd_dq": 1.5 * f_fwd}
+    dom = max(alg, key=lambda kname: per_kernel[kname])
+    achieved = alg[dom] / (per_kernel[dom] * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 1), "peak": sustained,
+                "peak_kind": f"bf16_tflops_sustained ({peaks_src})", "unit": "TFLOP/s",
+                "frac": round(achieved / sustained, 4), "frac_of_burst": round(achieved / burst, 4),
+                "traffic": recorded_traffic(dom)}
+
+    # ---------------------------------------------------------------- e2e
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv, hdo = (t.cpu().pin_memory() for t in (q, k, v, do))
+        ho, hdq, hdk, hdv = (torch.empty(q.shape, dtype=q.dtype).pin_memory() for _ in range(4))
+        hlse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+
+        def e2e_step():
+            for dst, src in ((q, hq), (k, hk), (v, hv), (do, hdo)):
+                dst.copy_(src, non_blocking=True)
+            step()
+            for dst, src in ((ho, o), (hlse, lse), (hdq, dq), (hdk, dk), (hdv, dv)):
+                dst.copy_(src, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        n_e2e = max(3, min(args.steps, 10))
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        e_ms = torch.tensor([a.elapsed_time(b) / n_e2e], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
+        e_ms = float(e_ms)
+        elt = q.element_size()
+        h2d = 4 * q.numel() * elt
+        d2h = 4 * q.numel() * elt + lse.numel() * 4
+        e2e = {"value": round(3.5 * f_fwd * world / (e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms, 3),
+               "steps": n_e2e}
+        assert attn.attn_check_status(stream) == attn.ATTN_OK
+
+    # ------------------------------------------------------- CPU baseline
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline_sample(q[0, 0], k[0, 0], v[0, 0], do[0, 0], w, rows=args.cpu_rows)
+
+    line = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 3),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded N(0, 0.5^2) bf16 Q, K, V, dO; generated on the device)",
+        "config": {"workload": f"{WORKLOAD}: B=8 H=32 N=16384 d=128 causal, fwd+bwd per step",
+                   "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": True, "scale": scale,
+                   "global_batch": w.B * world, "seq_len": w.N, "parallelism": f"dp{world} (heads/batches per rank)",
+                   "l2": "inputs 1 GiB per tensor > 126 MB L2; no flush"},
+        "fwd_tflops": round(fwd_tflops, 2),
+        "fwdbwd_kernel_tflops": round(fwdbwd_kernel_tflops, 2),
+        "pct_of_peak": {
+            "fwd_of_burst": round(fwd_tflops / world / burst, 4),
+            "fwdbwd_of_burst": round(value / world / burst, 4),
+            "fwd_of_sustained": round(fwd_tflops / world / sustained, 4),
+            "fwdbwd_of_sustained": round(value / world / sustained, 4),
+            "fwd_of_datasheet_2250": round(fwd_tflops / world / 2250.0, 4),
+            "fwdbwd_of_datasheet_2250": round(value / world / 2250.0, 4),
+            "peaks": peaks_src,
+        },
+        "kernel_ms": {kname: round(t, 3) for kname, t in per_kernel.items()},
+        "roofline": roofline,
+        "gpu_launches": 4 * args.steps,
+        "clocks": clk,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+        "peak_mem_gib": round(torch.cuda.max_memory_allocated(dev) / 2**30, 3),
+        "naive_score_bytes_per_layer": 2 * w.N * w.N * w.B * w.H,
+    }
+    return line
+
+
+def cpu_baseline_sample(q, k, v, do, w, rows):
+    """The oracle (as it stands) on the exact causal prefix sub-problem of one
+    head: its first ``rows`` queries see only its first ``rows`` keys, so this
+    is a self-contained forward+backward of size ``rows``."""
+    import numpy as np
+    import torch
+
+    from oracle import attn_oracle as orc
+
+    def host(t):
+        return t[:rows].float().cpu().numpy().astype(np.float64)[None]
+
+    Q, K, V, dO = host(q), host(k), host(v), host(do)
+    threads = os.cpu_count()
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([int(i.get("num_threads", 1)) for i in threadpool_info()] + [1])
+    except Exception:
+        pass
+    t = time.perf_counter()
+    orc.attn_fwd(Q, K, V, w.scale, True)
+    orc.attn_bwd(Q, K, V, dO, w.scale, True)
+    dt = time.perf_counter() - t
+    flops = 3.5 * 4.0 * rows * rows * w.d / 2
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "seconds": round(dt, 2),
+            "sample": f"causal prefix of head (0,0): first {rows} query rows and keys, fwd+bwd, fp64 numpy"}
+
+
+def run_reference(args):
+    """The oracle timed on the host cores: --warmup + --steps samples."""
+    import torch
+
+    from exact_io_aware_58_b200.inputs import WORKLOADS, make_inputs
+
+    w = WORKLOADS[WORKLOAD]
+    rows = args.ref_rows
+    inp = make_inputs(1, 1, rows, w.d, seed=1234, std=w.std)
+    q, k, v, do = (inp[n][0, 0] for n in ("Q", "K", "V", "dO"))
+    for _ in range(args.warmup):
+        cpu_baseline_sample(q, k, v, do, w, rows)
+    times = []
+    res = None
+    for _ in range(args.steps):
+        res = cpu_baseline_sample(q, k, v, do, w, rows)
+        times.append(res["seconds"])
+    ms = 1000.0 * sum(times) / len(times)
+    flops = 3.5 * 4.0 * rows * rows * w.d / 2
+    value = flops / (ms * 1e-3) / 1e12
+    return {
+        "impl": "reference",
+        "metric": METRIC,
+        "value": round(value, 6),
+        "unit": "TFLOP/s",
+        "n_gpus": 0,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms, 1),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded N(0, 0.5^2), bf16-rounded, fp64 arithmetic)",
+        "config": {"workload": f"{WORKLOAD}: B=8 H=32 N=16384 d=128 causal, fwd+bwd per step",
+                   "sample": res["sample"] if res else None},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": res["cores"] if res else None,
+                         "kind": "oracle", "sample": res["sample"] if res else None},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=8192)
+    ap.add_argument("--ref-rows", type=int, default=4096)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    if world > 1:
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,217 @@
+"""Thin ctypes binding over libattn.so (the C ABI in include/attn.h).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of libattn.so.  PyTorch supplies device memory and the stream.  If the
+library is missing the import of a compute entry point fails loudly; there is
+no fallback path.
+
+Raw entry points keep the C names and argument order (``attn_fwd``,
+``attn_bwd``, ``attn_bwd_workspace_bytes``, ``attn_check_status``,
+``attn_status_string``); ``forward`` / ``backward`` allocate the outputs with
+torch and call them.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+from .build import LIB_PATH
+
+ATTN_OK = 0
+ATTN_ERR_INVALID_ARG = -1
+ATTN_ERR_UNSUPPORTED = -2
+ATTN_ERR_MISALIGNED = -3
+ATTN_ERR_WORKSPACE = -4
+ATTN_ERR_LAUNCH = -5
+ATTN_ERR_TIMEOUT = -6
+ATTN_ERR_DEVICE = -7
+
+EXPORTED = ("attn_fwd", "attn_bwd", "attn_bwd_workspace_bytes", "attn_bwd_preprocess", "attn_bwd_dkdv",
+            "attn_bwd_dq", "attn_check_status", "attn_status_string")
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {attn_status_string(status)} ({status})")
+
+
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libattn.so and declare the C signatures (once)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"{path} is missing: build it with `python -m exact_io_aware_58_b200.build` "
+            "(nvcc, sm_100a). There is no fallback implementation.")
+    lib = ctypes.CDLL(path)
+    i64, vp, f32, i32 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_float, ctypes.c_int
+    lib.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, f32, vp]
+    lib.attn_fwd.restype = i32
+    lib.attn_bwd_workspace_bytes.argtypes = [i64, i64, i64, i64]
+    lib.attn_bwd_workspace_bytes.restype = ctypes.c_size_t
+    lib.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, f32, vp,
+                             ctypes.c_size_t, vp]
+    lib.attn_bwd.restype = i32
+    lib.attn_bwd_preprocess.argtypes = [vp, vp, vp, i64, i64, i64, i64, vp, ctypes.c_size_t, vp]
+    lib.attn_bwd_preprocess.restype = i32
+    lib.attn_bwd_dkdv.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, f32, vp, ctypes.c_size_t, vp]
+    lib.attn_bwd_dkdv.restype = i32
+    lib.attn_bwd_dq.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, f32, vp, ctypes.c_size_t, vp]
+    lib.attn_bwd_dq.restype = i32
+    lib.attn_check_status.argtypes = [vp]
+    lib.attn_check_status.restype = i32
+    lib.attn_status_string.argtypes = [i32]
+    lib.attn_status_string.restype = ctypes.c_char_p
+    _lib = lib
+    return lib
+
+
+def attn_status_string(status: int) -> str:
+    return load_library().attn_status_string(int(status)).decode()
+
+
+def _stream_handle(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _ptr(t) -> ctypes.c_void_p:
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _check_bhnd(name: str, t: torch.Tensor, shape=None):
+    if not t.is_cuda or t.dtype != torch.bfloat16 or t.dim() != 4 or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor of shape (B, H, N, d)")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _check_lse(t: torch.Tensor, shape):
+    B, H, N, _ = shape
+    if not t.is_cuda or t.dtype != torch.float32 or tuple(t.shape) != (B, H, N) or not t.is_contiguous():
+        raise ValueError("LSE must be a contiguous CUDA float32 tensor of shape (B, H, N)")
+
+
+def attn_fwd(Q, K, V, O, LSE, causal: bool, scale: float, stream=None) -> None:
+    """O, LSE <- attention(Q, K, V); all tensors preallocated on the device."""
+    _check_bhnd("Q", Q)
+    for n, t in (("K", K), ("V", V), ("O", O)):
+        _check_bhnd(n, t, Q.shape)
+    _check_lse(LSE, Q.shape)
+    B, H, N, d = Q.shape
+    st = load_library().attn_fwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE), B, H, N, d, int(bool(causal)),
+                                 float(scale), _stream_handle(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd")
+
+
+def attn_bwd_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    return int(load_library().attn_bwd_workspace_bytes(B, H, N, d))
+
+
+def attn_bwd(Q, K, V, O, dO, LSE, dQ, dK, dV, causal: bool, scale: float, workspace, stream=None) -> None:
+    """dQ, dK, dV <- backward of attention; all tensors preallocated on the device."""
+    _check_bhnd("Q", Q)
+    for n, t in (("K", K), ("V", V), ("O", O), ("dO", dO), ("dQ", dQ), ("dK", dK), ("dV", dV)):
+        _check_bhnd(n, t, Q.shape)
+    _check_lse(LSE, Q.shape)
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    B, H, N, d = Q.shape
+    ws_bytes = workspace.numel() * workspace.element_size()
+    st = load_library().attn_bwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(dO), _ptr(LSE), _ptr(dQ), _ptr(dK),
+                                 _ptr(dV), B, H, N, d, int(bool(causal)), float(scale), _ptr(workspace), ws_bytes,
+                                 _stream_handle(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_bwd")
+
+
+def _ws(workspace):
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    return _ptr(workspace), workspace.numel() * workspace.element_size()
+
+
+def attn_bwd_preprocess(O, dO, LSE, workspace, stream=None) -> None:
+    _check_bhnd("O", O)
+    _check_bhnd("dO", dO, O.shape)
+    _check_lse(LSE, O.shape)
+    B, H, N, d = O.shape
+    wp, wb = _ws(workspace)
+    st = load_library().attn_bwd_preprocess(_ptr(O), _ptr(dO), _ptr(LSE), B, H, N, d, wp, wb,
+                                            _stream_handle(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_bwd_preprocess")
+
+
+def attn_bwd_dkdv(Q, K, V, dO, dK, dV, causal: bool, scale: float, workspace, stream=None) -> None:
+    _check_bhnd("Q", Q)
+    for n, t in (("K", K), ("V", V), ("dO", dO), ("dK", dK), ("dV", dV)):
+        _check_bhnd(n, t, Q.shape)
+    B, H, N, d = Q.shape
+    wp, wb = _ws(workspace)
+    st = load_library().attn_bwd_dkdv(_ptr(Q), _ptr(K), _ptr(V), _ptr(dO), _ptr(dK), _ptr(dV), B, H, N, d,
+                                      int(bool(causal)), float(scale), wp, wb, _stream_handle(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_bwd_dkdv")
+
+
+def attn_bwd_dq(Q, K, V, dO, dQ, causal: bool, scale: float, workspace, stream=None) -> None:
+    _check_bhnd("Q", Q)
+    for n, t in (("K", K), ("V", V), ("dO", dO), ("dQ", dQ)):
+        _check_bhnd(n, t, Q.shape)
+    B, H, N, d = Q.shape
+    wp, wb = _ws(workspace)
+    st = load_library().attn_bwd_dq(_ptr(Q), _ptr(K), _ptr(V), _ptr(dO), _ptr(dQ), B, H, N, d,
+                                    int(bool(causal)), float(scale), wp, wb, _stream_handle(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_bwd_dq")
+
+
+def attn_check_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status code."""
+    return int(load_library().attn_check_status(_stream_handle(stream)))
+
+
+# ---------------------------------------------------------------------------
+# Convenience wrappers: allocate outputs with torch, then call the C ABI.
+# ---------------------------------------------------------------------------
+
+def default_scale(d: int) -> float:
+    return 1.0 / math.sqrt(d)
+
+
+def forward(Q, K, V, causal: bool, scale: float | None = None, stream=None):
+    B, H, N, d = Q.shape
+    scale = default_scale(d) if scale is None else scale
+    O = torch.empty_like(Q)
+    LSE = torch.empty((B, H, N), dtype=torch.float32, device=Q.device)
+    attn_fwd(Q, K, V, O, LSE, causal, scale, stream)
+    return O, LSE
+
+
+def alloc_workspace(B: int, H: int, N: int, d: int, device) -> torch.Tensor:
+    nbytes = attn_bwd_workspace_bytes(B, H, N, d)
+    return torch.empty((max(nbytes, 16) + 15) // 16 * 4, dtype=torch.float32, device=device)
+
+
+def backward(Q, K, V, O, LSE, dO, causal: bool, scale: float | None = None, workspace=None, stream=None):
+    B, H, N, d = Q.shape
+    scale = default_scale(d) if scale is None else scale
+    if workspace is None:
+        workspace = alloc_workspace(B, H, N, d, Q.device)
+    dQ, dK, dV = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
+    attn_bwd(Q, K, V, O, dO, LSE, dQ, dK, dV, causal, scale, workspace, stream)
+    return dQ, dK, dV

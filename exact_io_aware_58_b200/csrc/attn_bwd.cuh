@@ -1,0 +1,611 @@
+// attn_bwd.cuh -- backward by recomputation.
+//
+// Method ("Attention and KV Compression", section "Recomputation in the
+// backward pass"; "FlashAttention -- how 100K-token attention fits in memory",
+// section "Training backward"): the probabilities are not stored by the
+// forward; each score tile is recomputed from Q, K and the saved per-row LSE,
+//   P = exp(scale * Q K^T - LSE),  dP = dO V^T,  dS = P o (dP - D),
+//   D_i = sum_k dO_ik O_ik,  dV = P^T dO,  dQ = scale dS K,  dK = scale dS^T Q.
+//
+// Three kernels:
+//   bwd_pre   per row: D_i and LSE_i*log2(e) into the workspace (HBM-bound).
+//   bwd_dkdv  one CTA per 128-key tile j: Q_i / dO_i tiles stream past a
+//             resident K_j, V_j; S^T and dP^T accumulate in TMEM, P^T and dS^T
+//             are written back into TMEM (bf16) and used as the A operand of
+//             dV += P^T dO_i and dK += dS^T Q_i (4 MMAs per tile pair).
+//   bwd_dq    one CTA per 128-query tile i: K_j / V_j tiles stream past a
+//             resident Q_i, dO_i; S and dP are recomputed, dS goes back to
+//             TMEM and feeds dQ += dS K_j (3 MMAs per tile pair).
+// Q_i, dO_i (and K_j) serve both as K-major operands (for S^T, dP^T) and as
+// MN-major operands (for dK, dV, dQ): one swizzled shared-memory copy, two
+// descriptors.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace attn {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ---------------------------------------------------------------------------
+// bwd_pre: D_i = sum_k dO_ik O_ik, lse2_i = LSE_i * log2(e); padding rows
+// (i >= N, up to Npad) get D = 0 and lse2 = +inf so that recomputed
+// probabilities of padding queries are exactly 0.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(256)
+attn_bwd_pre_kernel(const __nv_bfloat16* __restrict__ O, const __nv_bfloat16* __restrict__ dO,
+                    const float* __restrict__ lse, float* __restrict__ ws_lse2, float* __restrict__ ws_d,
+                    int n, int npad, long long rows_pad) {
+  constexpr int kTpr = D / 8;                 // threads per row, 16 bytes each
+  constexpr int kRowsPerBlock = 256 / kTpr;
+  const int sub = threadIdx.x % kTpr;
+  const long long stride = (long long)gridDim.x * kRowsPerBlock;
+  for (long long row = (long long)blockIdx.x * kRowsPerBlock + threadIdx.x / kTpr; row < rows_pad; row += stride) {
+    const long long bh = row / npad;
+    const int i = int(row - bh * npad);
+    float acc = 0.f;
+    if (i < n) {
+      const size_t off = (size_t(bh) * size_t(n) + size_t(i)) * D + sub * 8;
+      const uint4 a = *reinterpret_cast<const uint4*>(O + off);
+      const uint4 b = *reinterpret_cast<const uint4*>(dO + off);
+      const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a);
+      const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float2 fa = __bfloat1622float2(pa[k]);
+        const float2 fb = __bfloat1622float2(pb[k]);
+        acc = fmaf(fa.x, fb.x, acc);
+        acc = fmaf(fa.y, fb.y, acc);
+      }
+    }
+#pragma unroll
+    for (int o = kTpr / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o, kTpr);
+    if (sub == 0) {
+      ws_d[row] = (i < n) ? acc : 0.f;
+      ws_lse2[row] = (i < n) ? lse[size_t(bh) * size_t(n) + size_t(i)] * kLog2e : INFINITY;
+    }
+  }
+}
+
+struct BwdParams {
+  const float* ws_lse2;   // [BH][npad]
+  const float* ws_d;      // [BH][npad]
+  int n;
+  int npad;
+  int n_tiles;            // ceil(N / 128)
+  float scale;
+  float scale_log2;
+};
+
+template <int D>
+struct BwdCfg {
+  static constexpr int kTileBytes = 128 * D * 2;
+  static constexpr int kBlockBytes = 128 * 128;
+  static constexpr int kNumBlk = D / 64;
+  static constexpr int kStages = (D == 128) ? 2 : 4;
+  static constexpr int kVecBytes = 512;                    // 128 fp32
+  static constexpr int kThreads = 320;
+  static constexpr int kWarpMma = 8;
+  static constexpr int kWarpLoad = 9;
+  static constexpr uint32_t kTmemCols = 512;
+  // dK/dV kernel: resident K_j, V_j; stages of (Q_i, dO_i, lse2_i, D_i).
+  static constexpr int kKV_OffK = 0;
+  static constexpr int kKV_OffV = kTileBytes;
+  static constexpr int kKV_OffStage = 2 * kTileBytes;
+  static constexpr int kKV_StageBytes = 2 * kTileBytes + 2 * kVecBytes;
+  static constexpr int kKV_OffBar = kKV_OffStage + kStages * kKV_StageBytes;
+  // dQ kernel: resident Q_i, dO_i, lse2_i, D_i; stages of (K_j, V_j).
+  static constexpr int kQ_OffQ = 0;
+  static constexpr int kQ_OffDO = kTileBytes;
+  static constexpr int kQ_OffVec = 2 * kTileBytes;
+  static constexpr int kQ_OffStage = 2 * kTileBytes + 1024;
+  static constexpr int kQ_StageBytes = 2 * kTileBytes;
+  static constexpr int kQ_OffBar = kQ_OffStage + kStages * kQ_StageBytes;
+  static constexpr int kNumBars = 2 * kStages + 8;
+  static constexpr int kKV_SmemBytes = kKV_OffBar + kNumBars * 8 + 16 + 1024;
+  static constexpr int kQ_SmemBytes = kQ_OffBar + kNumBars * 8 + 16 + 1024;
+  // TMEM columns
+  static constexpr uint32_t kColA = 0;        // S^T (dkdv) / S (dq)
+  static constexpr uint32_t kColB = 128;      // dP^T (dkdv) / dP (dq)
+  static constexpr uint32_t kColAcc0 = 256;   // dV (dkdv) / dQ (dq)
+  static constexpr uint32_t kColAcc1 = 256 + D;   // dK (dkdv)
+};
+
+// Store a [128 x D] fp32 accumulator held in TMEM (this thread's lane = row r,
+// columns [c_lo, c_hi) in 32-column chunks) as bf16 into a 128B-swizzled
+// shared-memory tile, multiplied by `mul`.
+template <int D>
+__device__ __forceinline__ void tmem_acc_to_smem(uint32_t t_acc_lane, uint32_t stage_u32, int r, int chunk_lo,
+                                                 int chunk_hi, float mul) {
+#pragma unroll 1
+  for (int cc = chunk_lo; cc < chunk_hi; ++cc) {
+    uint32_t o[32];
+    tmem_ld32(t_acc_lane + cc * 32, o);
+    tmem_ld_wait(o);
+    const uint32_t blk = cc >> 1;
+#pragma unroll
+    for (int ch = 0; ch < 4; ++ch) {
+      const uint32_t w0 = pack_bf16x2(__uint_as_float(o[8 * ch + 0]) * mul, __uint_as_float(o[8 * ch + 1]) * mul);
+      const uint32_t w1 = pack_bf16x2(__uint_as_float(o[8 * ch + 2]) * mul, __uint_as_float(o[8 * ch + 3]) * mul);
+      const uint32_t w2 = pack_bf16x2(__uint_as_float(o[8 * ch + 4]) * mul, __uint_as_float(o[8 * ch + 5]) * mul);
+      const uint32_t w3 = pack_bf16x2(__uint_as_float(o[8 * ch + 6]) * mul, __uint_as_float(o[8 * ch + 7]) * mul);
+      const uint32_t chunk = (cc & 1) * 4 + ch;
+      st_shared_v4(stage_u32 + blk * (128 * 128) + sw128_offset(r, chunk), w0, w1, w2, w3);
+    }
+  }
+}
+
+// Load 64 fp32 columns [c0, c0+64) of this thread's TMEM lane.
+__device__ __forceinline__ void tmem_ld64f(uint32_t taddr, float (&v)[64]) {
+  uint32_t a[32], b[32];
+  tmem_ld32(taddr, a);
+  tmem_ld32(taddr + 32, b);
+  tmem_ld_wait(a);
+  reg_fence32(b);
+#pragma unroll
+  for (int k = 0; k < 32; ++k) {
+    v[k] = __uint_as_float(a[k]);
+    v[32 + k] = __uint_as_float(b[k]);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dK, dV
+// ---------------------------------------------------------------------------
+template <int D, bool CAUSAL>
+__global__ void __maxnreg__(200)
+attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                     const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
+                     const BwdParams prm) {
+  using C = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kKV_OffBar);
+  uint64_t* st_full = bars;                    // [kStages]
+  uint64_t* st_empty = st_full + C::kStages;   // [kStages]
+  uint64_t* kv_full = st_empty + C::kStages;
+  uint64_t* s_full = kv_full + 1;
+  uint64_t* dp_full = s_full + 1;
+  uint64_t* p_full = dp_full + 1;
+  uint64_t* ds_full = p_full + 1;
+  uint64_t* acc_full = ds_full + 1;
+  uint64_t* drain = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + C::kNumBars) + 1;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int nt = prm.n_tiles;
+  const int bh = blockIdx.x / nt;
+  const int jt = blockIdx.x % nt;              // key tile; small jt = most work under the causal mask
+  const int n0 = jt * 128;
+  const int i_start = CAUSAL ? jt : 0;
+  const int n_it = nt - i_start;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&st_full[s], 1);
+      mbar_init(&st_empty[s], 1);
+    }
+    mbar_init(kv_full, 1);
+    mbar_init(s_full, 1);
+    mbar_init(dp_full, 1);
+    mbar_init(p_full, 256);
+    mbar_init(ds_full, 256);
+    mbar_init(acc_full, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == C::kWarpMma) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == C::kWarpLoad) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(kv_full, 2 * C::kTileBytes);
+      for (int b = 0; b < C::kNumBlk; ++b) {
+        tma_load_3d(&tm_k, kv_full, smem + C::kKV_OffK + b * C::kBlockBytes, b * 64, n0, bh);
+        tma_load_3d(&tm_v, kv_full, smem + C::kKV_OffV + b * C::kBlockBytes, b * 64, n0, bh);
+      }
+      int issued = 0;
+      for (int it = 0; it < n_it; ++it) {
+        const int slot = it % C::kStages;
+        const int use = it / C::kStages;
+        if (use > 0 && !mbar_wait(&st_empty[slot], (use - 1) & 1, abort_flag)) break;
+        const int qi = i_start + it;
+        uint8_t* st = smem + C::kKV_OffStage + slot * C::kKV_StageBytes;
+        mbar_arrive_expect_tx(&st_full[slot], 2 * C::kTileBytes + 2 * C::kVecBytes);
+        for (int b = 0; b < C::kNumBlk; ++b) {
+          tma_load_3d(&tm_q, &st_full[slot], st + b * C::kBlockBytes, b * 64, qi * 128, bh);
+          tma_load_3d(&tm_do, &st_full[slot], st + C::kTileBytes + b * C::kBlockBytes, b * 64, qi * 128, bh);
+        }
+        const size_t voff = size_t(bh) * size_t(prm.npad) + size_t(qi) * 128;
+        bulk_load(st + 2 * C::kTileBytes, prm.ws_lse2 + voff, C::kVecBytes, &st_full[slot]);
+        bulk_load(st + 2 * C::kTileBytes + C::kVecBytes, prm.ws_d + voff, C::kVecBytes, &st_full[slot]);
+        ++issued;
+      }
+      mbar_wait(kv_full, 0, abort_flag, false);
+      for (int it = max(0, issued - C::kStages); it < issued; ++it)
+        mbar_wait(&st_full[it % C::kStages], (it / C::kStages) & 1, abort_flag, false);
+    }
+    __syncwarp();
+  } else if (warp == C::kWarpMma) {
+    if (lane == 0) {
+      constexpr uint32_t kIdescT = idesc_bf16(128, 128, false, false);   // S^T, dP^T
+      constexpr uint32_t kIdescAcc = idesc_bf16(128, D, false, true);    // dV, dK (B MN-major)
+      const uint32_t sK = smem_u32(smem + C::kKV_OffK);
+      const uint32_t sV = smem_u32(smem + C::kKV_OffV);
+      const uint32_t sSt = smem_u32(smem + C::kKV_OffStage);
+      auto issue_kmajor = [&](uint32_t dcol, uint32_t a0, uint32_t b0) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::kBlockBytes + (kk & 3) * 32;
+          mma_ss(tmem + dcol, smem_desc_sw128(a0 + off, 16, 1024), smem_desc_sw128(b0 + off, 16, 1024), kIdescT,
+                 kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_acc = [&](uint32_t dcol, uint32_t acol, uint32_t b0, bool acc) {
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk)
+          mma_ts(tmem + dcol, tmem + acol + 64 * (kk >> 2) + (kk & 3) * 8,
+                 smem_desc_sw128(b0 + kk * 2048, C::kBlockBytes, 1024), kIdescAcc, (acc || kk > 0) ? 1u : 0u);
+      };
+      auto stage_q = [&](int it) { return sSt + (it % C::kStages) * C::kKV_StageBytes; };
+      auto stage_do = [&](int it) { return sSt + (it % C::kStages) * C::kKV_StageBytes + C::kTileBytes; };
+
+      bool ok = mbar_wait(kv_full, 0, abort_flag);
+      if (ok) ok = mbar_wait(&st_full[0], 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        issue_kmajor(C::kColA, sK, stage_q(0));    // S^T = K_j Q_i^T
+        mma_commit(s_full);
+        issue_kmajor(C::kColB, sV, stage_do(0));   // dP^T = V_j dO_i^T
+        mma_commit(dp_full);
+      }
+      for (int it = 0; it < n_it && ok; ++it) {
+        if (!(ok = mbar_wait(p_full, it & 1, abort_flag))) break;
+        tc_fence_after();
+        issue_acc(C::kColAcc0, C::kColA, stage_do(it), it > 0);   // dV += P^T dO_i
+        const bool more = it + 1 < n_it;
+        if (more) {
+          if (!(ok = mbar_wait(&st_full[(it + 1) % C::kStages], ((it + 1) / C::kStages) & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_kmajor(C::kColA, sK, stage_q(it + 1));
+          mma_commit(s_full);
+        }
+        if (!(ok = mbar_wait(ds_full, it & 1, abort_flag))) break;
+        tc_fence_after();
+        issue_acc(C::kColAcc1, C::kColB, stage_q(it), it > 0);    // dK += dS^T Q_i
+        mma_commit(&st_empty[it % C::kStages]);
+        if (more) {
+          issue_kmajor(C::kColB, sV, stage_do(it + 1));
+          mma_commit(dp_full);
+        }
+      }
+      if (ok) mma_commit(acc_full);
+      mma_commit(drain);
+      mbar_wait(drain, 0, abort_flag, false);
+    }
+    __syncwarp();
+  } else {
+    // compute warps: thread = key row r (TMEM lane), group g = query columns [64g, 64g+64)
+    const int g = warp >> 2;
+    const int qw = warp & 3;
+    const int r = qw * 32 + lane;
+    const int key = n0 + r;
+    const uint32_t lane_base = uint32_t(qw * 32) << 16;
+    const uint32_t tA = tmem + lane_base + C::kColA + 64 * g;
+    const uint32_t tB = tmem + lane_base + C::kColB + 64 * g;
+    const float c = prm.scale_log2;
+    bool ok = true;
+    for (int it = 0; it < n_it; ++it) {
+      const int qi = i_start + it;
+      const float* vec = reinterpret_cast<const float*>(smem + C::kKV_OffStage + (it % C::kStages) * C::kKV_StageBytes +
+                                                        2 * C::kTileBytes);
+      // The stage's LSE/D vectors: wait on the copy's own barrier (already
+      // complete by the time S^T of this stage is; the slot is only refilled
+      // after this iteration's dK MMA, i.e. after these reads).
+      if (!(ok = mbar_wait_warp(&st_full[it % C::kStages], (it / C::kStages) & 1, abort_flag))) break;
+      if (!(ok = mbar_wait_warp(s_full, it & 1, abort_flag))) break;
+      tc_fence_after();
+      float p[64];
+      tmem_ld64f(tA, p);
+      const float4* l4 = reinterpret_cast<const float4*>(vec + 64 * g);
+#pragma unroll
+      for (int k4 = 0; k4 < 16; ++k4) {
+        const float4 lv = l4[k4];
+        p[4 * k4 + 0] = ex2(fmaf(p[4 * k4 + 0], c, -lv.x));
+        p[4 * k4 + 1] = ex2(fmaf(p[4 * k4 + 1], c, -lv.y));
+        p[4 * k4 + 2] = ex2(fmaf(p[4 * k4 + 2], c, -lv.z));
+        p[4 * k4 + 3] = ex2(fmaf(p[4 * k4 + 3], c, -lv.w));
+      }
+      if (CAUSAL && qi == jt) {
+        // query (qi*128 + 64g + k) sees this key only if query >= key
+        const int lim = key - (qi * 128 + 64 * g);   // mask k < lim
+#pragma unroll
+        for (int k = 0; k < 64; ++k)
+          if (k < lim) p[k] = 0.f;
+      }
+      {
+        uint32_t pk[32];
+#pragma unroll
+        for (int k = 0; k < 32; ++k) pk[k] = pack_bf16x2(p[2 * k], p[2 * k + 1]);
+        tmem_st32(tA, pk);   // P^T over the first 32 of this group's 64 S^T columns
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(p_full);
+
+      if (!(ok = mbar_wait_warp(dp_full, it & 1, abort_flag))) break;
+      tc_fence_after();
+      {
+        float dp[64];
+        tmem_ld64f(tB, dp);
+        const float4* d4 = reinterpret_cast<const float4*>(vec + 128 + 64 * g);
+        uint32_t pk[32];
+#pragma unroll
+        for (int k4 = 0; k4 < 16; ++k4) {
+          const float4 dv = d4[k4];
+          const float s0 = p[4 * k4 + 0] * (dp[4 * k4 + 0] - dv.x);
+          const float s1 = p[4 * k4 + 1] * (dp[4 * k4 + 1] - dv.y);
+          const float s2 = p[4 * k4 + 2] * (dp[4 * k4 + 2] - dv.z);
+          const float s3 = p[4 * k4 + 3] * (dp[4 * k4 + 3] - dv.w);
+          pk[2 * k4] = pack_bf16x2(s0, s1);
+          pk[2 * k4 + 1] = pack_bf16x2(s2, s3);
+        }
+        tmem_st32(tB, pk);   // dS^T over the first 32 of this group's 64 dP^T columns
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(ds_full);
+    }
+    (void)key;
+    // epilogue: group 0 writes dV (into the K_j... V_j slot), group 1 writes dK (into the K_j slot)
+    if (ok) ok = mbar_wait_warp(acc_full, 0, abort_flag);
+    uint8_t* stage = smem + (g == 0 ? C::kKV_OffV : C::kKV_OffK);
+    if (ok) {
+      tc_fence_after();
+      tmem_acc_to_smem<D>(tmem + lane_base + (g == 0 ? C::kColAcc0 : C::kColAcc1), smem_u32(stage), r, 0, D / 32,
+                          g == 0 ? 1.f : prm.scale);
+    }
+    fence_proxy_async_smem();
+    named_barrier_sync(1 + g, 128);
+    if (qw == 0 && lane == 0 && *abort_flag == 0) {
+      const CUtensorMap* tm = (g == 0) ? &tm_dv : &tm_dk;
+      for (int b = 0; b < C::kNumBlk; ++b) tma_store_3d(tm, stage + b * C::kBlockBytes, b * 64, n0, bh);
+      bulk_commit_group();
+      bulk_wait_group_read0();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == C::kWarpMma) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// dQ
+// ---------------------------------------------------------------------------
+template <int D, bool CAUSAL>
+__global__ void __maxnreg__(200)
+attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                   const __grid_constant__ CUtensorMap tm_dq, const BwdParams prm) {
+  using C = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kQ_OffBar);
+  uint64_t* st_full = bars;
+  uint64_t* st_empty = st_full + C::kStages;
+  uint64_t* q_full = st_empty + C::kStages;
+  uint64_t* s_full = q_full + 1;
+  uint64_t* s_free = s_full + 1;
+  uint64_t* dp_full = s_free + 1;
+  uint64_t* ds_full = dp_full + 1;
+  uint64_t* acc_full = ds_full + 1;
+  uint64_t* drain = acc_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + C::kNumBars) + 1;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n = prm.n;
+  const int nt = prm.n_tiles;
+  const int bh = blockIdx.x / nt;
+  const int it_q = nt - 1 - (blockIdx.x % nt);   // query tile; large = most work under the causal mask
+  const int m0 = it_q * 128;
+  const int n_it = CAUSAL ? it_q + 1 : nt;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&st_full[s], 1);
+      mbar_init(&st_empty[s], 1);
+    }
+    mbar_init(q_full, 1);
+    mbar_init(s_full, 1);
+    mbar_init(s_free, 256);
+    mbar_init(dp_full, 1);
+    mbar_init(ds_full, 256);
+    mbar_init(acc_full, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == C::kWarpMma) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == C::kWarpLoad) {
+    if (lane == 0) {
+      mbar_arrive_expect_tx(q_full, 2 * C::kTileBytes + 2 * C::kVecBytes);
+      for (int b = 0; b < C::kNumBlk; ++b) {
+        tma_load_3d(&tm_q, q_full, smem + C::kQ_OffQ + b * C::kBlockBytes, b * 64, m0, bh);
+        tma_load_3d(&tm_do, q_full, smem + C::kQ_OffDO + b * C::kBlockBytes, b * 64, m0, bh);
+      }
+      const size_t voff = size_t(bh) * size_t(prm.npad) + size_t(m0);
+      bulk_load(smem + C::kQ_OffVec, prm.ws_lse2 + voff, C::kVecBytes, q_full);
+      bulk_load(smem + C::kQ_OffVec + C::kVecBytes, prm.ws_d + voff, C::kVecBytes, q_full);
+      int issued = 0;
+      for (int it = 0; it < n_it; ++it) {
+        const int slot = it % C::kStages;
+        const int use = it / C::kStages;
+        if (use > 0 && !mbar_wait(&st_empty[slot], (use - 1) & 1, abort_flag)) break;
+        uint8_t* st = smem + C::kQ_OffStage + slot * C::kQ_StageBytes;
+        mbar_arrive_expect_tx(&st_full[slot], 2 * C::kTileBytes);
+        for (int b = 0; b < C::kNumBlk; ++b) {
+          tma_load_3d(&tm_k, &st_full[slot], st + b * C::kBlockBytes, b * 64, it * 128, bh);
+          tma_load_3d(&tm_v, &st_full[slot], st + C::kTileBytes + b * C::kBlockBytes, b * 64, it * 128, bh);
+        }
+        ++issued;
+      }
+      mbar_wait(q_full, 0, abort_flag, false);
+      for (int it = max(0, issued - C::kStages); it < issued; ++it)
+        mbar_wait(&st_full[it % C::kStages], (it / C::kStages) & 1, abort_flag, false);
+    }
+    __syncwarp();
+  } else if (warp == C::kWarpMma) {
+    if (lane == 0) {
+      constexpr uint32_t kIdescS = idesc_bf16(128, 128, false, false);
+      constexpr uint32_t kIdescAcc = idesc_bf16(128, D, false, true);
+      const uint32_t sQ = smem_u32(smem + C::kQ_OffQ);
+      const uint32_t sDO = smem_u32(smem + C::kQ_OffDO);
+      const uint32_t sSt = smem_u32(smem + C::kQ_OffStage);
+      auto issue_kmajor = [&](uint32_t dcol, uint32_t a0, uint32_t b0) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::kBlockBytes + (kk & 3) * 32;
+          mma_ss(tmem + dcol, smem_desc_sw128(a0 + off, 16, 1024), smem_desc_sw128(b0 + off, 16, 1024), kIdescS,
+                 kk > 0 ? 1u : 0u);
+        }
+      };
+      auto stage_k = [&](int it) { return sSt + (it % C::kStages) * C::kQ_StageBytes; };
+      auto stage_v = [&](int it) { return sSt + (it % C::kStages) * C::kQ_StageBytes + C::kTileBytes; };
+
+      bool ok = mbar_wait(q_full, 0, abort_flag);
+      if (ok) ok = mbar_wait(&st_full[0], 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        issue_kmajor(C::kColA, sQ, stage_k(0));    // S = Q_i K_j^T
+        mma_commit(s_full);
+        issue_kmajor(C::kColB, sDO, stage_v(0));   // dP = dO_i V_j^T
+        mma_commit(dp_full);
+      }
+      for (int it = 0; it < n_it && ok; ++it) {
+        const bool more = it + 1 < n_it;
+        if (more) {
+          if (!(ok = mbar_wait(&st_full[(it + 1) % C::kStages], ((it + 1) / C::kStages) & 1, abort_flag))) break;
+          if (!(ok = mbar_wait(s_free, it & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_kmajor(C::kColA, sQ, stage_k(it + 1));
+          mma_commit(s_full);
+        }
+        if (!(ok = mbar_wait(ds_full, it & 1, abort_flag))) break;
+        tc_fence_after();
+        // dQ += dS K_j: A = dS in TMEM (over dP columns), B = K_j MN-major
+        const uint32_t bk = stage_k(it);
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk)
+          mma_ts(tmem + C::kColAcc0, tmem + C::kColB + 64 * (kk >> 2) + (kk & 3) * 8,
+                 smem_desc_sw128(bk + kk * 2048, C::kBlockBytes, 1024), kIdescAcc, (it > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&st_empty[it % C::kStages]);
+        if (more) {
+          issue_kmajor(C::kColB, sDO, stage_v(it + 1));
+          mma_commit(dp_full);
+        }
+      }
+      if (ok) mma_commit(acc_full);
+      mma_commit(drain);
+      mbar_wait(drain, 0, abort_flag, false);
+    }
+    __syncwarp();
+  } else {
+    // compute warps: thread = query row r, group g = key columns [64g, 64g+64)
+    const int g = warp >> 2;
+    const int qw = warp & 3;
+    const int r = qw * 32 + lane;
+    const int row = m0 + r;
+    const uint32_t lane_base = uint32_t(qw * 32) << 16;
+    const uint32_t tA = tmem + lane_base + C::kColA + 64 * g;
+    const uint32_t tB = tmem + lane_base + C::kColB + 64 * g;
+    const float c = prm.scale_log2;
+    bool ok = mbar_wait_warp(q_full, 0, abort_flag);
+    const float* vec = reinterpret_cast<const float*>(smem + C::kQ_OffVec);
+    const float neg_lse2 = ok ? -vec[r] : 0.f;
+    const float dval = ok ? vec[128 + r] : 0.f;
+    for (int it = 0; it < n_it && ok; ++it) {
+      if (!(ok = mbar_wait_warp(s_full, it & 1, abort_flag))) break;
+      tc_fence_after();
+      float p[64];
+      tmem_ld64f(tA, p);
+      tc_fence_before();
+      mbar_arrive(s_free);
+#pragma unroll
+      for (int k = 0; k < 64; ++k) p[k] = ex2(fmaf(p[k], c, neg_lse2));
+      const int kbase = it * 128 + 64 * g;
+      const bool need_mask = (CAUSAL && it == it_q) || (kbase + 64 > n);
+      if (need_mask) {
+        int lim = n - 1 - kbase;                 // keep k <= lim
+        if (CAUSAL) lim = min(lim, row - kbase);
+#pragma unroll
+        for (int k = 0; k < 64; ++k)
+          if (k > lim) p[k] = 0.f;
+      }
+      if (!(ok = mbar_wait_warp(dp_full, it & 1, abort_flag))) break;
+      tc_fence_after();
+      {
+        float dp[64];
+        tmem_ld64f(tB, dp);
+        uint32_t pk[32];
+#pragma unroll
+        for (int k = 0; k < 32; ++k)
+          pk[k] = pack_bf16x2(p[2 * k] * (dp[2 * k] - dval), p[2 * k + 1] * (dp[2 * k + 1] - dval));
+        tmem_st32(tB, pk);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(ds_full);
+    }
+    if (ok) ok = mbar_wait_warp(acc_full, 0, abort_flag);
+    uint8_t* stage = smem + C::kQ_OffQ;   // Q_i is no longer read
+    if (ok) {
+      tc_fence_after();
+      constexpr int kChunks = D / 32;
+      tmem_acc_to_smem<D>(tmem + lane_base + C::kColAcc0, smem_u32(stage), r, g * kChunks / 2, (g + 1) * kChunks / 2,
+                          prm.scale);
+    }
+    fence_proxy_async_smem();
+    named_barrier_sync(1, 256);
+    if (warp == 0 && lane == 0 && *abort_flag == 0) {
+      for (int b = 0; b < C::kNumBlk; ++b) tma_store_3d(&tm_dq, stage + b * C::kBlockBytes, b * 64, m0, bh);
+      bulk_commit_group();
+      bulk_wait_group_read0();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == C::kWarpMma) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+}  // namespace attn

@@ -1,0 +1,364 @@
+// attn_fwd.cuh -- forward kernel: tiled exact attention with online softmax.
+//
+// Method ("Attention and KV Compression", section "Tiling and online softmax";
+// "FlashAttention -- how 100K-token attention fits in memory", sections
+// "FlashAttention idea" and "Online softmax intuition"): a block of query rows
+// stays on chip while blocks of keys and values stream past it; for each key
+// block the scores are formed on chip, a running row max m and row sum l are
+// kept, the partial output is rescaled by exp(m_old - m_new) when the max
+// grows, and only O and one statistic per row (LSE) are written out.
+//
+// B200 mapping (one CTA = two 128-row query tiles of one head, 320 threads):
+//   warp 9      TMA producer: Q0, Q1 once, then K_j / V_j 128-row tiles into a
+//               ring of shared-memory slots (128-byte swizzle).
+//   warp 8      MMA issuer (one thread): S_t = Q_t K_j^T and O_t += P_t V_j as
+//               tcgen05.mma with fp32 accumulators in tensor memory (TMEM).
+//   warps 0-3   softmax for query tile 0, warps 4-7 for tile 1: each thread owns
+//               one query row (= one TMEM lane), so the row max and sum need no
+//               shuffles.  P is rounded to bf16 and written back into TMEM over
+//               the upper half of S, where the PV MMA reads it as its A operand.
+// The issue order PV_t(j-1), S_t(j) lets the tensor core run one tile's GEMMs
+// while the other tile's softmax runs (ping-pong between the two tiles).
+//
+// Rescaling is lazy but exact: the reference max m_ref used in the exponent is
+// only moved when a tile's max exceeds it by more than kRescaleLog2 (2^8); O
+// and l always share the same m_ref, so O = acc / l is unchanged, and LSE is
+// computed from the same pair.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace attn {
+
+constexpr float kRescaleLog2 = 8.0f;
+constexpr float kLn2 = 0.6931471805599453f;
+
+struct FwdParams {
+  float* lse;          // [BH][N] natural-log LSE
+  int n;               // sequence length N
+  int n_mblk;          // number of 256-row query blocks per head
+  float scale_log2;    // scale * log2(e)
+};
+
+template <int D>
+struct FwdCfg {
+  static constexpr int kTileBytes = 128 * D * 2;        // one 128 x D bf16 tile
+  static constexpr int kBlockBytes = 128 * 128;          // one [128][64] bf16 column block
+  static constexpr int kNumBlk = D / 64;
+  static constexpr int kSlots = (D == 128) ? 4 : 8;      // K/V ring depth
+  static constexpr int kThreads = 320;
+  static constexpr int kWarpMma = 8;
+  static constexpr int kWarpLoad = 9;
+  static constexpr uint32_t kTmemCols = 512;
+  static constexpr uint32_t kColS0 = 0, kColS1 = 128;
+  static constexpr uint32_t kColO0 = 256, kColO1 = 256 + D;
+  static constexpr uint32_t kColPOff = 64;               // P (bf16 pairs) over S columns 64..127
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffKV = 2 * kTileBytes;
+  static constexpr int kOffBar = kOffKV + kSlots * kTileBytes;
+  static constexpr int kNumBars = 2 + 2 * kSlots + 2 + 2 + 2 + 1;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;   // + slack for 1024-byte alignment
+};
+
+template <int D, bool CAUSAL>
+__global__ void __maxnreg__(200)
+attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                const FwdParams prm) {
+  using C = FwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
+  uint64_t* q_full = bars;
+  uint64_t* kv_full = q_full + 2;
+  uint64_t* kv_empty = kv_full + C::kSlots;
+  uint64_t* s_full = kv_empty + C::kSlots;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* o_full = p_full + 2;
+  uint64_t* drain = o_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n = prm.n;
+  const int bh = blockIdx.x / prm.n_mblk;
+  const int m_blk = prm.n_mblk - 1 - (blockIdx.x % prm.n_mblk);   // heaviest causal blocks first
+  const int m0 = m_blk * 256;
+  const int n_kv_total = (n + 127) >> 7;
+  const int nkv = CAUSAL ? min(n_kv_total, (m0 >> 7) + 2) : n_kv_total;
+
+  if (threadIdx.x == 0) {
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&q_full[t], 1);
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_full[t], 128);
+      mbar_init(&o_full[t], 1);
+    }
+    for (int s = 0; s < C::kSlots; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == C::kWarpMma) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == C::kWarpLoad && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_k);
+    tma_prefetch_desc(&tm_v);
+    tma_prefetch_desc(&tm_o);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == C::kWarpLoad) {
+    // ------------------------------------------------------------------ TMA
+    if (lane == 0) {
+      for (int t = 0; t < 2; ++t) {
+        mbar_arrive_expect_tx(&q_full[t], C::kTileBytes);
+        for (int b = 0; b < C::kNumBlk; ++b)
+          tma_load_3d(&tm_q, &q_full[t], smem + C::kOffQ + t * C::kTileBytes + b * C::kBlockBytes,
+                      b * 64, m0 + 128 * t, bh);
+      }
+      int issued = 0;
+      bool ok = true;
+      for (int it = 0; it < 2 * nkv; ++it) {
+        const int slot = it % C::kSlots;
+        const int use = it / C::kSlots;
+        if (use > 0 && !mbar_wait(&kv_empty[slot], (use - 1) & 1, abort_flag)) { ok = false; break; }
+        const CUtensorMap* tm = (it & 1) ? &tm_v : &tm_k;
+        const int j = it >> 1;
+        mbar_arrive_expect_tx(&kv_full[slot], C::kTileBytes);
+        for (int b = 0; b < C::kNumBlk; ++b)
+          tma_load_3d(tm, &kv_full[slot], smem + C::kOffKV + slot * C::kTileBytes + b * C::kBlockBytes,
+                      b * 64, 128 * j, bh);
+        ++issued;
+      }
+      (void)ok;
+      // No copy may still be landing in shared memory when the CTA leaves.
+      mbar_wait(&q_full[0], 0, abort_flag, false);
+      mbar_wait(&q_full[1], 0, abort_flag, false);
+      for (int it = max(0, issued - C::kSlots); it < issued; ++it)
+        mbar_wait(&kv_full[it % C::kSlots], (it / C::kSlots) & 1, abort_flag, false);
+    }
+    __syncwarp();
+  } else if (warp == C::kWarpMma) {
+    // ------------------------------------------------------------------ MMA
+    if (lane == 0) {
+      constexpr uint32_t kIdescS = idesc_bf16(128, 128, false, false);
+      constexpr uint32_t kIdescPV = idesc_bf16(128, D, false, true);
+      const uint32_t sQ = smem_u32(smem + C::kOffQ);
+      const uint32_t sKV = smem_u32(smem + C::kOffKV);
+      int it = 0;
+      auto wait_kv = [&](int& slot) -> bool {
+        slot = it % C::kSlots;
+        const bool r = mbar_wait(&kv_full[slot], (it / C::kSlots) & 1, abort_flag);
+        ++it;
+        return r;
+      };
+      auto issue_s = [&](int t, int kslot) {
+        const uint32_t a0 = sQ + t * C::kTileBytes;
+        const uint32_t b0 = sKV + kslot * C::kTileBytes;
+        const uint32_t dt = tmem + (t ? C::kColS1 : C::kColS0);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::kBlockBytes + (kk & 3) * 32;
+          mma_ss(dt, smem_desc_sw128(a0 + off, 16, 1024), smem_desc_sw128(b0 + off, 16, 1024), kIdescS,
+                 kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int t, int vslot, bool acc) {
+        const uint32_t b0 = sKV + vslot * C::kTileBytes;
+        const uint32_t dt = tmem + (t ? C::kColO1 : C::kColO0);
+        const uint32_t at = tmem + (t ? C::kColS1 : C::kColS0) + C::kColPOff;
+#pragma unroll
+        for (int kk = 0; kk < 128 / 16; ++kk)
+          mma_ts(dt, at + kk * 8, smem_desc_sw128(b0 + kk * 2048, C::kBlockBytes, 1024), kIdescPV,
+                 (acc || kk > 0) ? 1u : 0u);
+      };
+
+      bool ok = mbar_wait(&q_full[0], 0, abort_flag) && mbar_wait(&q_full[1], 0, abort_flag);
+      if (ok) {
+        int ks;
+        ok = wait_kv(ks);
+        if (ok) {
+          tc_fence_after();
+          issue_s(0, ks);
+          mma_commit(&s_full[0]);
+          issue_s(1, ks);
+          mma_commit(&s_full[1]);
+          mma_commit(&kv_empty[ks]);
+        }
+      }
+      for (int j = 1; j < nkv && ok; ++j) {
+        int vs, ks;
+        if (!(ok = wait_kv(vs))) break;
+        if (!(ok = wait_kv(ks))) break;
+        for (int t = 0; t < 2; ++t) {
+          if (!(ok = mbar_wait(&p_full[t], (j - 1) & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_pv(t, vs, j - 1 > 0);
+          if (t == 1) mma_commit(&kv_empty[vs]);
+          issue_s(t, ks);
+          mma_commit(&s_full[t]);
+        }
+        if (ok) mma_commit(&kv_empty[ks]);
+      }
+      if (ok) {
+        int vs;
+        ok = wait_kv(vs);
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (!(ok = mbar_wait(&p_full[t], (nkv - 1) & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_pv(t, vs, nkv - 1 > 0);
+          mma_commit(&o_full[t]);
+        }
+        if (ok) mma_commit(&kv_empty[vs]);
+      }
+      // Every MMA issued so far must finish before tensor memory is released.
+      mma_commit(drain);
+      mbar_wait(drain, 0, abort_flag, false);
+    }
+    __syncwarp();
+  } else {
+    // -------------------------------------------------------------- softmax
+    const int t = warp >> 2;
+    const int qw = warp & 3;
+    const int r = qw * 32 + lane;           // row inside the tile = TMEM lane
+    const int i = m0 + 128 * t + r;         // global query row
+    const uint32_t lane_base = uint32_t(qw * 32) << 16;
+    const uint32_t tS = tmem + lane_base + (t ? C::kColS1 : C::kColS0);
+    const uint32_t tP = tS + C::kColPOff;
+    const uint32_t tO = tmem + lane_base + (t ? C::kColO1 : C::kColO0);
+    const float c = prm.scale_log2;
+    float m_ref = -INFINITY;
+    float l = 0.f;
+    bool ok = true;
+
+    for (int j = 0; j < nkv; ++j) {
+      if (!(ok = mbar_wait_warp(&s_full[t], j & 1, abort_flag))) break;
+      tc_fence_after();
+      float s[128];
+      {
+        uint32_t a[32], b[32], e[32], f[32];
+        tmem_ld32(tS + 0, a);
+        tmem_ld32(tS + 32, b);
+        tmem_ld32(tS + 64, e);
+        tmem_ld32(tS + 96, f);
+        tmem_ld_wait(a);
+        reg_fence32(b);
+        reg_fence32(e);
+        reg_fence32(f);
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+          s[k] = __uint_as_float(a[k]);
+          s[32 + k] = __uint_as_float(b[k]);
+          s[64 + k] = __uint_as_float(e[k]);
+          s[96 + k] = __uint_as_float(f[k]);
+        }
+      }
+      const bool need_mask = (CAUSAL && (128 * j + 127 > m0 + 128 * t)) || (128 * j + 128 > n);
+      if (need_mask) {
+        int limit = n - 1 - 128 * j;
+        if (CAUSAL) limit = min(limit, i - 128 * j);
+#pragma unroll
+        for (int k = 0; k < 128; ++k)
+          if (k > limit) s[k] = -INFINITY;
+      }
+      float mx = s[0];
+#pragma unroll
+      for (int k = 1; k < 128; ++k) mx = fmaxf(mx, s[k]);
+      const float m_tile = mx * c;
+      float alpha = 1.f;
+      bool rescale = false;
+      if (m_tile > m_ref + kRescaleLog2) {
+        alpha = ex2(m_ref - m_tile);      // 0 when m_ref is still -inf
+        m_ref = m_tile;
+        rescale = (j > 0);
+      }
+      l *= alpha;
+      const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
+      float rowsum = 0.f;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+          const float p0 = ex2(fmaf(s[h * 64 + 2 * k], c, neg_m));
+          const float p1 = ex2(fmaf(s[h * 64 + 2 * k + 1], c, neg_m));
+          rowsum += p0 + p1;
+          pk[k] = pack_bf16x2(p0, p1);
+        }
+        tmem_st32(tP + h * 32, pk);
+      }
+      l += rowsum;
+      if (__any_sync(0xffffffffu, rescale)) {
+        // O_t holds the sum through key tile j-1 (its last PV completed before S_t(j)).
+        const float a = rescale ? alpha : 1.f;
+#pragma unroll 1
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(tO + cc * 32, o);
+          tmem_ld_wait(o);
+#pragma unroll
+          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * a);
+          tmem_st32(tO + cc * 32, o);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&p_full[t]);
+    }
+
+    // ------------------------------------------------------------ epilogue
+    if (ok) ok = mbar_wait_warp(&o_full[t], 0, abort_flag);
+    uint8_t* stage = smem + C::kOffQ + t * C::kTileBytes;   // Q_t is no longer read
+    if (ok) {
+      tc_fence_after();
+      const float inv_l = 1.f / l;
+#pragma unroll 1
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t o[32];
+        tmem_ld32(tO + cc * 32, o);
+        tmem_ld_wait(o);
+        const uint32_t blk = cc >> 1;
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          const uint32_t w0 = pack_bf16x2(__uint_as_float(o[8 * ch + 0]) * inv_l, __uint_as_float(o[8 * ch + 1]) * inv_l);
+          const uint32_t w1 = pack_bf16x2(__uint_as_float(o[8 * ch + 2]) * inv_l, __uint_as_float(o[8 * ch + 3]) * inv_l);
+          const uint32_t w2 = pack_bf16x2(__uint_as_float(o[8 * ch + 4]) * inv_l, __uint_as_float(o[8 * ch + 5]) * inv_l);
+          const uint32_t w3 = pack_bf16x2(__uint_as_float(o[8 * ch + 6]) * inv_l, __uint_as_float(o[8 * ch + 7]) * inv_l);
+          const uint32_t chunk = (cc & 1) * 4 + ch;
+          st_shared_v4(smem_u32(stage) + blk * C::kBlockBytes + sw128_offset(r, chunk), w0, w1, w2, w3);
+        }
+      }
+      if (i < n) prm.lse[size_t(bh) * size_t(n) + size_t(i)] = (m_ref + __log2f(l)) * kLn2;
+    }
+    fence_proxy_async_smem();
+    named_barrier_sync(1 + t, 128);
+    // A store never starts past the last row (rows past N inside a box are dropped by TMA).
+    if (qw == 0 && lane == 0 && *abort_flag == 0 && m0 + 128 * t < n) {
+      for (int b = 0; b < C::kNumBlk; ++b) tma_store_3d(&tm_o, stage + b * C::kBlockBytes, b * 64, m0 + 128 * t, bh);
+      bulk_commit_group();
+      bulk_wait_group_read0();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == C::kWarpMma) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+}  // namespace attn

@@ -3,9 +3,11 @@
 This module only draws random numbers and describes workload shapes; it holds
 none of the attention arithmetic.  Recipe (the same for every workload):
 
-* ``torch.Generator('cpu').manual_seed(seed)``, then ``torch.randn`` in
+* ``torch.Generator(device).manual_seed(seed)``, then ``torch.randn`` in
   float32 in the order Q, K, V, dO, each of shape (B, H, N, d), each
-  multiplied by ``std``;
+  multiplied by ``std``.  ``device`` is "cpu" by default; the largest
+  workloads draw on the GPU (CPU ``randn`` needs ~30 s per 2^29 values), and
+  the oracle is then given a host copy of exactly those bf16 tensors;
 * optionally a fraction of query rows is multiplied by ``outlier_mult``
   (rows drawn without replacement by a generator seeded ``seed + 1``), to
   stress the running-max rescaling of online softmax;
@@ -84,22 +86,22 @@ def sample_rows(B: int, H: int, N: int, count: int, seed: int) -> torch.Tensor:
 
 def make_inputs(B: int, H: int, N: int, d: int, seed: int = 0, std: float = 1.0,
                 with_dO: bool = True, outlier_frac: float = 0.0,
-                outlier_mult: float = 8.0) -> dict:
-    """Q, K, V (and dO) as contiguous bf16 CPU tensors of shape (B, H, N, d)."""
-    g = torch.Generator("cpu").manual_seed(seed)
+                outlier_mult: float = 8.0, device="cpu") -> dict:
+    """Q, K, V (and dO) as contiguous bf16 tensors of shape (B, H, N, d) on ``device``."""
+    g = torch.Generator(device).manual_seed(seed)
     names = ["Q", "K", "V"] + (["dO"] if with_dO else [])
     out = {}
     for name in names:
-        x = torch.randn((B, H, N, d), generator=g, dtype=torch.float32)
+        x = torch.randn((B, H, N, d), generator=g, dtype=torch.float32, device=device)
         if std != 1.0:
             x.mul_(std)
         if name == "Q" and outlier_frac > 0:
-            rows = outlier_rows(B, H, N, outlier_frac, seed)
+            rows = outlier_rows(B, H, N, outlier_frac, seed).to(x.device)
             x.view(-1, d)[rows] *= outlier_mult
         out[name] = x.to(torch.bfloat16).contiguous()
     return out
 
 
-def workload_inputs(w: Workload, seed: int = 0) -> dict:
+def workload_inputs(w: Workload, seed: int = 0, device="cpu") -> dict:
     return make_inputs(w.B, w.H, w.N, w.d, seed=seed, std=w.std, with_dO=w.with_dO,
-                       outlier_frac=w.outlier_frac, outlier_mult=w.outlier_mult)
+                       outlier_frac=w.outlier_frac, outlier_mult=w.outlier_mult, device=device)

@@ -1,0 +1,142 @@
+/*
+ * attn.h -- C ABI of libattn.so: exact, IO-aware tiled softmax attention on
+ * NVIDIA B200 (sm_100a), forward and backward.
+ *
+ * What is computed (per batch b and head h, rows indexed 0..N-1):
+ *
+ *   S = scale * Q K^T,  S_ij = -inf for j > i when causal,
+ *   P = rowwise softmax(S),  O = P V,  LSE_i = ln sum_j exp(S_ij).
+ *
+ * The result is the dense softmax attention of the standard four-step
+ * computation (score, mask, softmax, weight -- "FlashAttention" flagship
+ * module, Beat 01), reached tile by tile: a Q block stays on chip while K/V
+ * blocks stream past it, and an online softmax keeps a running row max and
+ * row sum and rescales the accumulator when the max grows ("Attention and KV
+ * Compression", section "Tiling and online softmax"; "FlashAttention -- how
+ * 100K-token attention fits in memory", sections "FlashAttention idea" and
+ * "Online softmax intuition").  Only O and one statistic per row (LSE) are
+ * written to device memory; no N x N buffer exists at any point.  The
+ * backward recomputes score tiles from Q, K, V and LSE instead of storing P
+ * ("Attention and KV Compression", section "Recomputation in the backward
+ * pass").
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Layout "BHND": contiguous [B][H][N][d] bfloat16 (row stride d elements).
+ *    Q, K, V, O, dO, dQ, dK, dV all use it.  LSE is fp32 [B][H][N], natural log.
+ *  - d must be 64 or 128 (otherwise ATTN_ERR_UNSUPPORTED).  N >= 1 is any
+ *    value; partial tiles are handled.  B, H >= 1.  B*H and N must each fit
+ *    in 31 bits.
+ *  - scale must be finite and > 0 (otherwise ATTN_ERR_INVALID_ARG).
+ *  - Every pointer is a DEVICE pointer owned by the caller; the library keeps
+ *    no reference after the call returns and never allocates device memory.
+ *    Every pointer must be 16-byte aligned (ATTN_ERR_MISALIGNED otherwise).
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  All work is
+ *    enqueued asynchronously on it; the call returns once it is enqueued.
+ *  - Argument errors are reported synchronously, before anything is launched.
+ *    A launch failure returns ATTN_ERR_LAUNCH.  Device-side waits are bounded:
+ *    a wait that runs out sets a device status word that attn_check_status
+ *    reports as ATTN_ERR_TIMEOUT (the kernel then releases its tensor memory
+ *    and returns; its outputs are undefined).  The library never traps,
+ *    aborts or prints.
+ */
+#ifndef EXACT_ATTN_B200_ATTN_H
+#define EXACT_ATTN_B200_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = -1,
+  ATTN_ERR_UNSUPPORTED = -2,
+  ATTN_ERR_MISALIGNED = -3,
+  ATTN_ERR_WORKSPACE = -4,
+  ATTN_ERR_LAUNCH = -5,
+  ATTN_ERR_TIMEOUT = -6,
+  ATTN_ERR_DEVICE = -7
+} attn_status_t;
+
+/*
+ * Forward pass.  Reads Q, K, V; writes O (bf16, BHND) and LSE (fp32 [B][H][N]).
+ * Tiled exact attention with online softmax ("Attention and KV Compression",
+ * section "Tiling and online softmax").  O and LSE must not alias the inputs.
+ */
+int attn_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE,
+             int64_t B, int64_t H, int64_t N, int64_t d, int causal, float scale,
+             void* stream);
+
+/*
+ * Bytes of caller-provided device workspace that attn_bwd needs for these
+ * sizes (two fp32 per-row vectors per head, each padded to a multiple of 128
+ * rows).  Returns 0 for sizes that attn_bwd would reject.
+ */
+size_t attn_bwd_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d);
+
+/*
+ * Backward pass by recomputation ("Attention and KV Compression", section
+ * "Recomputation in the backward pass"; "FlashAttention -- how 100K-token
+ * attention fits in memory", section "Training backward").
+ * Inputs: Q, K, V, the forward's O and LSE, and the output gradient dO.
+ * Outputs: dQ, dK, dV (bf16, BHND).  Three kernels run on `stream`:
+ *   (1) per row, D_i = sum_k dO_ik O_ik and LSE_i * log2(e), into `workspace`;
+ *   (2) per 128-key tile, dK and dV (score tiles recomputed, 4 MMAs per tile pair);
+ *   (3) per 128-query tile, dQ (score tiles recomputed, 3 MMAs per tile pair).
+ * `workspace` (device, 16-byte aligned) must hold attn_bwd_workspace_bytes()
+ * bytes, else ATTN_ERR_WORKSPACE; its layout after the call is
+ * [B*H][Npad] fp32 LSE*log2(e) (padding rows +inf) followed by
+ * [B*H][Npad] fp32 D (padding rows 0), Npad = N rounded up to 128.
+ * Outputs must not alias inputs or the workspace.
+ */
+int attn_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+             const float* LSE, void* dQ, void* dK, void* dV,
+             int64_t B, int64_t H, int64_t N, int64_t d, int causal, float scale,
+             void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * The three steps of attn_bwd, callable one at a time (same arguments and
+ * rules as attn_bwd; attn_bwd is exactly these three calls in this order on
+ * one stream).  Useful to time the steps separately or to run dK/dV and dQ on
+ * different streams once the preprocess step has completed.
+ *
+ * attn_bwd_preprocess: per row, D_i = sum_k dO_ik O_ik and LSE_i*log2(e)
+ *   into `workspace` (layout as for attn_bwd).  D is the row term of the
+ *   softmax gradient dS = P o (dP - D) ("Attention and KV Compression",
+ *   section "Recomputation in the backward pass": only the small per-row
+ *   statistics are kept from the forward).
+ * attn_bwd_dkdv: dK and dV, one CTA per 128-key tile; reads the workspace.
+ * attn_bwd_dq: dQ, one CTA per 128-query tile; reads the workspace.
+ */
+int attn_bwd_preprocess(const void* O, const void* dO, const float* LSE,
+                        int64_t B, int64_t H, int64_t N, int64_t d,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+int attn_bwd_dkdv(const void* Q, const void* K, const void* V, const void* dO,
+                  void* dK, void* dV,
+                  int64_t B, int64_t H, int64_t N, int64_t d, int causal, float scale,
+                  const void* workspace, size_t workspace_bytes, void* stream);
+
+int attn_bwd_dq(const void* Q, const void* K, const void* V, const void* dO, void* dQ,
+                int64_t B, int64_t H, int64_t N, int64_t d, int causal, float scale,
+                const void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Synchronises `stream`, then reports and clears the device status word:
+ * ATTN_OK, ATTN_ERR_TIMEOUT (a bounded device-side wait ran out in some
+ * kernel since the last check), or ATTN_ERR_DEVICE (the CUDA context reports
+ * an error).
+ */
+int attn_check_status(void* stream);
+
+/* Static, human-readable name of a status code. */
+const char* attn_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* EXACT_ATTN_B200_ATTN_H */

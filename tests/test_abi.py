@@ -1,0 +1,105 @@
+"""The C-ABI library builds, loads without a GPU, exports every symbol that
+include/attn.h declares, and rejects bad arguments before launching anything."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from exact_io_aware_58_b200 import attn, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "attn.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(attn_[a-z_0-9]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return attn.load_library()
+
+
+def test_header_declares_the_abi():
+    assert _declared_functions() == sorted(attn.EXPORTED)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+    # and nothing internal leaks out under the attn_ prefix
+    out = os.popen(f"nm -D --defined-only {build.LIB_PATH}").read()
+    exported = sorted(set(re.findall(r"\bT (attn_[a-z_0-9]+)\b", out)))
+    assert exported == _declared_functions()
+
+
+def test_status_strings(lib):
+    for code, name in [(0, "ATTN_OK"), (-1, "ATTN_ERR_INVALID_ARG"), (-2, "ATTN_ERR_UNSUPPORTED"),
+                       (-3, "ATTN_ERR_MISALIGNED"), (-4, "ATTN_ERR_WORKSPACE"), (-5, "ATTN_ERR_LAUNCH"),
+                       (-6, "ATTN_ERR_TIMEOUT"), (-7, "ATTN_ERR_DEVICE")]:
+        assert attn.attn_status_string(code) == name
+    assert attn.attn_status_string(42) == "ATTN_ERR_UNKNOWN"
+
+
+def test_workspace_bytes(lib):
+    # two fp32 vectors per head, rows padded to a multiple of 128
+    assert attn.attn_bwd_workspace_bytes(1, 2, 256, 64) == 2 * 4 * 2 * 256
+    assert attn.attn_bwd_workspace_bytes(8, 32, 16384, 128) == 2 * 4 * 256 * 16384
+    assert attn.attn_bwd_workspace_bytes(1, 8, 100000, 128) == 2 * 4 * 8 * 100096
+    assert attn.attn_bwd_workspace_bytes(1, 1, 1, 64) == 2 * 4 * 128
+    assert attn.attn_bwd_workspace_bytes(1, 1, 1, 96) == 0       # unsupported d
+    assert attn.attn_bwd_workspace_bytes(0, 1, 1, 64) == 0
+
+
+# Fake, never-dereferenced device addresses: argument checks happen before any
+# CUDA call, so these return synchronously without a GPU.
+A = ctypes.c_void_p(0x100000)
+MIS = ctypes.c_void_p(0x100008)
+
+
+def _fwd(lib, B=1, H=1, N=128, d=64, scale=0.125, ptrs=None):
+    p = ptrs or [A] * 5
+    return lib.attn_fwd(*p, B, H, N, d, 0, scale, None)
+
+
+def test_fwd_argument_errors(lib):
+    assert _fwd(lib, N=0) == attn.ATTN_ERR_INVALID_ARG
+    assert _fwd(lib, B=0) == attn.ATTN_ERR_INVALID_ARG
+    assert _fwd(lib, d=96) == attn.ATTN_ERR_UNSUPPORTED
+    assert _fwd(lib, d=256) == attn.ATTN_ERR_UNSUPPORTED
+    assert _fwd(lib, scale=0.0) == attn.ATTN_ERR_INVALID_ARG
+    assert _fwd(lib, scale=float("nan")) == attn.ATTN_ERR_INVALID_ARG
+    assert _fwd(lib, scale=-1.0) == attn.ATTN_ERR_INVALID_ARG
+    assert _fwd(lib, ptrs=[A, A, None, A, A]) == attn.ATTN_ERR_INVALID_ARG
+    for k in range(5):
+        p = [A] * 5
+        p[k] = MIS
+        assert _fwd(lib, ptrs=p) == attn.ATTN_ERR_MISALIGNED
+
+
+def test_bwd_argument_errors(lib):
+    ws = attn.attn_bwd_workspace_bytes(1, 1, 128, 64)
+
+    def bwd(ptrs=None, ws_ptr=A, ws_bytes=ws, d=64):
+        p = ptrs or [A] * 9
+        return lib.attn_bwd(*p, 1, 1, 128, d, 1, 0.125, ws_ptr, ws_bytes, None)
+
+    assert bwd(ws_bytes=ws - 4) == attn.ATTN_ERR_WORKSPACE
+    assert bwd(ws_ptr=None) == attn.ATTN_ERR_INVALID_ARG
+    assert bwd(ws_ptr=MIS) == attn.ATTN_ERR_MISALIGNED
+    assert bwd(d=32) == attn.ATTN_ERR_UNSUPPORTED
+    for k in range(9):
+        p = [A] * 9
+        p[k] = MIS
+        assert bwd(ptrs=p) == attn.ATTN_ERR_MISALIGNED
+
+
+def test_python_binding_validates_tensors():
+    import torch
+    q = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        attn.attn_fwd(q, q, q, q, torch.zeros(1, 1, 8), False, 0.125)

@@ -1,0 +1,226 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the
+same seeded bf16 inputs.  Every hot-path step is covered: the forward (Q-tile
+load, K/V streaming, QK^T, masking + online softmax, rescale, PV, epilogue)
+through O and LSE; bwd_pre through the workspace's D and LSE*log2(e)
+vectors; bwd_dkdv and bwd_dq through dK, dV and dQ.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from exact_io_aware_58_b200 import attn
+from exact_io_aware_58_b200.inputs import WORKLOADS, make_inputs, sample_rows, workload_inputs
+from oracle import attn_oracle as orc
+
+from ._parity import assert_grad, assert_lse, assert_o, f64
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+def _run(inp, causal, scale, with_bwd):
+    q, k, v = (inp[n].to(DEV) for n in ("Q", "K", "V"))
+    for n in list(inp):
+        inp[n] = inp[n].cpu()        # the oracle reads host copies of the same bf16 values
+    o, lse = attn.forward(q, k, v, causal, scale)
+    out = {"O": o, "LSE": lse}
+    if with_bwd:
+        do = inp["dO"].to(DEV)
+        B, H, N, d = q.shape
+        ws = attn.alloc_workspace(B, H, N, d, q.device)
+        dq, dk, dv = attn.backward(q, k, v, o, lse, do, causal, scale, workspace=ws)
+        out.update(dQ=dq, dK=dk, dV=dv, ws=ws)
+    assert attn.attn_check_status() == attn.ATTN_OK
+    return out
+
+
+def _check_full(inp, out, causal, scale, with_bwd, heads=None):
+    N, d = inp["Q"].shape[2], inp["Q"].shape[3]
+    Q, K, V = (f64(inp[n]) for n in ("Q", "K", "V"))
+    sel = slice(None) if heads is None else heads
+    O_ref, L_ref = orc.attn_fwd(Q[sel], K[sel], V[sel], scale, causal)
+    assert_o(f64(out["O"])[sel], O_ref)
+    assert_lse(f64(out["LSE"])[sel], L_ref)
+    if with_bwd:
+        dO = f64(inp["dO"])
+        dQ_ref, dK_ref, dV_ref = orc.attn_bwd(Q[sel], K[sel], V[sel], dO[sel], scale, causal)
+        assert_grad(f64(out["dQ"])[sel], dQ_ref, "dQ")
+        assert_grad(f64(out["dK"])[sel], dK_ref, "dK")
+        assert_grad(f64(out["dV"])[sel], dV_ref, "dV")
+
+
+# ---------------------------------------------------------------------------
+# Small shapes: several tiles and ragged tails, both head dims, both masks
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [1, 7, 64, 127, 128, 129, 255, 256, 300, 513])
+def test_small_shapes_fwd_bwd(N, d, causal):
+    inp = make_inputs(1, 2, N, d, seed=1000 + N + d)
+    scale = 1.0 / math.sqrt(d)
+    out = _run(inp, causal, scale, True)
+    _check_full(inp, out, causal, scale, True)
+
+
+def test_workspace_vectors_bwd_pre():
+    """bwd_pre: D_i = sum_k dO_ik O_ik and LSE_i*log2(e), padded rows +inf / 0."""
+    B, H, N, d = 1, 3, 200, 128
+    inp = make_inputs(B, H, N, d, seed=7)
+    scale = 1.0 / math.sqrt(d)
+    out = _run(inp, True, scale, True)
+    npad = 256
+    ws = out["ws"].view(-1)[: 2 * B * H * npad].cpu().numpy().astype(np.float64)
+    lse2, Dv = ws[: B * H * npad].reshape(B * H, npad), ws[B * H * npad:].reshape(B * H, npad)
+    Q, K, V, dO = (f64(inp[n]) for n in ("Q", "K", "V", "dO"))
+    O_ref, L_ref = orc.attn_fwd(Q, K, V, scale, True)
+    np.testing.assert_allclose(lse2[:, :N], L_ref * math.log2(math.e), rtol=0, atol=2e-3)
+    assert np.isinf(lse2[:, N:]).all() and (lse2[:, N:] > 0).all()
+    D_ref = np.sum(O_ref * dO, axis=-1)
+    assert np.abs(Dv[:, :N] - D_ref).max() <= 2e-2 * np.abs(D_ref).max()
+    assert (Dv[:, N:] == 0).all()
+
+
+# ---------------------------------------------------------------------------
+# The five workloads
+# ---------------------------------------------------------------------------
+
+def test_tiny_fwd_bwd():
+    w = WORKLOADS["tiny"]
+    inp = workload_inputs(w)
+    out = _run(inp, False, w.scale, True)
+    _check_full(inp, out, False, w.scale, True)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_fwd_outliers_full(causal):
+    w = WORKLOADS["fwd_outliers"]
+    inp = workload_inputs(w)
+    out = _run(inp, causal, w.scale, False)
+    _check_full(inp, out, causal, w.scale, False)
+
+
+def test_train_d64():
+    w = WORKLOADS["train_d64"]
+    inp = workload_inputs(w)
+    out = _run(inp, True, w.scale, True)
+    # forward on every head, backward on 6 seeded heads
+    Q, K, V = (f64(inp[n]) for n in ("Q", "K", "V"))
+    O_ref, L_ref = orc.attn_fwd(Q, K, V, w.scale, True)
+    assert_o(f64(out["O"]), O_ref)
+    assert_lse(f64(out["LSE"]), L_ref)
+    heads = np.sort(np.random.default_rng(3).choice(w.B * w.H, 6, replace=False))
+    _check_full(inp, out, True, w.scale, True, heads=heads)
+
+
+@pytest.mark.slow
+def test_long_batch_sampled():
+    w = WORKLOADS["long_batch"]
+    inp = workload_inputs(w, device=DEV)
+    out = _run(inp, True, w.scale, True)
+    BH = w.B * w.H
+    # two full heads, forward and backward
+    heads = np.sort(np.random.default_rng(4).choice(BH, 2, replace=False))
+    _check_full(inp, out, True, w.scale, True, heads=heads)
+    # 512 sampled rows of O and LSE across all heads
+    _check_sampled_rows(inp, out, w, 512)
+
+
+def _check_sampled_rows(inp, out, w, count):
+    rows = sample_rows(w.B, w.H, w.N, count, 0).numpy()
+    bh, i = rows // w.N, rows % w.N
+    O = out["O"].view(-1, w.N, w.d)
+    LSE = out["LSE"].view(-1, w.N)
+    Qh, Kh, Vh = (inp[n].view(-1, w.N, w.d) for n in ("Q", "K", "V"))
+    for h in np.unique(bh):
+        sel = i[bh == h]
+        q = Qh[h].float().numpy().astype(np.float64)
+        k = Kh[h].float().numpy().astype(np.float64)
+        v = Vh[h].float().numpy().astype(np.float64)
+        o_ref, l_ref = orc.attn_fwd_rows(q, k, v, w.scale, True, sel)
+        assert_o(O[h, torch.as_tensor(sel)].float().cpu().numpy().astype(np.float64), o_ref)
+        assert_lse(LSE[h, torch.as_tensor(sel)].cpu().numpy().astype(np.float64), l_ref)
+
+
+@pytest.mark.slow
+def test_long_context_sampled_no_quadratic_memory():
+    w = WORKLOADS["long_context"]
+    inp = workload_inputs(w, device=DEV)
+    q, k, v = (inp[n] for n in ("Q", "K", "V"))
+    inp = {n: t.cpu() for n, t in inp.items()}
+    o = torch.empty_like(q)
+    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=DEV)
+    torch.cuda.synchronize()
+    torch.cuda.reset_peak_memory_stats()
+    base_alloc = torch.cuda.memory_allocated()
+    free0, _ = torch.cuda.mem_get_info()
+    attn.attn_fwd(q, k, v, o, lse, True, w.scale)
+    assert attn.attn_check_status() == attn.ATTN_OK
+    free1, _ = torch.cuda.mem_get_info()
+    # nothing is allocated by the call: no N x N buffer (20 GB per head if materialised)
+    assert torch.cuda.max_memory_allocated() - base_alloc == 0
+    assert free0 - free1 < 64 * 2**20
+    _check_sampled_rows(inp, {"O": o, "LSE": lse}, w, w.check_rows)
+
+
+# ---------------------------------------------------------------------------
+# Closed forms on the GPU (no oracle involved)
+# ---------------------------------------------------------------------------
+
+def test_worked_example_on_gpu():
+    """Scores [1, 2, 3] in the first key tile and 4 in the second (the pages'
+    online-softmax example): the result equals the one-shot softmax of those
+    four scores.  Integer scores are exact in bf16; V is one-hot."""
+    N, d = 256, 64
+    Q = torch.zeros(1, 1, N, d)
+    K = torch.zeros(1, 1, N, d)
+    V = torch.zeros(1, 1, N, d)
+    row = 200
+    Q[0, 0, row, 0] = 1.0
+    K[0, 0, :, 0] = -60.0
+    keys = {0: 1.0, 1: 2.0, 2: 3.0, 129: 4.0}
+    for slot, (j, s) in enumerate(keys.items()):
+        K[0, 0, j, 0] = s
+        V[0, 0, j, slot] = 1.0
+    q, k, v = (x.to(torch.bfloat16).to(DEV) for x in (Q, K, V))
+    o, lse = attn.forward(q, k, v, True, 1.0)
+    assert attn.attn_check_status() == attn.ATTN_OK
+    sc = list(keys.values())
+    z = math.fsum(math.exp(s) for s in sc)
+    p = [math.exp(s) / z for s in sc]
+    got = o[0, 0, row, :4].float().cpu().numpy()
+    np.testing.assert_allclose(got, p, rtol=0, atol=4e-3)    # bf16 output
+    assert abs(float(lse[0, 0, row]) - math.log(z)) < 1e-4
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_equal_keys_give_mean_of_visible_values(causal):
+    N, d = 300, 128
+    g = torch.Generator().manual_seed(11)
+    Q = torch.randn(1, 2, N, d, generator=g)
+    K = torch.randn(1, 2, 1, d, generator=g).expand(1, 2, N, d).contiguous()
+    V = torch.randn(1, 2, N, d, generator=g)
+    q, k, v = (x.to(torch.bfloat16).to(DEV) for x in (Q, K, V))
+    o, _ = attn.forward(q, k, v, causal, 0.1)
+    vb = v.float().cpu()
+    if causal:
+        ref = torch.cumsum(vb, dim=2) / torch.arange(1, N + 1).view(1, 1, N, 1)
+    else:
+        ref = vb.mean(dim=2, keepdim=True).expand_as(vb)
+    assert_o(f64(o), f64(ref))
+
+
+def test_status_and_argument_errors_on_gpu():
+    q = torch.zeros(1, 1, 64, 64, dtype=torch.bfloat16, device=DEV)
+    lse = torch.zeros(1, 1, 64, dtype=torch.float32, device=DEV)
+    lib = attn.load_library()
+    import ctypes
+    bad = ctypes.c_void_p(q.data_ptr() + 2)
+    p = ctypes.c_void_p(q.data_ptr())
+    st = lib.attn_fwd(bad, p, p, p, ctypes.c_void_p(lse.data_ptr()), 1, 1, 64, 64, 0, 0.125, None)
+    assert st == attn.ATTN_ERR_MISALIGNED
+    assert attn.attn_check_status() == attn.ATTN_OK

@@ -131,15 +131,20 @@ def run_ours(args, rank, world, local_rank):
 
     from exact_io_aware_58_b200 import attn
     from exact_io_aware_58_b200.inputs import WORKLOADS, workload_inputs
+    from exact_io_aware_58_b200.multi import aggregate_tflops, max_over_ranks, rank_seed
 
     w = WORKLOADS[WORKLOAD]
+    if args.batch or args.heads or args.seq:
+        # smaller cases of the same kernels, for profiler captures only
+        import dataclasses
+        w = dataclasses.replace(w, B=args.batch or w.B, H=args.heads or w.H, N=args.seq or w.N)
     causal = True
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     attn.load_library()
     stream = torch.cuda.current_stream()
 
-    inp = workload_inputs(w, seed=1234 + rank, device=dev)
+    inp = workload_inputs(w, seed=rank_seed(1234, rank), device=dev)
     q, k, v, do = inp["Q"], inp["K"], inp["V"], inp["dO"]
     o = torch.empty_like(q)
     lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
@@ -200,17 +205,15 @@ def run_ours(args, rank, world, local_rank):
     t_bwd = per_kernel["bwd_pre"] + per_kernel["bwd_dkdv"] + per_kernel["bwd_dq"]
 
     # max over ranks of the timed-region duration and of the per-kernel means
-    vals = torch.tensor([total_ms, t_fwd, t_bwd] + list(per_kernel.values()), dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    total_ms, t_fwd, t_bwd = float(vals[0]), float(vals[1]), float(vals[2])
-    per_kernel = dict(zip(per_kernel.keys(), [float(x) for x in vals[3:]]))
+    vals = max_over_ranks([total_ms, t_fwd, t_bwd] + list(per_kernel.values()), device=dev)
+    total_ms, t_fwd, t_bwd = vals[0], vals[1], vals[2]
+    per_kernel = dict(zip(per_kernel.keys(), vals[3:]))
     ms_per_step = total_ms / args.steps
 
     f_fwd = flops_fwd_per_rank(w)
-    value = 3.5 * f_fwd * world / (ms_per_step * 1e-3) / 1e12
-    fwd_tflops = f_fwd * world / (t_fwd * 1e-3) / 1e12
-    fwdbwd_kernel_tflops = 3.5 * f_fwd * world / ((t_fwd + t_bwd) * 1e-3) / 1e12
+    value = aggregate_tflops(3.5 * f_fwd, world, ms_per_step)
+    fwd_tflops = aggregate_tflops(f_fwd, world, t_fwd)
+    fwdbwd_kernel_tflops = aggregate_tflops(3.5 * f_fwd, world, t_fwd + t_bwd)
 
     peaks, peaks_src = load_peaks()
     burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
@@ -253,14 +256,11 @@ def run_ours(args, rank, world, local_rank):
             e2e_step()
         b.record(stream)
         torch.cuda.synchronize()
-        e_ms = torch.tensor([a.elapsed_time(b) / n_e2e], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(e_ms, op=dist.ReduceOp.MAX)
-        e_ms = float(e_ms)
+        e_ms = max_over_ranks([a.elapsed_time(b) / n_e2e], device=dev)[0]
         elt = q.element_size()
         h2d = 4 * q.numel() * elt
         d2h = 4 * q.numel() * elt + lse.numel() * 4
-        e2e = {"value": round(3.5 * f_fwd * world / (e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+        e2e = {"value": round(aggregate_tflops(3.5 * f_fwd, world, e_ms), 2), "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms, 3),
                "steps": n_e2e}
         assert attn.attn_check_status(stream) == attn.ATTN_OK
@@ -283,7 +283,7 @@ def run_ours(args, rank, world, local_rank):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic (seeded N(0, 0.5^2) bf16 Q, K, V, dO; generated on the device)",
-        "config": {"workload": f"{WORKLOAD}: B=8 H=32 N=16384 d=128 causal, fwd+bwd per step",
+        "config": {"workload": f"{WORKLOAD}: B={w.B} H={w.H} N={w.N} d={w.d} causal, fwd+bwd per step",
                    "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": True, "scale": scale,
                    "global_batch": w.B * world, "seq_len": w.N, "parallelism": f"dp{world} (heads/batches per rank)",
                    "l2": "inputs 1 GiB per tensor > 126 MB L2; no flush"},
@@ -373,7 +373,7 @@ def run_reference(args):
         "vs_baseline": None,
         "dtype": "f64",
         "data": "synthetic (seeded N(0, 0.5^2), bf16-rounded, fp64 arithmetic)",
-        "config": {"workload": f"{WORKLOAD}: B=8 H=32 N=16384 d=128 causal, fwd+bwd per step",
+        "config": {"workload": f"{WORKLOAD}: B={w.B} H={w.H} N={w.N} d={w.d} causal, fwd+bwd per step",
                    "sample": res["sample"] if res else None},
         "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": res["cores"] if res else None,
                          "kind": "oracle", "sample": res["sample"] if res else None},
@@ -391,6 +391,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=8192)
     ap.add_argument("--ref-rows", type=int, default=4096)
+    ap.add_argument("--batch", type=int, default=0, help="override B (profiling captures only)")
+    ap.add_argument("--heads", type=int, default=0, help="override H (profiling captures only)")
+    ap.add_argument("--seq", type=int, default=0, help="override N (profiling captures only)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

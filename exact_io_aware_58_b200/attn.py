@@ -31,13 +31,14 @@ ATTN_ERR_TIMEOUT = -6
 ATTN_ERR_DEVICE = -7
 
 EXPORTED = ("attn_fwd", "attn_bwd", "attn_bwd_workspace_bytes", "attn_bwd_preprocess", "attn_bwd_dkdv",
-            "attn_bwd_dq", "attn_check_status", "attn_status_string")
+            "attn_bwd_dq", "attn_check_status", "attn_last_error", "attn_status_string")
 
 
 class AttnError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {attn_status_string(status)} ({status})")
+        detail = attn_last_error()
+        super().__init__(f"{where}: {attn_status_string(status)} ({status})" + (f": {detail}" if detail else ""))
 
 
 _lib = None
@@ -69,6 +70,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.attn_bwd_dq.restype = i32
     lib.attn_check_status.argtypes = [vp]
     lib.attn_check_status.restype = i32
+    lib.attn_last_error.argtypes = []
+    lib.attn_last_error.restype = ctypes.c_char_p
     lib.attn_status_string.argtypes = [i32]
     lib.attn_status_string.restype = ctypes.c_char_p
     _lib = lib
@@ -77,6 +80,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
 
 def attn_status_string(status: int) -> str:
     return load_library().attn_status_string(int(status)).decode()
+
+
+def attn_last_error() -> str:
+    return load_library().attn_last_error().decode()
 
 
 def _stream_handle(stream) -> ctypes.c_void_p:

@@ -8,6 +8,7 @@
 
 #include <cmath>
 #include <cstdint>
+#include <cstdio>
 #include <mutex>
 
 #include <cuda.h>
@@ -18,6 +19,14 @@
 #include "attn_fwd.cuh"
 
 namespace {
+
+// Detail of the most recent failure on this host thread (attn_last_error).
+thread_local char g_last_error[256] = "";
+
+int fail(int status, const char* fmt, const char* a = "", long long b = 0) {
+  std::snprintf(g_last_error, sizeof(g_last_error), fmt, a, b);
+  return status;
+}
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -41,14 +50,22 @@ EncodeTiledFn encode_fn() {
 // past N are dropped.
 bool make_map(CUtensorMap* m, const void* base, int64_t bh, int64_t n, int64_t d) {
   EncodeTiledFn enc = encode_fn();
-  if (!enc) return false;
+  if (!enc) {
+    fail(ATTN_ERR_LAUNCH, "%sdriver entry point cuTensorMapEncodeTiled unavailable%lld", "", 0);
+    return false;
+  }
   const cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(n), cuuint64_t(bh)};
   const cuuint64_t strides[2] = {cuuint64_t(d * 2), cuuint64_t(n * d * 2)};
   const cuuint32_t box[3] = {64, 128, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    fail(ATTN_ERR_LAUNCH, "%scuTensorMapEncodeTiled returned CUresult %lld", "", (long long)r);
+    return false;
+  }
+  return true;
 }
 
 bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -65,15 +82,25 @@ int check_sizes(int64_t B, int64_t H, int64_t N, int64_t d) {
 
 int check_scale(float scale) { return (std::isfinite(scale) && scale > 0.f) ? ATTN_OK : ATTN_ERR_INVALID_ARG; }
 
-int launch_status() { return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_LAUNCH; }
+int launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) return ATTN_OK;
+  return fail(ATTN_ERR_LAUNCH, "kernel launch: %s (%lld)", cudaGetErrorString(e), (long long)e);
+}
+
+int set_smem(const void* kern, int bytes) {
+  const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) return ATTN_OK;
+  return fail(ATTN_ERR_LAUNCH, "cudaFuncSetAttribute(max dynamic smem): %s (bytes %lld)", cudaGetErrorString(e),
+              (long long)bytes);
+}
 
 template <int D, bool CAUSAL>
 int launch_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const CUtensorMap& o,
                const attn::FwdParams& prm, int grid, cudaStream_t st) {
   auto kern = attn::attn_fwd_kernel<D, CAUSAL>;
   constexpr int smem = attn::FwdCfg<D>::kSmemBytes;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-    return ATTN_ERR_LAUNCH;
+  if (set_smem(reinterpret_cast<const void*>(kern), smem) != ATTN_OK) return ATTN_ERR_LAUNCH;
   kern<<<grid, attn::FwdCfg<D>::kThreads, smem, st>>>(q, k, v, o, prm);
   return launch_status();
 }
@@ -83,8 +110,7 @@ int launch_dkdv(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v
                 const CUtensorMap& dk, const CUtensorMap& dv, const attn::BwdParams& prm, int grid, cudaStream_t st) {
   using C = attn::BwdCfg<D>;
   auto kern = attn::attn_bwd_dkdv_kernel<D, CAUSAL>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kKV_SmemBytes) != cudaSuccess)
-    return ATTN_ERR_LAUNCH;
+  if (set_smem(reinterpret_cast<const void*>(kern), C::kKV_SmemBytes) != ATTN_OK) return ATTN_ERR_LAUNCH;
   kern<<<grid, C::kThreads, C::kKV_SmemBytes, st>>>(q, k, v, dO, dk, dv, prm);
   return launch_status();
 }
@@ -94,8 +120,7 @@ int launch_dq(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, 
               const CUtensorMap& dq, const attn::BwdParams& prm, int grid, cudaStream_t st) {
   using C = attn::BwdCfg<D>;
   auto kern = attn::attn_bwd_dq_kernel<D, CAUSAL>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kQ_SmemBytes) != cudaSuccess)
-    return ATTN_ERR_LAUNCH;
+  if (set_smem(reinterpret_cast<const void*>(kern), C::kQ_SmemBytes) != ATTN_OK) return ATTN_ERR_LAUNCH;
   kern<<<grid, C::kThreads, C::kQ_SmemBytes, st>>>(q, k, v, dO, dq, prm);
   return launch_status();
 }
@@ -281,6 +306,8 @@ ATTN_EXPORT int attn_check_status(void* stream) {
   }
   return ATTN_OK;
 }
+
+ATTN_EXPORT const char* attn_last_error(void) { return g_last_error; }
 
 ATTN_EXPORT const char* attn_status_string(int status) {
   switch (status) {

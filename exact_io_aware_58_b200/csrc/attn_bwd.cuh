@@ -154,7 +154,7 @@ __device__ __forceinline__ void tmem_ld64f(uint32_t taddr, float (&v)[64]) {
 // dK, dV
 // ---------------------------------------------------------------------------
 template <int D, bool CAUSAL>
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(320, 1)
 attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                      const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
@@ -399,7 +399,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
 // dQ
 // ---------------------------------------------------------------------------
 template <int D, bool CAUSAL>
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(320, 1)
 attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                    const __grid_constant__ CUtensorMap tm_dq, const BwdParams prm) {

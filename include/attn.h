@@ -132,6 +132,13 @@ int attn_bwd_dq(const void* Q, const void* K, const void* V, const void* dO, voi
  */
 int attn_check_status(void* stream);
 
+/*
+ * Detail of the most recent failure reported by an entry point on the calling
+ * host thread (which CUDA call failed and its error), or "" if none.  The
+ * string is owned by the library and valid until the next call on the thread.
+ */
+const char* attn_last_error(void);
+
 /* Static, human-readable name of a status code. */
 const char* attn_status_string(int status);
 

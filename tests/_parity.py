@@ -6,7 +6,10 @@ Tolerances (bf16 inputs, fp32 accumulation):
           already 0.0156 for |O| in [4, 8), so a bare 1e-2 bound cannot hold for
           any bf16 output there.  The extra term is exactly that rounding.
   * LSE:  max |LSE - LSE_ref| <= 1e-3 (fp32 output).
-  * dQ, dK, dV: max |g - g_ref| <= 2e-2 * max |g_ref| per tensor.
+  * dQ, dK, dV: max |g - g_ref| <= 2e-2 * max |g_ref| + 1e-5 per tensor.
+          The 1e-5 floor only matters where the reference is identically zero:
+          with N = 1, dS = P (dP - D) vanishes in exact arithmetic, but the
+          kernel's D comes from the bf16 O, so its dS, and dQ, dK, are ~1e-7.
 """
 
 from __future__ import annotations
@@ -17,6 +20,7 @@ import torch
 O_TOL = 1e-2
 LSE_TOL = 1e-3
 GRAD_REL = 2e-2
+GRAD_ABS_FLOOR = 1e-5
 
 
 def f64(t: torch.Tensor, n: int | None = None, d: int | None = None) -> np.ndarray:
@@ -57,4 +61,5 @@ def assert_grad(g: np.ndarray, g_ref: np.ndarray, what: str):
     assert np.isfinite(g).all(), f"{what}: non-finite values"
     ref_max = float(np.abs(g_ref).max())
     mx = float(np.abs(g - g_ref).max())
-    assert mx <= GRAD_REL * max(ref_max, 1e-30), f"{what}: max err {mx:.3e} > {GRAD_REL} * {ref_max:.3e}"
+    assert mx <= GRAD_REL * ref_max + GRAD_ABS_FLOOR, \
+        f"{what}: max err {mx:.3e} > {GRAD_REL} * {ref_max:.3e} + {GRAD_ABS_FLOOR}"

@@ -389,8 +389,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-rows", type=int, default=8192)
-    ap.add_argument("--ref-rows", type=int, default=4096)
+    ap.add_argument("--cpu-rows", type=int, default=16384)
+    ap.add_argument("--ref-rows", type=int, default=8192)
     ap.add_argument("--batch", type=int, default=0, help="override B (profiling captures only)")
     ap.add_argument("--heads", type=int, default=0, help="override H (profiling captures only)")
     ap.add_argument("--seq", type=int, default=0, help="override N (profiling captures only)")

@@ -31,7 +31,11 @@ ATTN_ERR_TIMEOUT = -6
 ATTN_ERR_DEVICE = -7
 
 EXPORTED = ("attn_fwd", "attn_bwd", "attn_bwd_workspace_bytes", "attn_bwd_preprocess", "attn_bwd_dkdv",
-            "attn_bwd_dq", "attn_check_status", "attn_last_error", "attn_status_string")
+            "attn_bwd_dq", "attn_bwd_static_workspace", "attn_check_status", "attn_last_error",
+            "attn_status_string")
+
+# Size of the library-owned workspace used by attn_bwd_static_workspace (bytes).
+ATTN_STATIC_WORKSPACE_BYTES = 32 * 1024 * 1024
 
 
 class AttnError(RuntimeError):
@@ -68,6 +72,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.attn_bwd_dkdv.restype = i32
     lib.attn_bwd_dq.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, f32, vp, ctypes.c_size_t, vp]
     lib.attn_bwd_dq.restype = i32
+    lib.attn_bwd_static_workspace.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, f32, vp]
+    lib.attn_bwd_static_workspace.restype = i32
     lib.attn_check_status.argtypes = [vp]
     lib.attn_check_status.restype = i32
     lib.attn_last_error.argtypes = []
@@ -143,6 +149,22 @@ def attn_bwd(Q, K, V, O, dO, LSE, dQ, dK, dV, causal: bool, scale: float, worksp
                                  _stream_handle(stream))
     if st != ATTN_OK:
         raise AttnError(st, "attn_bwd")
+
+
+def attn_bwd_static_workspace(Q, K, V, O, dO, LSE, dQ, dK, dV, causal: bool, scale: float, stream=None) -> None:
+    """attn_bwd without a caller workspace: for callers that cannot allocate
+    device memory; the library's fixed device array (ATTN_STATIC_WORKSPACE_BYTES)
+    is used instead.  Calls that overlap on the GPU race on that array."""
+    _check_bhnd("Q", Q)
+    for n, t in (("K", K), ("V", V), ("O", O), ("dO", dO), ("dQ", dQ), ("dK", dK), ("dV", dV)):
+        _check_bhnd(n, t, Q.shape)
+    _check_lse(LSE, Q.shape)
+    B, H, N, d = Q.shape
+    st = load_library().attn_bwd_static_workspace(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(dO), _ptr(LSE), _ptr(dQ),
+                                                  _ptr(dK), _ptr(dV), B, H, N, d, int(bool(causal)), float(scale),
+                                                  _stream_handle(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_bwd_static_workspace")
 
 
 def _ws(workspace):

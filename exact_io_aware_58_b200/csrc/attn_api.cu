@@ -295,6 +295,72 @@ ATTN_EXPORT int attn_bwd(const void* Q, const void* K, const void* V, const void
   return attn_bwd_dq(Q, K, V, dO, dQ, B, H, N, d, causal, scale, workspace, workspace_bytes, stream);
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Backward with a library-owned, fixed-size workspace.
+//
+// Some callers cannot allocate device memory at the point where they run the
+// backward: code whose memory is owned by another allocator that exposes no
+// way to hand out a raw scratch buffer across a C boundary (plugin hosts,
+// inference/training runtimes with a "no allocation after start-up" rule),
+// and code that runs where cudaMalloc is not allowed or would synchronise the
+// device.  For them the workspace lives in this file-scope device array.  It
+// exists on every GPU that loads the library, from module load until process
+// exit.  Its address is looked up once per device (cudaGetSymbolAddress with
+// that device current) and cached.
+// ---------------------------------------------------------------------------
+namespace {
+
+static __device__ __align__(256) unsigned char g_static_workspace[ATTN_STATIC_WORKSPACE_BYTES];
+
+constexpr int kMaxDevices = 64;
+
+void* static_workspace_for_current_device() {
+  static std::mutex mu;
+  static void* ptr[kMaxDevices] = {};
+  int dev = -1;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    fail(ATTN_ERR_DEVICE, "cudaGetDevice: %s (%lld)", cudaGetErrorString(e), (long long)dev);
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (ptr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_static_workspace);
+    if (e != cudaSuccess || p == nullptr) {
+      fail(ATTN_ERR_DEVICE, "cudaGetSymbolAddress(static workspace): %s (%lld)", cudaGetErrorString(e),
+           (long long)e);
+      return nullptr;
+    }
+    ptr[dev] = p;
+  }
+  return ptr[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+ATTN_EXPORT int attn_bwd_static_workspace(const void* Q, const void* K, const void* V, const void* O,
+                                          const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
+                                          int64_t B, int64_t H, int64_t N, int64_t d, int causal, float scale,
+                                          void* stream) {
+  const int s = check_sizes(B, H, N, d);
+  if (s != ATTN_OK) return s;
+  const size_t need = attn_bwd_workspace_bytes(B, H, N, d);
+  if (need > size_t(ATTN_STATIC_WORKSPACE_BYTES))
+    return fail(ATTN_ERR_WORKSPACE,
+                "%sattn_bwd_static_workspace: these sizes need %lld workspace bytes, more than the "
+                "ATTN_STATIC_WORKSPACE_BYTES the library holds; use attn_bwd with a caller workspace",
+                "", (long long)need);
+  void* ws = static_workspace_for_current_device();
+  if (ws == nullptr) return ATTN_ERR_DEVICE;
+  return attn_bwd(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, d, causal, scale, ws,
+                  size_t(ATTN_STATIC_WORKSPACE_BYTES), stream);
+}
+
 ATTN_EXPORT int attn_check_status(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ERR_DEVICE;
   unsigned int v = 0;

@@ -125,6 +125,42 @@ int attn_bwd_dq(const void* Q, const void* K, const void* V, const void* dO, voi
                 const void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Backward without any caller-provided memory: same computation, arguments
+ * and results as attn_bwd, but the workspace is a fixed array that the
+ * library owns in device memory.  (The pages have no counterpart: this is a
+ * deployment convenience, not part of the method.)
+ *
+ * Who needs it: callers that cannot allocate device memory where they run
+ * the backward -- e.g. code inside a runtime whose memory is owned by another
+ * allocator that offers no way to pass a raw scratch buffer across a C
+ * boundary, or code under a "no device allocation after start-up" rule (an
+ * allocation there can synchronise the device or is forbidden outright).
+ *
+ * Limits and behaviour:
+ *  - The array is ATTN_STATIC_WORKSPACE_BYTES (32 MiB) on every GPU that
+ *    loads the library, held from module load until process exit.  Sizes
+ *    whose attn_bwd_workspace_bytes() exceed it are rejected with
+ *    ATTN_ERR_WORKSPACE before anything is launched (attn_last_error() says
+ *    how many bytes they need).  32 MiB covers B*H*ceil(N/128)*128 up to 2^22
+ *    rows, e.g. B=8, H=32, N=16384.
+ *  - The first call on a device looks the array's device address up (with
+ *    that device current) and caches it; make that first call before any
+ *    stream capture.  The device used is the calling thread's current device.
+ *  - It calls no cudaMalloc, cudaFree or other allocating routine.
+ *  - Every call on a device shares the one array, and the array keeps the
+ *    last call's contents.  Nothing in it needs to start at zero: the
+ *    preprocess step writes every workspace element a call reads before the
+ *    other kernels read it.  Calls whose GPU work overlaps (e.g. on two
+ *    streams, or from two threads) race on the array; serialise them.
+ */
+#define ATTN_STATIC_WORKSPACE_BYTES (32u * 1024u * 1024u)
+
+int attn_bwd_static_workspace(const void* Q, const void* K, const void* V, const void* O,
+                              const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
+                              int64_t B, int64_t H, int64_t N, int64_t d, int causal, float scale,
+                              void* stream);
+
+/*
  * Synchronises `stream`, then reports and clears the device status word:
  * ATTN_OK, ATTN_ERR_TIMEOUT (a bounded device-side wait ran out in some
  * kernel since the last check), or ATTN_ERR_DEVICE (the CUDA context reports

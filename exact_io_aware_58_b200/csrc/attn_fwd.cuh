@@ -273,9 +273,17 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int k = 0; k < 128; ++k)
           if (k > limit) s[k] = -INFINITY;
       }
-      float mx = s[0];
+      // Row max as 8 independent chains (a single 127-long dependency chain
+      // would leave the issue slots idle for its whole latency).
+      float mxp[8];
 #pragma unroll
-      for (int k = 1; k < 128; ++k) mx = fmaxf(mx, s[k]);
+      for (int u = 0; u < 8; ++u) mxp[u] = s[u];
+#pragma unroll
+      for (int k = 8; k < 128; k += 8)
+#pragma unroll
+        for (int u = 0; u < 8; ++u) mxp[u] = fmaxf(mxp[u], s[k + u]);
+      const float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
+                             fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
       const float m_tile = mx * c;
       float alpha = 1.f;
       bool rescale = false;
@@ -286,7 +294,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
       l *= alpha;
       const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
-      float rowsum = 0.f;
+      float sump[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t pk[32];
@@ -294,12 +302,12 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         for (int k = 0; k < 32; ++k) {
           const float p0 = ex2(fmaf(s[h * 64 + 2 * k], c, neg_m));
           const float p1 = ex2(fmaf(s[h * 64 + 2 * k + 1], c, neg_m));
-          rowsum += p0 + p1;
+          sump[k & 3] += p0 + p1;
           pk[k] = pack_bf16x2(p0, p1);
         }
         tmem_st32(tP + h * 32, pk);
       }
-      l += rowsum;
+      l += (sump[0] + sump[1]) + (sump[2] + sump[3]);
       if (__any_sync(0xffffffffu, rescale)) {
         // O_t holds the sum through key tile j-1 (its last PV completed before S_t(j)).
         const float a = rescale ? alpha : 1.f;

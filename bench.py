@@ -49,25 +49,34 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def csrc_hash() -> str:
+KERNEL_SOURCES = {
+    "attn_fwd": ("attn_fwd.cuh", "sm100.cuh"),
+    "bwd_pre": ("attn_bwd.cuh", "sm100.cuh"),
+    "bwd_dkdv": ("attn_bwd.cuh", "sm100.cuh"),
+    "bwd_dq": ("attn_bwd.cuh", "sm100.cuh"),
+}
+
+
+def kernel_source_hash(kernel: str) -> str:
+    """Hash of the source files a kernel is compiled from."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "exact_io_aware_58_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
 def recorded_traffic(kernel: str):
-    """DRAM bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel sources (else None)."""
+    """DRAM bytes per launch (read + write) from a committed ncu summary, scaled
+    to the full workload, if it was taken on the kernel's current sources."""
     p = os.path.join(ROOT, "profiles", "dram_traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:
         rec = json.load(f)
     ent = rec.get(WORKLOAD, {}).get(kernel)
-    if not ent or ent.get("csrc_hash") != csrc_hash():
+    if not ent or ent.get("source_hash") != kernel_source_hash(kernel):
         return None
     return ent.get("bytes_per_launch")
 

@@ -368,6 +368,8 @@ ATTN_EXPORT int attn_check_status(void* stream) {
   if (v != 0) {
     const unsigned int zero = 0;
     if (cudaMemcpyToSymbol(attn::g_attn_status, &zero, sizeof(zero)) != cudaSuccess) return ATTN_ERR_DEVICE;
+    if (v & attn::kStatusLayout)
+      return fail(ATTN_ERR_DEVICE, "%sa kernel found its shared memory window misaligned and did no work%lld", "", 0);
     return ATTN_ERR_TIMEOUT;
   }
   return ATTN_OK;

@@ -83,28 +83,37 @@ struct BwdCfg {
   static constexpr int kTileBytes = 128 * D * 2;
   static constexpr int kBlockBytes = 128 * 128;
   static constexpr int kNumBlk = D / 64;
-  static constexpr int kStages = (D == 128) ? 2 : 4;
   static constexpr int kVecBytes = 512;                    // 128 fp32
   static constexpr int kThreads = 320;
   static constexpr int kWarpMma = 8;
   static constexpr int kWarpLoad = 9;
   static constexpr uint32_t kTmemCols = 512;
-  // dK/dV kernel: resident K_j, V_j; stages of (Q_i, dO_i, lse2_i, D_i).
+  // Ring depths.  The operand read last in an iteration (Q_i in dK/dV, K_j in
+  // dQ) gets the deeper ring, so its refill has more than one iteration to land.
+  static constexpr int kDeep = (D == 128) ? 3 : 4;
+  static constexpr int kShallow = (D == 128) ? 2 : 4;
+  // dK/dV kernel: resident K_j, V_j; ring of Q_i (+ its LSE/D vectors); ring of dO_i.
   static constexpr int kKV_OffK = 0;
   static constexpr int kKV_OffV = kTileBytes;
-  static constexpr int kKV_OffStage = 2 * kTileBytes;
-  static constexpr int kKV_StageBytes = 2 * kTileBytes + 2 * kVecBytes;
-  static constexpr int kKV_OffBar = kKV_OffStage + kStages * kKV_StageBytes;
-  // dQ kernel: resident Q_i, dO_i, lse2_i, D_i; stages of (K_j, V_j).
+  static constexpr int kKV_OffQ = 2 * kTileBytes;
+  static constexpr int kKV_OffDO = kKV_OffQ + kDeep * kTileBytes;
+  static constexpr int kVecSlots = 2;                                      // ring of (lse2[128], D[128])
+  static constexpr int kKV_OffVec = kKV_OffDO + kShallow * kTileBytes;
+  static constexpr int kKV_OffBar = kKV_OffVec + kVecSlots * 2 * kVecBytes;
+  // dQ kernel: resident Q_i, dO_i, LSE/D vectors; ring of K_j; ring of V_j.
   static constexpr int kQ_OffQ = 0;
   static constexpr int kQ_OffDO = kTileBytes;
-  static constexpr int kQ_OffVec = 2 * kTileBytes;
-  static constexpr int kQ_OffStage = 2 * kTileBytes + 1024;
-  static constexpr int kQ_StageBytes = 2 * kTileBytes;
-  static constexpr int kQ_OffBar = kQ_OffStage + kStages * kQ_StageBytes;
-  static constexpr int kNumBars = 2 * kStages + 8;
-  static constexpr int kKV_SmemBytes = kKV_OffBar + kNumBars * 8 + 16 + 1024;
-  static constexpr int kQ_SmemBytes = kQ_OffBar + kNumBars * 8 + 16 + 1024;
+  static constexpr int kQ_OffK = 2 * kTileBytes;
+  static constexpr int kQ_OffV = kQ_OffK + kDeep * kTileBytes;
+  static constexpr int kQ_OffVec = kQ_OffV + kShallow * kTileBytes;
+  static constexpr int kQ_OffBar = kQ_OffVec + 2 * kVecBytes;
+  static constexpr int kNumBars = 2 * kDeep + 2 * kShallow + 2 * kVecSlots + 8;
+  // Every tile offset above is a multiple of 1024 (the 128B-swizzle atom).
+  // The dynamic shared memory window starts 1024-byte aligned (checked at run
+  // time), so no alignment slack is reserved.
+  static constexpr int kKV_SmemBytes = kKV_OffBar + kNumBars * 8 + 16;
+  static constexpr int kQ_SmemBytes = kQ_OffBar + kNumBars * 8 + 16;
+  static_assert(kKV_SmemBytes <= 232448 && kQ_SmemBytes <= 232448, "shared memory budget");
   // TMEM columns
   static constexpr uint32_t kColA = 0;        // S^T (dkdv) / S (dq)
   static constexpr uint32_t kColB = 128;      // dP^T (dkdv) / dP (dq)
@@ -160,12 +169,16 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
                      const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
                      const BwdParams prm) {
   using C = BwdCfg<D>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  constexpr int QS = C::kDeep, OS = C::kShallow, VS = C::kVecSlots;
+  extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kKV_OffBar);
-  uint64_t* st_full = bars;                    // [kStages]
-  uint64_t* st_empty = st_full + C::kStages;   // [kStages]
-  uint64_t* kv_full = st_empty + C::kStages;
+  uint64_t* q_full = bars;                 // [QS]  Q_i landed
+  uint64_t* q_empty = q_full + QS;         // [QS]  dK(i) done: slot free
+  uint64_t* o_full = q_empty + QS;         // [OS]  dO_i landed
+  uint64_t* o_empty = o_full + OS;         // [OS]  dV(i) done: slot free
+  uint64_t* v_full = o_empty + OS;         // [VS]  LSE/D vectors of Q tile i landed
+  uint64_t* v_empty = v_full + VS;         // [VS]  compute warps done reading them
+  uint64_t* kv_full = v_empty + VS;
   uint64_t* s_full = kv_full + 1;
   uint64_t* dp_full = s_full + 1;
   uint64_t* p_full = dp_full + 1;
@@ -174,6 +187,10 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   uint64_t* drain = acc_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + C::kNumBars) + 1;
+  if (smem_u32(smem) & 1023u) {            // the layout needs a 1024-aligned window
+    if (threadIdx.x == 0) atomicOr(&g_attn_status, kStatusLayout);
+    return;
+  }
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -185,9 +202,17 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   const int n_it = nt - i_start;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(&st_full[s], 1);
-      mbar_init(&st_empty[s], 1);
+    for (int s = 0; s < QS; ++s) {
+      mbar_init(&q_full[s], 1);
+      mbar_init(&q_empty[s], 1);
+    }
+    for (int s = 0; s < OS; ++s) {
+      mbar_init(&o_full[s], 1);
+      mbar_init(&o_empty[s], 1);
+    }
+    for (int s = 0; s < VS; ++s) {
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 256);
     }
     mbar_init(kv_full, 1);
     mbar_init(s_full, 1);
@@ -215,26 +240,46 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         tma_load_3d(&tm_k, kv_full, smem + C::kKV_OffK + b * C::kBlockBytes, b * 64, n0, bh);
         tma_load_3d(&tm_v, kv_full, smem + C::kKV_OffV + b * C::kBlockBytes, b * 64, n0, bh);
       }
-      int issued = 0;
+      int q_issued = 0, o_issued = 0, v_issued = 0;
       for (int it = 0; it < n_it; ++it) {
-        const int slot = it % C::kStages;
-        const int use = it / C::kStages;
-        if (use > 0 && !mbar_wait(&st_empty[slot], (use - 1) & 1, abort_flag)) break;
         const int qi = i_start + it;
-        uint8_t* st = smem + C::kKV_OffStage + slot * C::kKV_StageBytes;
-        mbar_arrive_expect_tx(&st_full[slot], 2 * C::kTileBytes + 2 * C::kVecBytes);
-        for (int b = 0; b < C::kNumBlk; ++b) {
-          tma_load_3d(&tm_q, &st_full[slot], st + b * C::kBlockBytes, b * 64, qi * 128, bh);
-          tma_load_3d(&tm_do, &st_full[slot], st + C::kTileBytes + b * C::kBlockBytes, b * 64, qi * 128, bh);
+        {   // LSE*log2(e) and D of query tile i
+          const int slot = it % VS, use = it / VS;
+          if (use > 0 && !mbar_wait(&v_empty[slot], (use - 1) & 1, abort_flag)) break;
+          mbar_arrive_expect_tx(&v_full[slot], 2 * C::kVecBytes);
+          const size_t voff = size_t(bh) * size_t(prm.npad) + size_t(qi) * 128;
+          uint8_t* vec = smem + C::kKV_OffVec + slot * 2 * C::kVecBytes;
+          bulk_load(vec, prm.ws_lse2 + voff, C::kVecBytes, &v_full[slot]);
+          bulk_load(vec + C::kVecBytes, prm.ws_d + voff, C::kVecBytes, &v_full[slot]);
+          ++v_issued;
         }
-        const size_t voff = size_t(bh) * size_t(prm.npad) + size_t(qi) * 128;
-        bulk_load(st + 2 * C::kTileBytes, prm.ws_lse2 + voff, C::kVecBytes, &st_full[slot]);
-        bulk_load(st + 2 * C::kTileBytes + C::kVecBytes, prm.ws_d + voff, C::kVecBytes, &st_full[slot]);
-        ++issued;
+        {   // Q_i
+          const int slot = it % QS, use = it / QS;
+          if (use > 0 && !mbar_wait(&q_empty[slot], (use - 1) & 1, abort_flag)) break;
+          mbar_arrive_expect_tx(&q_full[slot], C::kTileBytes);
+          for (int b = 0; b < C::kNumBlk; ++b)
+            tma_load_3d(&tm_q, &q_full[slot], smem + C::kKV_OffQ + slot * C::kTileBytes + b * C::kBlockBytes, b * 64,
+                        qi * 128, bh);
+          ++q_issued;
+        }
+        {   // dO_i
+          const int slot = it % OS, use = it / OS;
+          if (use > 0 && !mbar_wait(&o_empty[slot], (use - 1) & 1, abort_flag)) break;
+          mbar_arrive_expect_tx(&o_full[slot], C::kTileBytes);
+          for (int b = 0; b < C::kNumBlk; ++b)
+            tma_load_3d(&tm_do, &o_full[slot], smem + C::kKV_OffDO + slot * C::kTileBytes + b * C::kBlockBytes, b * 64,
+                        qi * 128, bh);
+          ++o_issued;
+        }
       }
+      // No copy may still be landing in shared memory when the CTA leaves.
       mbar_wait(kv_full, 0, abort_flag, false);
-      for (int it = max(0, issued - C::kStages); it < issued; ++it)
-        mbar_wait(&st_full[it % C::kStages], (it / C::kStages) & 1, abort_flag, false);
+      for (int it = max(0, q_issued - QS); it < q_issued; ++it)
+        mbar_wait(&q_full[it % QS], (it / QS) & 1, abort_flag, false);
+      for (int it = max(0, o_issued - OS); it < o_issued; ++it)
+        mbar_wait(&o_full[it % OS], (it / OS) & 1, abort_flag, false);
+      for (int it = max(0, v_issued - VS); it < v_issued; ++it)
+        mbar_wait(&v_full[it % VS], (it / VS) & 1, abort_flag, false);
     }
     __syncwarp();
   } else if (warp == C::kWarpMma) {
@@ -243,7 +288,8 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       constexpr uint32_t kIdescAcc = idesc_bf16(128, D, false, true);    // dV, dK (B MN-major)
       const uint32_t sK = smem_u32(smem + C::kKV_OffK);
       const uint32_t sV = smem_u32(smem + C::kKV_OffV);
-      const uint32_t sSt = smem_u32(smem + C::kKV_OffStage);
+      auto q_tile = [&](int it) { return smem_u32(smem + C::kKV_OffQ + (it % QS) * C::kTileBytes); };
+      auto o_tile = [&](int it) { return smem_u32(smem + C::kKV_OffDO + (it % OS) * C::kTileBytes); };
       auto issue_kmajor = [&](uint32_t dcol, uint32_t a0, uint32_t b0) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -258,35 +304,37 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           mma_ts(tmem + dcol, tmem + acol + 64 * (kk >> 2) + (kk & 3) * 8,
                  smem_desc_sw128(b0 + kk * 2048, C::kBlockBytes, 1024), kIdescAcc, (acc || kk > 0) ? 1u : 0u);
       };
-      auto stage_q = [&](int it) { return sSt + (it % C::kStages) * C::kKV_StageBytes; };
-      auto stage_do = [&](int it) { return sSt + (it % C::kStages) * C::kKV_StageBytes + C::kTileBytes; };
+      auto wait_q = [&](int it) { return mbar_wait(&q_full[it % QS], (it / QS) & 1, abort_flag); };
+      auto wait_o = [&](int it) { return mbar_wait(&o_full[it % OS], (it / OS) & 1, abort_flag); };
 
-      bool ok = mbar_wait(kv_full, 0, abort_flag);
-      if (ok) ok = mbar_wait(&st_full[0], 0, abort_flag);
+      bool ok = mbar_wait(kv_full, 0, abort_flag) && wait_q(0) && wait_o(0);
       if (ok) {
         tc_fence_after();
-        issue_kmajor(C::kColA, sK, stage_q(0));    // S^T = K_j Q_i^T
+        issue_kmajor(C::kColA, sK, q_tile(0));    // S^T = K_j Q_i^T
         mma_commit(s_full);
-        issue_kmajor(C::kColB, sV, stage_do(0));   // dP^T = V_j dO_i^T
+        issue_kmajor(C::kColB, sV, o_tile(0));    // dP^T = V_j dO_i^T
         mma_commit(dp_full);
       }
       for (int it = 0; it < n_it && ok; ++it) {
+        const bool more = it + 1 < n_it;
         if (!(ok = mbar_wait(p_full, it & 1, abort_flag))) break;
         tc_fence_after();
-        issue_acc(C::kColAcc0, C::kColA, stage_do(it), it > 0);   // dV += P^T dO_i
-        const bool more = it + 1 < n_it;
+        issue_acc(C::kColAcc0, C::kColA, o_tile(it), it > 0);    // dV += P^T dO_i
+        mma_commit(&o_empty[it % OS]);                            // dO_i read for the last time
         if (more) {
-          if (!(ok = mbar_wait(&st_full[(it + 1) % C::kStages], ((it + 1) / C::kStages) & 1, abort_flag))) break;
+          if (!(ok = wait_q(it + 1))) break;
           tc_fence_after();
-          issue_kmajor(C::kColA, sK, stage_q(it + 1));
+          issue_kmajor(C::kColA, sK, q_tile(it + 1));
           mma_commit(s_full);
         }
         if (!(ok = mbar_wait(ds_full, it & 1, abort_flag))) break;
         tc_fence_after();
-        issue_acc(C::kColAcc1, C::kColB, stage_q(it), it > 0);    // dK += dS^T Q_i
-        mma_commit(&st_empty[it % C::kStages]);
+        issue_acc(C::kColAcc1, C::kColB, q_tile(it), it > 0);    // dK += dS^T Q_i
+        mma_commit(&q_empty[it % QS]);                            // Q_i read for the last time
         if (more) {
-          issue_kmajor(C::kColB, sV, stage_do(it + 1));
+          if (!(ok = wait_o(it + 1))) break;
+          tc_fence_after();
+          issue_kmajor(C::kColB, sV, o_tile(it + 1));
           mma_commit(dp_full);
         }
       }
@@ -308,12 +356,9 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
       const int qi = i_start + it;
-      const float* vec = reinterpret_cast<const float*>(smem + C::kKV_OffStage + (it % C::kStages) * C::kKV_StageBytes +
-                                                        2 * C::kTileBytes);
-      // The stage's LSE/D vectors: wait on the copy's own barrier (already
-      // complete by the time S^T of this stage is; the slot is only refilled
-      // after this iteration's dK MMA, i.e. after these reads).
-      if (!(ok = mbar_wait_warp(&st_full[it % C::kStages], (it / C::kStages) & 1, abort_flag))) break;
+      const float* vec = reinterpret_cast<const float*>(smem + C::kKV_OffVec + (it % VS) * 2 * C::kVecBytes);
+      // LSE/D vectors of this query tile (released below, after the dS reads).
+      if (!(ok = mbar_wait_warp(&v_full[it % VS], (it / VS) & 1, abort_flag))) break;
       if (!(ok = mbar_wait_warp(s_full, it & 1, abort_flag))) break;
       tc_fence_after();
       float p[64];
@@ -363,12 +408,12 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         }
         tmem_st32(tB, pk);   // dS^T over the first 32 of this group's 64 dP^T columns
       }
+      mbar_arrive(&v_empty[it % VS]);   // this thread is done with the LSE/D vectors
       tmem_st_wait();
       tc_fence_before();
       mbar_arrive(ds_full);
     }
-    (void)key;
-    // epilogue: group 0 writes dV (into the K_j... V_j slot), group 1 writes dK (into the K_j slot)
+    // epilogue: group 0 writes dV (staged in the V_j slot), group 1 writes dK (in the K_j slot)
     if (ok) ok = mbar_wait_warp(acc_full, 0, abort_flag);
     uint8_t* stage = smem + (g == 0 ? C::kKV_OffV : C::kKV_OffK);
     if (ok) {
@@ -404,12 +449,14 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                    const __grid_constant__ CUtensorMap tm_dq, const BwdParams prm) {
   using C = BwdCfg<D>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  constexpr int KS = C::kDeep, VS = C::kShallow;
+  extern __shared__ __align__(1024) uint8_t smem[];
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kQ_OffBar);
-  uint64_t* st_full = bars;
-  uint64_t* st_empty = st_full + C::kStages;
-  uint64_t* q_full = st_empty + C::kStages;
+  uint64_t* k_full = bars;                 // [KS]
+  uint64_t* k_empty = k_full + KS;         // [KS]  dQ(j) done
+  uint64_t* v_full = k_empty + KS;         // [VS]
+  uint64_t* v_empty = v_full + VS;         // [VS]  dP(j) done
+  uint64_t* q_full = v_empty + VS;
   uint64_t* s_full = q_full + 1;
   uint64_t* s_free = s_full + 1;
   uint64_t* dp_full = s_free + 1;
@@ -418,6 +465,10 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   uint64_t* drain = acc_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + C::kNumBars) + 1;
+  if (smem_u32(smem) & 1023u) {            // the layout needs a 1024-aligned window
+    if (threadIdx.x == 0) atomicOr(&g_attn_status, kStatusLayout);
+    return;
+  }
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -429,9 +480,13 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   const int n_it = CAUSAL ? it_q + 1 : nt;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(&st_full[s], 1);
-      mbar_init(&st_empty[s], 1);
+    for (int s = 0; s < KS; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+    }
+    for (int s = 0; s < VS; ++s) {
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     mbar_init(q_full, 1);
     mbar_init(s_full, 1);
@@ -462,22 +517,32 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       const size_t voff = size_t(bh) * size_t(prm.npad) + size_t(m0);
       bulk_load(smem + C::kQ_OffVec, prm.ws_lse2 + voff, C::kVecBytes, q_full);
       bulk_load(smem + C::kQ_OffVec + C::kVecBytes, prm.ws_d + voff, C::kVecBytes, q_full);
-      int issued = 0;
+      int k_issued = 0, v_issued = 0;
       for (int it = 0; it < n_it; ++it) {
-        const int slot = it % C::kStages;
-        const int use = it / C::kStages;
-        if (use > 0 && !mbar_wait(&st_empty[slot], (use - 1) & 1, abort_flag)) break;
-        uint8_t* st = smem + C::kQ_OffStage + slot * C::kQ_StageBytes;
-        mbar_arrive_expect_tx(&st_full[slot], 2 * C::kTileBytes);
-        for (int b = 0; b < C::kNumBlk; ++b) {
-          tma_load_3d(&tm_k, &st_full[slot], st + b * C::kBlockBytes, b * 64, it * 128, bh);
-          tma_load_3d(&tm_v, &st_full[slot], st + C::kTileBytes + b * C::kBlockBytes, b * 64, it * 128, bh);
+        {
+          const int slot = it % KS, use = it / KS;
+          if (use > 0 && !mbar_wait(&k_empty[slot], (use - 1) & 1, abort_flag)) break;
+          mbar_arrive_expect_tx(&k_full[slot], C::kTileBytes);
+          for (int b = 0; b < C::kNumBlk; ++b)
+            tma_load_3d(&tm_k, &k_full[slot], smem + C::kQ_OffK + slot * C::kTileBytes + b * C::kBlockBytes, b * 64,
+                        it * 128, bh);
+          ++k_issued;
         }
-        ++issued;
+        {
+          const int slot = it % VS, use = it / VS;
+          if (use > 0 && !mbar_wait(&v_empty[slot], (use - 1) & 1, abort_flag)) break;
+          mbar_arrive_expect_tx(&v_full[slot], C::kTileBytes);
+          for (int b = 0; b < C::kNumBlk; ++b)
+            tma_load_3d(&tm_v, &v_full[slot], smem + C::kQ_OffV + slot * C::kTileBytes + b * C::kBlockBytes, b * 64,
+                        it * 128, bh);
+          ++v_issued;
+        }
       }
       mbar_wait(q_full, 0, abort_flag, false);
-      for (int it = max(0, issued - C::kStages); it < issued; ++it)
-        mbar_wait(&st_full[it % C::kStages], (it / C::kStages) & 1, abort_flag, false);
+      for (int it = max(0, k_issued - KS); it < k_issued; ++it)
+        mbar_wait(&k_full[it % KS], (it / KS) & 1, abort_flag, false);
+      for (int it = max(0, v_issued - VS); it < v_issued; ++it)
+        mbar_wait(&v_full[it % VS], (it / VS) & 1, abort_flag, false);
     }
     __syncwarp();
   } else if (warp == C::kWarpMma) {
@@ -486,7 +551,10 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       constexpr uint32_t kIdescAcc = idesc_bf16(128, D, false, true);
       const uint32_t sQ = smem_u32(smem + C::kQ_OffQ);
       const uint32_t sDO = smem_u32(smem + C::kQ_OffDO);
-      const uint32_t sSt = smem_u32(smem + C::kQ_OffStage);
+      auto k_tile = [&](int it) { return smem_u32(smem + C::kQ_OffK + (it % KS) * C::kTileBytes); };
+      auto v_tile = [&](int it) { return smem_u32(smem + C::kQ_OffV + (it % VS) * C::kTileBytes); };
+      auto wait_k = [&](int it) { return mbar_wait(&k_full[it % KS], (it / KS) & 1, abort_flag); };
+      auto wait_v = [&](int it) { return mbar_wait(&v_full[it % VS], (it / VS) & 1, abort_flag); };
       auto issue_kmajor = [&](uint32_t dcol, uint32_t a0, uint32_t b0) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -495,39 +563,40 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
                  kk > 0 ? 1u : 0u);
         }
       };
-      auto stage_k = [&](int it) { return sSt + (it % C::kStages) * C::kQ_StageBytes; };
-      auto stage_v = [&](int it) { return sSt + (it % C::kStages) * C::kQ_StageBytes + C::kTileBytes; };
 
-      bool ok = mbar_wait(q_full, 0, abort_flag);
-      if (ok) ok = mbar_wait(&st_full[0], 0, abort_flag);
+      bool ok = mbar_wait(q_full, 0, abort_flag) && wait_k(0) && wait_v(0);
       if (ok) {
         tc_fence_after();
-        issue_kmajor(C::kColA, sQ, stage_k(0));    // S = Q_i K_j^T
+        issue_kmajor(C::kColA, sQ, k_tile(0));    // S = Q_i K_j^T
         mma_commit(s_full);
-        issue_kmajor(C::kColB, sDO, stage_v(0));   // dP = dO_i V_j^T
+        issue_kmajor(C::kColB, sDO, v_tile(0));   // dP = dO_i V_j^T
         mma_commit(dp_full);
+        mma_commit(&v_empty[0]);                  // V_j read for the last time
       }
       for (int it = 0; it < n_it && ok; ++it) {
         const bool more = it + 1 < n_it;
         if (more) {
-          if (!(ok = mbar_wait(&st_full[(it + 1) % C::kStages], ((it + 1) / C::kStages) & 1, abort_flag))) break;
+          if (!(ok = wait_k(it + 1))) break;
           if (!(ok = mbar_wait(s_free, it & 1, abort_flag))) break;
           tc_fence_after();
-          issue_kmajor(C::kColA, sQ, stage_k(it + 1));
+          issue_kmajor(C::kColA, sQ, k_tile(it + 1));
           mma_commit(s_full);
         }
         if (!(ok = mbar_wait(ds_full, it & 1, abort_flag))) break;
         tc_fence_after();
         // dQ += dS K_j: A = dS in TMEM (over dP columns), B = K_j MN-major
-        const uint32_t bk = stage_k(it);
+        const uint32_t bk = k_tile(it);
 #pragma unroll
         for (int kk = 0; kk < 128 / 16; ++kk)
           mma_ts(tmem + C::kColAcc0, tmem + C::kColB + 64 * (kk >> 2) + (kk & 3) * 8,
                  smem_desc_sw128(bk + kk * 2048, C::kBlockBytes, 1024), kIdescAcc, (it > 0 || kk > 0) ? 1u : 0u);
-        mma_commit(&st_empty[it % C::kStages]);
+        mma_commit(&k_empty[it % KS]);            // K_j read for the last time
         if (more) {
-          issue_kmajor(C::kColB, sDO, stage_v(it + 1));
+          if (!(ok = wait_v(it + 1))) break;
+          tc_fence_after();
+          issue_kmajor(C::kColB, sDO, v_tile(it + 1));
           mma_commit(dp_full);
+          mma_commit(&v_empty[(it + 1) % VS]);
         }
       }
       if (ok) mma_commit(acc_full);

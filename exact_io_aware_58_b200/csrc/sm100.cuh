@@ -16,7 +16,8 @@ namespace attn {
 
 // Device status word, read and cleared by attn_check_status().
 __device__ unsigned int g_attn_status = 0;
-constexpr unsigned int kStatusTimeout = 1u;
+constexpr unsigned int kStatusTimeout = 1u;   // a bounded wait ran out
+constexpr unsigned int kStatusLayout = 2u;    // shared memory window not laid out as required
 
 constexpr unsigned long long kWaitTimeoutNs = 2000000000ull;   // 2 s per wait
 

@@ -239,40 +239,106 @@ def run_ours(args, rank, world, local_rank):
                 "frac": round(achieved / sustained, 4), "frac_of_burst": round(achieved / burst, 4),
                 "traffic": recorded_traffic(dom)}
 
+    # ------------------------------------------------- shared key/value heads
+    gqa = None
+    if not args.no_gqa and w.H % args.gqa_kv_heads == 0:
+        hk = args.gqa_kv_heads
+        kg, vg = k[:, :hk].contiguous(), v[:, :hk].contiguous()
+        dkg, dvg = torch.empty_like(kg), torch.empty_like(vg)
+
+        def gqa_step(ev=None):
+            if ev is not None:
+                ev[0].record(stream)
+            attn.attn_fwd_gqa(q, kg, vg, o, lse, causal, scale, stream)
+            if ev is not None:
+                ev[1].record(stream)
+            attn.attn_bwd_gqa(q, kg, vg, o, do, lse, dq, dkg, dvg, causal, scale, ws, stream)
+            if ev is not None:
+                ev[2].record(stream)
+
+        for _ in range(args.warmup):
+            gqa_step()
+        n_g = max(3, min(args.steps, 5))
+        gev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_g)]
+        torch.cuda.synchronize()
+        for e in gev:
+            gqa_step(e)
+        torch.cuda.synchronize()
+        assert attn.attn_check_status(stream) == attn.ATTN_OK
+        gf = sum(e[0].elapsed_time(e[1]) for e in gev) / n_g
+        gb = sum(e[1].elapsed_time(e[2]) for e in gev) / n_g
+        gf, gb = max_over_ranks([gf, gb], device=dev)
+        gqa = {"H_kv": hk, "group": w.H // hk, "ms_fwd": round(gf, 3), "ms_bwd": round(gb, 3),
+               "fwd_tflops": round(aggregate_tflops(f_fwd, world, gf), 2),
+               "fwdbwd_tflops": round(aggregate_tflops(3.5 * f_fwd, world, gf + gb), 2), "steps": n_g}
+        del kg, vg, dkg, dvg
+
     # ---------------------------------------------------------------- e2e
+    # Through host buffers: every step copies its inputs Q, K, V, dO from
+    # pinned host memory to the device and its results O, LSE, dQ, dK, dV back.
+    # Steps are pipelined over three streams with two device buffer sets, so
+    # step i+1's upload and step i-1's download overlap step i's kernels.
     e2e = None
     if not args.no_e2e:
-        hq, hk, hv, hdo = (t.cpu().pin_memory() for t in (q, k, v, do))
-        ho, hdq, hdk, hdv = (torch.empty(q.shape, dtype=q.dtype).pin_memory() for _ in range(4))
-        hlse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        del inp
+        sets = []
+        for b in range(2):
+            dev_in = [torch.empty_like(q) for _ in range(4)]
+            dev_out = [torch.empty_like(q), torch.empty_like(lse), torch.empty_like(q), torch.empty_like(q),
+                       torch.empty_like(q)]
+            host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in dev_out]
+            sets.append((dev_in, dev_out, host_out))
+        host_in = [t.cpu().pin_memory() for t in (q, k, v, do)]
+        s_up, s_run, s_down = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_up = [torch.cuda.Event() for _ in range(2)]
+        ev_run = [torch.cuda.Event() for _ in range(2)]
+        ev_down = [torch.cuda.Event() for _ in range(2)]
+        for e in ev_run + ev_down:
+            e.record(s_run)
 
-        def e2e_step():
-            for dst, src in ((q, hq), (k, hk), (v, hv), (do, hdo)):
-                dst.copy_(src, non_blocking=True)
-            step()
-            for dst, src in ((ho, o), (hlse, lse), (hdq, dq), (hdk, dk), (hdv, dv)):
-                dst.copy_(src, non_blocking=True)
+        def e2e_step(i):
+            b = i % 2
+            dev_in, dev_out, host_out = sets[b]
+            with torch.cuda.stream(s_up):
+                s_up.wait_event(ev_run[b])          # inputs of step i-2 no longer read
+                for dst, src in zip(dev_in, host_in):
+                    dst.copy_(src, non_blocking=True)
+                ev_up[b].record(s_up)
+            s_run.wait_event(ev_up[b])
+            s_run.wait_event(ev_down[b])            # outputs of step i-2 already downloaded
+            qi, ki, vi, doi = dev_in
+            oo, ll, dqo, dko, dvo = dev_out
+            attn.attn_fwd(qi, ki, vi, oo, ll, causal, scale, s_run)
+            attn.attn_bwd(qi, ki, vi, oo, doi, ll, dqo, dko, dvo, causal, scale, ws, s_run)
+            ev_run[b].record(s_run)
+            with torch.cuda.stream(s_down):
+                s_down.wait_event(ev_run[b])
+                for dst, src in zip(host_out, dev_out):
+                    dst.copy_(src, non_blocking=True)
+                ev_down[b].record(s_down)
 
-        e2e_step()
+        for i in range(2):
+            e2e_step(i)
         torch.cuda.synchronize()
         n_e2e = max(3, min(args.steps, 10))
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for _ in range(n_e2e):
-            e2e_step()
-        b.record(stream)
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(s_up)
+        for i in range(n_e2e):
+            e2e_step(i)
+        b_.record(s_down)
         torch.cuda.synchronize()
-        e_ms = max_over_ranks([a.elapsed_time(b) / n_e2e], device=dev)[0]
+        e_ms = max_over_ranks([a.elapsed_time(b_) / n_e2e], device=dev)[0]
         elt = q.element_size()
         h2d = 4 * q.numel() * elt
         d2h = 4 * q.numel() * elt + lse.numel() * 4
         e2e = {"value": round(aggregate_tflops(3.5 * f_fwd, world, e_ms), 2), "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e_ms, 3),
-               "steps": n_e2e}
+               "steps": n_e2e, "pipelined": "upload / kernels / download on three streams, two buffer sets"}
         assert attn.attn_check_status(stream) == attn.ATTN_OK
+        del sets, host_in
 
     # ------------------------------------------------------- CPU baseline
     cpu = None
@@ -309,6 +375,7 @@ def run_ours(args, rank, world, local_rank):
         },
         "kernel_ms": {kname: round(t, 3) for kname, t in per_kernel.items()},
         "roofline": roofline,
+        "gqa": gqa,
         "gpu_launches": 4 * args.steps,
         "clocks": clk,
         "e2e": e2e,
@@ -398,6 +465,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-gqa", action="store_true", help="skip the shared key/value head measurement")
+    ap.add_argument("--gqa-kv-heads", type=int, default=8)
     ap.add_argument("--cpu-rows", type=int, default=16384)
     ap.add_argument("--ref-rows", type=int, default=8192)
     ap.add_argument("--batch", type=int, default=0, help="override B (profiling captures only)")

@@ -30,7 +30,8 @@ ATTN_ERR_LAUNCH = -5
 ATTN_ERR_TIMEOUT = -6
 ATTN_ERR_DEVICE = -7
 
-EXPORTED = ("attn_fwd", "attn_bwd", "attn_bwd_workspace_bytes", "attn_bwd_preprocess", "attn_bwd_dkdv",
+EXPORTED = ("attn_fwd", "attn_fwd_gqa", "attn_bwd", "attn_bwd_gqa", "attn_bwd_workspace_bytes",
+            "attn_bwd_preprocess", "attn_bwd_dkdv",
             "attn_bwd_dq", "attn_bwd_static_workspace", "attn_check_status", "attn_last_error",
             "attn_status_string")
 
@@ -61,6 +62,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     i64, vp, f32, i32 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_float, ctypes.c_int
     lib.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, f32, vp]
     lib.attn_fwd.restype = i32
+    lib.attn_fwd_gqa.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i32, f32, vp]
+    lib.attn_fwd_gqa.restype = i32
+    lib.attn_bwd_gqa.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i32, f32, vp,
+                                 ctypes.c_size_t, vp]
+    lib.attn_bwd_gqa.restype = i32
     lib.attn_bwd_workspace_bytes.argtypes = [i64, i64, i64, i64]
     lib.attn_bwd_workspace_bytes.restype = ctypes.c_size_t
     lib.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, f32, vp,
@@ -128,6 +134,50 @@ def attn_fwd(Q, K, V, O, LSE, causal: bool, scale: float, stream=None) -> None:
                                  float(scale), _stream_handle(stream))
     if st != ATTN_OK:
         raise AttnError(st, "attn_fwd")
+
+
+def _check_kv(name: str, t: torch.Tensor, q_shape):
+    B, H, N, d = q_shape
+    if not t.is_cuda or t.dtype != torch.bfloat16 or t.dim() != 4 or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor of shape (B, H_kv, N, d)")
+    Hk = t.shape[1]
+    if t.shape[0] != B or t.shape[2] != N or t.shape[3] != d or Hk < 1 or H % Hk != 0:
+        raise ValueError(f"{name} has shape {tuple(t.shape)}; expected (B, H_kv, N, d) with H % H_kv == 0")
+    return Hk
+
+
+def attn_fwd_gqa(Q, K, V, O, LSE, causal: bool, scale: float, stream=None) -> None:
+    """attn_fwd with K, V of shape (B, H_kv, N, d) shared by groups of H / H_kv query heads."""
+    _check_bhnd("Q", Q)
+    _check_bhnd("O", O, Q.shape)
+    Hk = _check_kv("K", K, Q.shape)
+    if _check_kv("V", V, Q.shape) != Hk:
+        raise ValueError("K and V must have the same number of heads")
+    _check_lse(LSE, Q.shape)
+    B, H, N, d = Q.shape
+    st = load_library().attn_fwd_gqa(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE), B, H, Hk, N, d,
+                                     int(bool(causal)), float(scale), _stream_handle(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd_gqa")
+
+
+def attn_bwd_gqa(Q, K, V, O, dO, LSE, dQ, dK, dV, causal: bool, scale: float, workspace, stream=None) -> None:
+    """attn_bwd with K, V, dK, dV of shape (B, H_kv, N, d)."""
+    _check_bhnd("Q", Q)
+    for n, t in (("O", O), ("dO", dO), ("dQ", dQ)):
+        _check_bhnd(n, t, Q.shape)
+    Hk = _check_kv("K", K, Q.shape)
+    for n, t in (("V", V), ("dK", dK), ("dV", dV)):
+        if _check_kv(n, t, Q.shape) != Hk:
+            raise ValueError(f"{n} must have the same number of heads as K")
+    _check_lse(LSE, Q.shape)
+    B, H, N, d = Q.shape
+    wp, wb = _ws(workspace)
+    st = load_library().attn_bwd_gqa(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(dO), _ptr(LSE), _ptr(dQ), _ptr(dK),
+                                     _ptr(dV), B, H, Hk, N, d, int(bool(causal)), float(scale), wp, wb,
+                                     _stream_handle(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_bwd_gqa")
 
 
 def attn_bwd_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
@@ -223,11 +273,15 @@ def default_scale(d: int) -> float:
 
 
 def forward(Q, K, V, causal: bool, scale: float | None = None, stream=None):
+    """O, LSE for Q (B, H, N, d) and K, V (B, H_kv, N, d); H_kv == H is plain multi-head attention."""
     B, H, N, d = Q.shape
     scale = default_scale(d) if scale is None else scale
     O = torch.empty_like(Q)
     LSE = torch.empty((B, H, N), dtype=torch.float32, device=Q.device)
-    attn_fwd(Q, K, V, O, LSE, causal, scale, stream)
+    if K.shape[1] == H:
+        attn_fwd(Q, K, V, O, LSE, causal, scale, stream)
+    else:
+        attn_fwd_gqa(Q, K, V, O, LSE, causal, scale, stream)
     return O, LSE
 
 
@@ -242,5 +296,8 @@ def backward(Q, K, V, O, LSE, dO, causal: bool, scale: float | None = None, work
     if workspace is None:
         workspace = alloc_workspace(B, H, N, d, Q.device)
     dQ, dK, dV = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
-    attn_bwd(Q, K, V, O, dO, LSE, dQ, dK, dV, causal, scale, workspace, stream)
+    if K.shape[1] == H:
+        attn_bwd(Q, K, V, O, dO, LSE, dQ, dK, dV, causal, scale, workspace, stream)
+    else:
+        attn_bwd_gqa(Q, K, V, O, dO, LSE, dQ, dK, dV, causal, scale, workspace, stream)
     return dQ, dK, dV

@@ -80,6 +80,11 @@ int check_sizes(int64_t B, int64_t H, int64_t N, int64_t d) {
   return ATTN_OK;
 }
 
+int check_heads(int64_t H, int64_t H_kv) {
+  if (H_kv < 1 || H_kv > H || H % H_kv != 0) return ATTN_ERR_INVALID_ARG;
+  return ATTN_OK;
+}
+
 int check_scale(float scale) { return (std::isfinite(scale) && scale > 0.f) ? ATTN_OK : ATTN_ERR_INVALID_ARG; }
 
 int launch_status() {
@@ -145,23 +150,31 @@ int64_t npad_of(int64_t N) { return (N + 127) / 128 * 128; }
 
 extern "C" {
 
-ATTN_EXPORT int attn_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int64_t B, int64_t H, int64_t N,
-             int64_t d, int causal, float scale, void* stream) {
+}  // extern "C"
+
+namespace {
+
+int fwd_impl(const void* Q, const void* K, const void* V, void* O, float* LSE, int64_t B, int64_t H, int64_t H_kv,
+             int64_t N, int64_t d, int causal, float scale, void* stream) {
   int s = check_sizes(B, H, N, d);
   if (s != ATTN_OK) return s;
+  if ((s = check_heads(H, H_kv)) != ATTN_OK) return s;
   if ((s = check_scale(scale)) != ATTN_OK) return s;
   if (!Q || !K || !V || !O || !LSE) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE))
     return ATTN_ERR_MISALIGNED;
-  const int64_t bh = B * H;
+  const int64_t bh = B * H, bhkv = B * H_kv;
   CUtensorMap mq, mk, mv, mo;
-  if (!make_map(&mq, Q, bh, N, d) || !make_map(&mk, K, bh, N, d) || !make_map(&mv, V, bh, N, d) ||
+  if (!make_map(&mq, Q, bh, N, d) || !make_map(&mk, K, bhkv, N, d) || !make_map(&mv, V, bhkv, N, d) ||
       !make_map(&mo, O, bh, N, d))
     return ATTN_ERR_LAUNCH;
   attn::FwdParams prm;
   prm.lse = LSE;
   prm.n = int(N);
   prm.n_mblk = int((N + 255) / 256);
+  prm.h = int(H);
+  prm.h_kv = int(H_kv);
+  prm.group = int(H / H_kv);
   prm.scale_log2 = scale * 1.4426950408889634f;
   const int64_t grid = bh * prm.n_mblk;
   if (grid > INT32_MAX) return ATTN_ERR_INVALID_ARG;
@@ -171,6 +184,20 @@ ATTN_EXPORT int attn_fwd(const void* Q, const void* K, const void* V, void* O, f
                   : launch_fwd<128, false>(mq, mk, mv, mo, prm, int(grid), st);
   return causal ? launch_fwd<64, true>(mq, mk, mv, mo, prm, int(grid), st)
                 : launch_fwd<64, false>(mq, mk, mv, mo, prm, int(grid), st);
+}
+
+}  // namespace
+
+extern "C" {
+
+ATTN_EXPORT int attn_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int64_t B, int64_t H,
+                         int64_t N, int64_t d, int causal, float scale, void* stream) {
+  return fwd_impl(Q, K, V, O, LSE, B, H, H, N, d, causal, scale, stream);
+}
+
+ATTN_EXPORT int attn_fwd_gqa(const void* Q, const void* K, const void* V, void* O, float* LSE, int64_t B, int64_t H,
+                             int64_t H_kv, int64_t N, int64_t d, int causal, float scale, void* stream) {
+  return fwd_impl(Q, K, V, O, LSE, B, H, H_kv, N, d, causal, scale, stream);
 }
 
 ATTN_EXPORT size_t attn_bwd_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d) {
@@ -202,8 +229,11 @@ int bwd_common_checks(int64_t B, int64_t H, int64_t N, int64_t d, const void* wo
   return ATTN_OK;
 }
 
-attn::BwdParams bwd_params(const BwdSetup& su, int64_t N, float scale) {
+attn::BwdParams bwd_params(const BwdSetup& su, int64_t N, int64_t H, int64_t H_kv, float scale) {
   attn::BwdParams prm;
+  prm.h = int(H);
+  prm.h_kv = int(H_kv);
+  prm.group = int(H / H_kv);
   prm.ws_lse2 = su.ws_lse2;
   prm.ws_d = su.ws_d;
   prm.n = int(N);
@@ -230,22 +260,28 @@ ATTN_EXPORT int attn_bwd_preprocess(const void* O, const void* dO, const float* 
                     : launch_bwd_pre<64>(O, dO, LSE, su.ws_lse2, su.ws_d, int(N), int(su.npad), su.bh * su.npad, st);
 }
 
-ATTN_EXPORT int attn_bwd_dkdv(const void* Q, const void* K, const void* V, const void* dO, void* dK, void* dV,
-                              int64_t B, int64_t H, int64_t N, int64_t d, int causal, float scale,
-                              const void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+int dkdv_impl(const void* Q, const void* K, const void* V, const void* dO, void* dK, void* dV, int64_t B, int64_t H,
+              int64_t H_kv, int64_t N, int64_t d, int causal, float scale, const void* workspace,
+              size_t workspace_bytes, void* stream) {
   BwdSetup su;
   int s = bwd_common_checks(B, H, N, d, workspace, workspace_bytes, &su);
   if (s != ATTN_OK) return s;
+  if ((s = check_heads(H, H_kv)) != ATTN_OK) return s;
   if ((s = check_scale(scale)) != ATTN_OK) return s;
   if (!Q || !K || !V || !dO || !dK || !dV) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(dO) || !aligned16(dK) || !aligned16(dV))
     return ATTN_ERR_MISALIGNED;
+  const int64_t bhkv = B * H_kv;
   CUtensorMap mq, mk, mv, mdo, mdk, mdv;
-  if (!make_map(&mq, Q, su.bh, N, d) || !make_map(&mk, K, su.bh, N, d) || !make_map(&mv, V, su.bh, N, d) ||
-      !make_map(&mdo, dO, su.bh, N, d) || !make_map(&mdk, dK, su.bh, N, d) || !make_map(&mdv, dV, su.bh, N, d))
+  if (!make_map(&mq, Q, su.bh, N, d) || !make_map(&mk, K, bhkv, N, d) || !make_map(&mv, V, bhkv, N, d) ||
+      !make_map(&mdo, dO, su.bh, N, d) || !make_map(&mdk, dK, bhkv, N, d) || !make_map(&mdv, dV, bhkv, N, d))
     return ATTN_ERR_LAUNCH;
-  const attn::BwdParams prm = bwd_params(su, N, scale);
-  const int grid = int(su.bh * prm.n_tiles);
+  const attn::BwdParams prm = bwd_params(su, N, H, H_kv, scale);
+  const int grid = int(bhkv * prm.n_tiles);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (d == 128)
     return causal ? launch_dkdv<128, true>(mq, mk, mv, mdo, mdk, mdv, prm, grid, st)
@@ -254,20 +290,22 @@ ATTN_EXPORT int attn_bwd_dkdv(const void* Q, const void* K, const void* V, const
                 : launch_dkdv<64, false>(mq, mk, mv, mdo, mdk, mdv, prm, grid, st);
 }
 
-ATTN_EXPORT int attn_bwd_dq(const void* Q, const void* K, const void* V, const void* dO, void* dQ, int64_t B,
-                            int64_t H, int64_t N, int64_t d, int causal, float scale, const void* workspace,
-                            size_t workspace_bytes, void* stream) {
+int dq_impl(const void* Q, const void* K, const void* V, const void* dO, void* dQ, int64_t B, int64_t H, int64_t H_kv,
+            int64_t N, int64_t d, int causal, float scale, const void* workspace, size_t workspace_bytes,
+            void* stream) {
   BwdSetup su;
   int s = bwd_common_checks(B, H, N, d, workspace, workspace_bytes, &su);
   if (s != ATTN_OK) return s;
+  if ((s = check_heads(H, H_kv)) != ATTN_OK) return s;
   if ((s = check_scale(scale)) != ATTN_OK) return s;
   if (!Q || !K || !V || !dO || !dQ) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(dO) || !aligned16(dQ)) return ATTN_ERR_MISALIGNED;
+  const int64_t bhkv = B * H_kv;
   CUtensorMap mq, mk, mv, mdo, mdq;
-  if (!make_map(&mq, Q, su.bh, N, d) || !make_map(&mk, K, su.bh, N, d) || !make_map(&mv, V, su.bh, N, d) ||
+  if (!make_map(&mq, Q, su.bh, N, d) || !make_map(&mk, K, bhkv, N, d) || !make_map(&mv, V, bhkv, N, d) ||
       !make_map(&mdo, dO, su.bh, N, d) || !make_map(&mdq, dQ, su.bh, N, d))
     return ATTN_ERR_LAUNCH;
-  const attn::BwdParams prm = bwd_params(su, N, scale);
+  const attn::BwdParams prm = bwd_params(su, N, H, H_kv, scale);
   const int grid = int(su.bh * prm.n_tiles);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (d == 128)
@@ -277,11 +315,12 @@ ATTN_EXPORT int attn_bwd_dq(const void* Q, const void* K, const void* V, const v
                 : launch_dq<64, false>(mq, mk, mv, mdo, mdq, prm, grid, st);
 }
 
-ATTN_EXPORT int attn_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
-                         void* dQ, void* dK, void* dV, int64_t B, int64_t H, int64_t N, int64_t d, int causal,
-                         float scale, void* workspace, size_t workspace_bytes, void* stream) {
+int bwd_impl(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE, void* dQ,
+             void* dK, void* dV, int64_t B, int64_t H, int64_t H_kv, int64_t N, int64_t d, int causal, float scale,
+             void* workspace, size_t workspace_bytes, void* stream) {
   int s = check_sizes(B, H, N, d);
   if (s != ATTN_OK) return s;
+  if ((s = check_heads(H, H_kv)) != ATTN_OK) return s;
   if ((s = check_scale(scale)) != ATTN_OK) return s;
   if (!Q || !K || !V || !O || !dO || !LSE || !dQ || !dK || !dV || !workspace) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(dO) || !aligned16(LSE) ||
@@ -290,9 +329,39 @@ ATTN_EXPORT int attn_bwd(const void* Q, const void* K, const void* V, const void
   if (workspace_bytes < attn_bwd_workspace_bytes(B, H, N, d)) return ATTN_ERR_WORKSPACE;
   s = attn_bwd_preprocess(O, dO, LSE, B, H, N, d, workspace, workspace_bytes, stream);
   if (s != ATTN_OK) return s;
-  s = attn_bwd_dkdv(Q, K, V, dO, dK, dV, B, H, N, d, causal, scale, workspace, workspace_bytes, stream);
+  s = dkdv_impl(Q, K, V, dO, dK, dV, B, H, H_kv, N, d, causal, scale, workspace, workspace_bytes, stream);
   if (s != ATTN_OK) return s;
-  return attn_bwd_dq(Q, K, V, dO, dQ, B, H, N, d, causal, scale, workspace, workspace_bytes, stream);
+  return dq_impl(Q, K, V, dO, dQ, B, H, H_kv, N, d, causal, scale, workspace, workspace_bytes, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+ATTN_EXPORT int attn_bwd_dkdv(const void* Q, const void* K, const void* V, const void* dO, void* dK, void* dV,
+                              int64_t B, int64_t H, int64_t N, int64_t d, int causal, float scale,
+                              const void* workspace, size_t workspace_bytes, void* stream) {
+  return dkdv_impl(Q, K, V, dO, dK, dV, B, H, H, N, d, causal, scale, workspace, workspace_bytes, stream);
+}
+
+ATTN_EXPORT int attn_bwd_dq(const void* Q, const void* K, const void* V, const void* dO, void* dQ, int64_t B,
+                            int64_t H, int64_t N, int64_t d, int causal, float scale, const void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  return dq_impl(Q, K, V, dO, dQ, B, H, H, N, d, causal, scale, workspace, workspace_bytes, stream);
+}
+
+ATTN_EXPORT int attn_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
+                         void* dQ, void* dK, void* dV, int64_t B, int64_t H, int64_t N, int64_t d, int causal,
+                         float scale, void* workspace, size_t workspace_bytes, void* stream) {
+  return bwd_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, H, N, d, causal, scale, workspace, workspace_bytes, stream);
+}
+
+ATTN_EXPORT int attn_bwd_gqa(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                             const float* LSE, void* dQ, void* dK, void* dV, int64_t B, int64_t H, int64_t H_kv,
+                             int64_t N, int64_t d, int causal, float scale, void* workspace, size_t workspace_bytes,
+                             void* stream) {
+  return bwd_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, H_kv, N, d, causal, scale, workspace, workspace_bytes,
+                  stream);
 }
 
 }  // extern "C"

@@ -69,11 +69,14 @@ attn_bwd_pre_kernel(const __nv_bfloat16* __restrict__ O, const __nv_bfloat16* __
 }
 
 struct BwdParams {
-  const float* ws_lse2;   // [BH][npad]
-  const float* ws_d;      // [BH][npad]
+  const float* ws_lse2;   // [B*H][npad]
+  const float* ws_d;      // [B*H][npad]
   int n;
   int npad;
   int n_tiles;            // ceil(N / 128)
+  int h;                  // query heads per batch
+  int h_kv;               // key/value heads per batch (h % h_kv == 0)
+  int group;              // h / h_kv
   float scale;
   float scale_log2;
 };
@@ -195,11 +198,13 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int nt = prm.n_tiles;
-  const int bh = blockIdx.x / nt;
+  const int bkv = blockIdx.x / nt;             // key/value head
   const int jt = blockIdx.x % nt;              // key tile; small jt = most work under the causal mask
   const int n0 = jt * 128;
   const int i_start = CAUSAL ? jt : 0;
-  const int n_it = nt - i_start;
+  const int n_q = nt - i_start;                // query tiles per query head
+  const int n_it = prm.group * n_q;            // every query head sharing this key/value head
+  const int bq0 = (bkv / prm.h_kv) * prm.h + (bkv % prm.h_kv) * prm.group;   // first such query head
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < QS; ++s) {
@@ -237,17 +242,18 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     if (lane == 0) {
       mbar_arrive_expect_tx(kv_full, 2 * C::kTileBytes);
       for (int b = 0; b < C::kNumBlk; ++b) {
-        tma_load_3d(&tm_k, kv_full, smem + C::kKV_OffK + b * C::kBlockBytes, b * 64, n0, bh);
-        tma_load_3d(&tm_v, kv_full, smem + C::kKV_OffV + b * C::kBlockBytes, b * 64, n0, bh);
+        tma_load_3d(&tm_k, kv_full, smem + C::kKV_OffK + b * C::kBlockBytes, b * 64, n0, bkv);
+        tma_load_3d(&tm_v, kv_full, smem + C::kKV_OffV + b * C::kBlockBytes, b * 64, n0, bkv);
       }
       int q_issued = 0, o_issued = 0, v_issued = 0;
       for (int it = 0; it < n_it; ++it) {
-        const int qi = i_start + it;
+        const int qi = i_start + it % n_q;
+        const int bq = bq0 + it / n_q;
         {   // LSE*log2(e) and D of query tile i
           const int slot = it % VS, use = it / VS;
           if (use > 0 && !mbar_wait(&v_empty[slot], (use - 1) & 1, abort_flag)) break;
           mbar_arrive_expect_tx(&v_full[slot], 2 * C::kVecBytes);
-          const size_t voff = size_t(bh) * size_t(prm.npad) + size_t(qi) * 128;
+          const size_t voff = size_t(bq) * size_t(prm.npad) + size_t(qi) * 128;
           uint8_t* vec = smem + C::kKV_OffVec + slot * 2 * C::kVecBytes;
           bulk_load(vec, prm.ws_lse2 + voff, C::kVecBytes, &v_full[slot]);
           bulk_load(vec + C::kVecBytes, prm.ws_d + voff, C::kVecBytes, &v_full[slot]);
@@ -259,7 +265,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           mbar_arrive_expect_tx(&q_full[slot], C::kTileBytes);
           for (int b = 0; b < C::kNumBlk; ++b)
             tma_load_3d(&tm_q, &q_full[slot], smem + C::kKV_OffQ + slot * C::kTileBytes + b * C::kBlockBytes, b * 64,
-                        qi * 128, bh);
+                        qi * 128, bq);
           ++q_issued;
         }
         {   // dO_i
@@ -268,7 +274,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
           mbar_arrive_expect_tx(&o_full[slot], C::kTileBytes);
           for (int b = 0; b < C::kNumBlk; ++b)
             tma_load_3d(&tm_do, &o_full[slot], smem + C::kKV_OffDO + slot * C::kTileBytes + b * C::kBlockBytes, b * 64,
-                        qi * 128, bh);
+                        qi * 128, bq);
           ++o_issued;
         }
       }
@@ -355,7 +361,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const float c = prm.scale_log2;
     bool ok = true;
     for (int it = 0; it < n_it; ++it) {
-      const int qi = i_start + it;
+      const int qi = i_start + it % n_q;
       const float* vec = reinterpret_cast<const float*>(smem + C::kKV_OffVec + (it % VS) * 2 * C::kVecBytes);
       // LSE/D vectors of this query tile (released below, after the dS reads).
       if (!(ok = mbar_wait_warp(&v_full[it % VS], (it / VS) & 1, abort_flag))) break;
@@ -425,7 +431,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     named_barrier_sync(1 + g, 128);
     if (qw == 0 && lane == 0 && *abort_flag == 0) {
       const CUtensorMap* tm = (g == 0) ? &tm_dv : &tm_dk;
-      for (int b = 0; b < C::kNumBlk; ++b) tma_store_3d(tm, stage + b * C::kBlockBytes, b * 64, n0, bh);
+      for (int b = 0; b < C::kNumBlk; ++b) tma_store_3d(tm, stage + b * C::kBlockBytes, b * 64, n0, bkv);
       bulk_commit_group();
       bulk_wait_group_read0();
     }
@@ -474,7 +480,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   const int lane = threadIdx.x & 31;
   const int n = prm.n;
   const int nt = prm.n_tiles;
-  const int bh = blockIdx.x / nt;
+  const int bh = blockIdx.x / nt;                                             // query head
+  const int bkv = (bh / prm.h) * prm.h_kv + (bh % prm.h) / prm.group;        // its key/value head
   const int it_q = nt - 1 - (blockIdx.x % nt);   // query tile; large = most work under the causal mask
   const int m0 = it_q * 128;
   const int n_it = CAUSAL ? it_q + 1 : nt;
@@ -525,7 +532,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           mbar_arrive_expect_tx(&k_full[slot], C::kTileBytes);
           for (int b = 0; b < C::kNumBlk; ++b)
             tma_load_3d(&tm_k, &k_full[slot], smem + C::kQ_OffK + slot * C::kTileBytes + b * C::kBlockBytes, b * 64,
-                        it * 128, bh);
+                        it * 128, bkv);
           ++k_issued;
         }
         {
@@ -534,7 +541,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           mbar_arrive_expect_tx(&v_full[slot], C::kTileBytes);
           for (int b = 0; b < C::kNumBlk; ++b)
             tma_load_3d(&tm_v, &v_full[slot], smem + C::kQ_OffV + slot * C::kTileBytes + b * C::kBlockBytes, b * 64,
-                        it * 128, bh);
+                        it * 128, bkv);
           ++v_issued;
         }
       }

@@ -34,9 +34,12 @@ constexpr float kRescaleLog2 = 8.0f;
 constexpr float kLn2 = 0.6931471805599453f;
 
 struct FwdParams {
-  float* lse;          // [BH][N] natural-log LSE
+  float* lse;          // [B*H][N] natural-log LSE
   int n;               // sequence length N
   int n_mblk;          // number of 256-row query blocks per head
+  int h;               // query heads per batch
+  int h_kv;            // key/value heads per batch (h % h_kv == 0)
+  int group;           // h / h_kv query heads share one key/value head
   float scale_log2;    // scale * log2(e)
 };
 
@@ -83,7 +86,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int n = prm.n;
-  const int bh = blockIdx.x / prm.n_mblk;
+  const int bh = blockIdx.x / prm.n_mblk;                                      // query head
+  const int bkv = (bh / prm.h) * prm.h_kv + (bh % prm.h) / prm.group;          // its key/value head
   const int m_blk = prm.n_mblk - 1 - (blockIdx.x % prm.n_mblk);   // heaviest causal blocks first
   const int m0 = m_blk * 256;
   const int n_kv_total = (n + 127) >> 7;
@@ -139,7 +143,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mbar_arrive_expect_tx(&kv_full[slot], C::kTileBytes);
         for (int b = 0; b < C::kNumBlk; ++b)
           tma_load_3d(tm, &kv_full[slot], smem + C::kOffKV + slot * C::kTileBytes + b * C::kBlockBytes,
-                      b * 64, 128 * j, bh);
+                      b * 64, 128 * j, bkv);
         ++issued;
       }
       (void)ok;
@@ -294,18 +298,20 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
       l *= alpha;
       const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
+      // P in 32-key chunks (16 packed columns each): a chunk's registers are
+      // free again as soon as it is stored, which keeps the loop spill-free.
       float sump[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        uint32_t pk[32];
+      for (int q = 0; q < 4; ++q) {
+        uint32_t pk[16];
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          const float p0 = ex2(fmaf(s[h * 64 + 2 * k], c, neg_m));
-          const float p1 = ex2(fmaf(s[h * 64 + 2 * k + 1], c, neg_m));
+        for (int k = 0; k < 16; ++k) {
+          const float p0 = ex2(fmaf(s[32 * q + 2 * k], c, neg_m));
+          const float p1 = ex2(fmaf(s[32 * q + 2 * k + 1], c, neg_m));
           sump[k & 3] += p0 + p1;
           pk[k] = pack_bf16x2(p0, p1);
         }
-        tmem_st32(tP + h * 32, pk);
+        tmem_st16(tP + 16 * q, pk);
       }
       l += (sump[0] + sump[1]) + (sump[2] + sump[3]);
       if (__any_sync(0xffffffffu, rescale)) {

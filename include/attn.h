@@ -71,6 +71,19 @@ int attn_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE,
              void* stream);
 
 /*
+ * Forward with shared key/value heads (grouped-query / multi-query attention):
+ * H query heads, H_kv key/value heads, H % H_kv == 0; query head h of batch b
+ * attends with key/value head h / (H / H_kv) of batch b.  Head sharing changes
+ * how many key/value heads exist while the kernel still tiles over them
+ * ("Attention and KV Compression", section "The composability point").
+ * Q, O: [B][H][N][d]; K, V: [B][H_kv][N][d]; LSE: [B][H][N].  attn_fwd is this
+ * call with H_kv = H.
+ */
+int attn_fwd_gqa(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                 int64_t B, int64_t H, int64_t H_kv, int64_t N, int64_t d, int causal, float scale,
+                 void* stream);
+
+/*
  * Bytes of caller-provided device workspace that attn_bwd needs for these
  * sizes (two fp32 per-row vectors per head, each padded to a multiple of 128
  * rows).  Returns 0 for sizes that attn_bwd would reject.
@@ -96,6 +109,19 @@ int attn_bwd(const void* Q, const void* K, const void* V, const void* O, const v
              const float* LSE, void* dQ, void* dK, void* dV,
              int64_t B, int64_t H, int64_t N, int64_t d, int causal, float scale,
              void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Backward with shared key/value heads (see attn_fwd_gqa for the layout).
+ * dQ: [B][H][N][d]; dK, dV: [B][H_kv][N][d], each the sum over the H / H_kv
+ * query heads that share the key/value head (the dK/dV kernel loops over
+ * those query heads, so the sum is formed in tensor memory without atomics).
+ * The workspace is sized by attn_bwd_workspace_bytes(B, H, N, d) (query heads).
+ * attn_bwd is this call with H_kv = H.
+ */
+int attn_bwd_gqa(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                 const float* LSE, void* dQ, void* dK, void* dV,
+                 int64_t B, int64_t H, int64_t H_kv, int64_t N, int64_t d, int causal, float scale,
+                 void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * The three steps of attn_bwd, callable one at a time (same arguments and

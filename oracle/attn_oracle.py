@@ -47,6 +47,9 @@ __all__ = [
     "attn_fwd",
     "attn_fwd_rows",
     "attn_bwd",
+    "expand_kv",
+    "attn_fwd_gqa",
+    "attn_bwd_gqa",
 ]
 
 
@@ -148,4 +151,37 @@ def attn_bwd(Q, K, V, dO, scale: float, causal: bool):
         del dp, p
         dQ[h] = float(scale) * (ds @ K[h])
         dK[h] = float(scale) * (ds.T @ Q[h])
+    return dQ, dK, dV
+
+
+# ---------------------------------------------------------------------------
+# Shared key/value heads (grouped-query / multi-query attention): H query heads
+# and H_kv key/value heads per batch, query head h using key/value head
+# h // (H // H_kv) ("Attention and KV Compression", section "The
+# composability point": head sharing changes how many key/value heads exist).
+# By definition this is multi-head attention on keys/values repeated to H
+# heads; the gradient of a shared key/value head is the sum of the gradients
+# of its copies (chain rule through the repetition).
+# ---------------------------------------------------------------------------
+
+def expand_kv(X, B: int, H: int, H_kv: int):
+    """(B*H_kv, N, d) -> (B*H, N, d): row b*H + h is X[b*H_kv + h // (H // H_kv)]."""
+    X = _as3(X)
+    g = H // H_kv
+    idx = np.array([b * H_kv + h // g for b in range(B) for h in range(H)], dtype=np.int64)
+    return X[idx]
+
+
+def attn_fwd_gqa(Q, K, V, scale: float, causal: bool, B: int, H: int, H_kv: int):
+    """Forward with shared key/value heads: O, LSE of shape (B*H, N, d), (B*H, N)."""
+    return attn_fwd(Q, expand_kv(K, B, H, H_kv), expand_kv(V, B, H, H_kv), scale, causal)
+
+
+def attn_bwd_gqa(Q, K, V, dO, scale: float, causal: bool, B: int, H: int, H_kv: int):
+    """Backward with shared key/value heads: dQ (B*H, N, d); dK, dV (B*H_kv, N, d)."""
+    dQ, dKe, dVe = attn_bwd(Q, expand_kv(K, B, H, H_kv), expand_kv(V, B, H, H_kv), dO, scale, causal)
+    g = H // H_kv
+    n, d = dKe.shape[1:]
+    dK = dKe.reshape(B, H_kv, g, n, d).sum(axis=2).reshape(B * H_kv, n, d)
+    dV = dVe.reshape(B, H_kv, g, n, d).sum(axis=2).reshape(B * H_kv, n, d)
     return dQ, dK, dV

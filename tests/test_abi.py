@@ -81,6 +81,18 @@ def test_fwd_argument_errors(lib):
         assert _fwd(lib, ptrs=p) == attn.ATTN_ERR_MISALIGNED
 
 
+def test_gqa_argument_errors(lib):
+    p = [A] * 5
+    # H must be a multiple of H_kv, and 1 <= H_kv <= H
+    assert lib.attn_fwd_gqa(*p, 1, 4, 3, 128, 64, 0, 0.125, None) == attn.ATTN_ERR_INVALID_ARG
+    assert lib.attn_fwd_gqa(*p, 1, 4, 0, 128, 64, 0, 0.125, None) == attn.ATTN_ERR_INVALID_ARG
+    assert lib.attn_fwd_gqa(*p, 1, 4, 8, 128, 64, 0, 0.125, None) == attn.ATTN_ERR_INVALID_ARG
+    ws = attn.attn_bwd_workspace_bytes(1, 4, 128, 64)
+    assert lib.attn_bwd_gqa(*([A] * 9), 1, 4, 3, 128, 64, 1, 0.125, A, ws, None) == attn.ATTN_ERR_INVALID_ARG
+    p[1] = MIS
+    assert lib.attn_fwd_gqa(*p, 1, 4, 2, 128, 64, 0, 0.125, None) == attn.ATTN_ERR_MISALIGNED
+
+
 def test_bwd_argument_errors(lib):
     ws = attn.attn_bwd_workspace_bytes(1, 1, 128, 64)
 

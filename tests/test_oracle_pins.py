@@ -406,3 +406,80 @@ def test_planted_mistakes_are_caught(mutant, monkeypatch):
     mod.attn_fwd = attn_fwd
     _MUTANTS[mutant](mod)
     assert not _pins_hold(mod), f"planted mistake {mutant!r} was not caught by any pin"
+
+
+# ---------------------------------------------------------------------------
+# Shared key/value heads
+# ---------------------------------------------------------------------------
+
+def test_gqa_with_one_query_head_per_kv_head_is_mha():
+    B, H, N, d = 2, 3, 9, 4
+    q, k, v, g = (_rand((B * H, N, d), 300 + i) for i in range(4))
+    O1, L1 = orc.attn_fwd_gqa(q, k, v, 0.4, True, B, H, H)
+    O2, L2 = orc.attn_fwd(q, k, v, 0.4, True)
+    np.testing.assert_array_equal(O1, O2)
+    np.testing.assert_array_equal(L1, L2)
+    a = orc.attn_bwd_gqa(q, k, v, g, 0.4, True, B, H, H)
+    b = orc.attn_bwd(q, k, v, g, 0.4, True)
+    for x, y in zip(a, b):
+        np.testing.assert_array_equal(x, y)
+
+
+def test_gqa_heads_read_their_shared_kv_head():
+    # query head h of batch b must see exactly key/value head b*H_kv + h // G:
+    # give every key/value head a constant, distinct value row and check O.
+    B, H, H_kv, N, d = 2, 6, 2, 7, 3
+    q, k = _rand((B * H, N, d), 310), _rand((B * H_kv, N, d), 311)
+    v = np.zeros((B * H_kv, N, d))
+    for j in range(B * H_kv):
+        v[j] = float(j + 1)
+    O, _ = orc.attn_fwd_gqa(q, k, v, 0.5, False, B, H, H_kv)
+    for b in range(B):
+        for h in range(H):
+            np.testing.assert_allclose(O[b * H + h], b * H_kv + h // (H // H_kv) + 1.0, rtol=1e-14)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_gqa_backward_matches_central_differences(causal):
+    B, H, H_kv, N, d, scale = 1, 4, 2, 5, 3, 0.45
+    q, g = _rand((B * H, N, d), 320), _rand((B * H, N, d), 321)
+    k, v = _rand((B * H_kv, N, d), 322), _rand((B * H_kv, N, d), 323)
+    dQ, dK, dV = orc.attn_bwd_gqa(q, k, v, g, scale, causal, B, H, H_kv)
+    assert dK.shape == k.shape and dV.shape == v.shape and dQ.shape == q.shape
+
+    def loss(q_, k_, v_):
+        O, _ = orc.attn_fwd_gqa(q_, k_, v_, scale, causal, B, H, H_kv)
+        return float(np.sum(O * g))
+
+    h = 1e-6
+    for name, x, grad in (("q", q, dQ), ("k", k, dK), ("v", v, dV)):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(*x.shape):
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args_p = {"q": q, "k": k, "v": v}; args_p[name] = xp
+            args_m = {"q": q, "k": k, "v": v}; args_m[name] = xm
+            num[idx] = (loss(**{kk + "_": vv for kk, vv in args_p.items()})
+                        - loss(**{kk + "_": vv for kk, vv in args_m.items()})) / (2 * h)
+        np.testing.assert_allclose(grad, num, rtol=0, atol=1e-7 * max(1.0, np.abs(num).max()), err_msg=name)
+
+
+def test_gqa_matches_torch_autograd_fp64():
+    torch = pytest.importorskip("torch")
+    B, H, H_kv, N, d, scale = 2, 4, 1, 11, 8, 0.3
+    q, g = _rand((B * H, N, d), 330), _rand((B * H, N, d), 331)
+    k, v = _rand((B * H_kv, N, d), 332), _rand((B * H_kv, N, d), 333)
+    dQ, dK, dV = orc.attn_bwd_gqa(q, k, v, g, scale, True, B, H, H_kv)
+    tq = torch.tensor(q.reshape(B, H, N, d), requires_grad=True)
+    tk = torch.tensor(k.reshape(B, H_kv, N, d), requires_grad=True)
+    tv = torch.tensor(v.reshape(B, H_kv, N, d), requires_grad=True)
+    ke = tk.repeat_interleave(H // H_kv, dim=1)
+    ve = tv.repeat_interleave(H // H_kv, dim=1)
+    s = scale * tq @ ke.transpose(-1, -2)
+    s = s.masked_fill(torch.ones(N, N, dtype=torch.bool).triu(1), float("-inf"))
+    o = torch.softmax(s, dim=-1) @ ve
+    o.backward(torch.tensor(g.reshape(B, H, N, d)))
+    np.testing.assert_allclose(dQ, tq.grad.numpy().reshape(B * H, N, d), rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(dK, tk.grad.numpy().reshape(B * H_kv, N, d), rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(dV, tv.grad.numpy().reshape(B * H_kv, N, d), rtol=1e-11, atol=1e-12)

@@ -239,6 +239,8 @@ def run_ours(args, rank, world, local_rank):
                 "frac": round(achieved / sustained, 4), "frac_of_burst": round(achieved / burst, 4),
                 "traffic": recorded_traffic(dom)}
 
+    peak_mem = torch.cuda.max_memory_allocated(dev)
+
     # ------------------------------------------------- shared key/value heads
     gqa = None
     if not args.no_gqa and w.H % args.gqa_kv_heads == 0:
@@ -380,7 +382,7 @@ def run_ours(args, rank, world, local_rank):
         "clocks": clk,
         "e2e": e2e,
         "cpu_baseline": cpu,
-        "peak_mem_gib": round(torch.cuda.max_memory_allocated(dev) / 2**30, 3),
+        "peak_mem_gib": round(peak_mem / 2**30, 3),
         "naive_score_bytes_per_layer": 2 * w.N * w.N * w.B * w.H,
     }
     return line

@@ -275,6 +275,95 @@ def run_ours(args, rank, world, local_rank):
                "fwdbwd_tflops": round(aggregate_tflops(3.5 * f_fwd, world, gf + gb), 2), "steps": n_g}
         del kg, vg, dkg, dvg
 
+    # ------------------------------------------------- block-sparse selection
+    sparse = None
+    if not args.no_sparse:
+        import numpy as np
+        nt = (w.N + 127) // 128
+        ii, jj = np.meshgrid(np.arange(nt), np.arange(nt), indexing="ij")
+        sel = ((ii - jj >= 0) & (ii - jj < args.sparse_window)) | (jj < args.sparse_sink)
+        sel &= jj <= ii                                    # causal: tiles above the diagonal are never visible
+        # visible score entries: full tiles below the diagonal, 128*129/2 on it
+        vis = float(np.sum(np.where(ii == jj, 128 * 129 / 2, 128 * 128) * sel))
+        f_sparse = 4.0 * w.d * vis * w.B * w.H
+        mask = torch.from_numpy(np.broadcast_to(sel.astype(np.uint8), (w.B, w.H, nt, nt)).copy()).to(dev)
+
+        def sparse_step(ev=None):
+            if ev is not None:
+                ev[0].record(stream)
+            attn.attn_fwd_blocksparse(q, k, v, o, lse, mask, causal, scale, stream)
+            if ev is not None:
+                ev[1].record(stream)
+            attn.attn_bwd_blocksparse(q, k, v, o, do, lse, mask, dq, dk, dv, causal, scale, ws, stream)
+            if ev is not None:
+                ev[2].record(stream)
+
+        for _ in range(args.warmup):
+            sparse_step()
+        n_s = max(3, min(args.steps, 5))
+        sev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_s)]
+        torch.cuda.synchronize()
+        for e in sev:
+            sparse_step(e)
+        torch.cuda.synchronize()
+        assert attn.attn_check_status(stream) == attn.ATTN_OK
+        sf = sum(e[0].elapsed_time(e[1]) for e in sev) / n_s
+        sb = sum(e[1].elapsed_time(e[2]) for e in sev) / n_s
+        sf, sb = max_over_ranks([sf, sb], device=dev)
+        sparse = {"pattern": f"causal sliding window of {args.sparse_window} key tiles + first {args.sparse_sink} tiles",
+                  "tile_density_vs_causal": round(float(sel.sum()) / float((jj <= ii).sum()), 4),
+                  "ms_fwd": round(sf, 3), "ms_bwd": round(sb, 3),
+                  "fwd_tflops": round(aggregate_tflops(f_sparse, world, sf), 2),
+                  "fwdbwd_tflops": round(aggregate_tflops(3.5 * f_sparse, world, sf + sb), 2), "steps": n_s}
+        del mask
+
+    # ------------------------------------------- decode against a KV cache
+    # One new query row per head of the same batch against a cache of N rows
+    # held in H_kv shared key/value heads: HBM-bound (each cache byte is used
+    # by H / H_kv query rows), so its roofline is the measured copy bandwidth.
+    kvcache = None
+    if not args.no_kvcache and w.H % args.gqa_kv_heads == 0:
+        hk = args.gqa_kv_heads
+        kc, vc = k[:, :hk].contiguous(), v[:, :hk].contiguous()
+        qd = q[:, :, -1:].contiguous()
+        od = torch.empty_like(qd)
+        lsed = torch.empty((w.B, w.H, 1), dtype=torch.float32, device=dev)
+        gen = torch.Generator("cpu").manual_seed(rank_seed(99, rank))
+        lens_var = torch.randint(w.N // 2, w.N + 1, (w.B,), generator=gen, dtype=torch.int32)
+        hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        kvcache = {"workload": f"decode: B={w.B}, H={w.H}, H_kv={hk}, Nq=1, Nk={w.N}, d={w.d}, causal",
+                   "peak_gbs": hbm, "peak_kind": f"hbm_gbs ({peaks_src})"}
+        for name, lens in (("full", None), ("varlen", lens_var)):
+            lens_dev = None if lens is None else lens.to(dev)
+            splits = attn.attn_fwd_kvcache_splits(w.B, w.H, hk, 1, w.N, w.d, 0)
+            wsb = attn.attn_fwd_kvcache_workspace_bytes(w.B, w.H, hk, 1, w.N, w.d, 0)
+            wsd = torch.empty((max(wsb, 16) // 4,), dtype=torch.float32, device=dev)
+            rows_read = w.B * w.N if lens is None else int(lens.sum())
+            alg_bytes = rows_read * hk * w.d * 2 * 2 + 2 * qd.numel() * 2 + lsed.numel() * 4
+
+            def dec():
+                attn.attn_fwd_kvcache(qd, kc, vc, od, lsed, lens_dev, causal, scale, 0, wsd, stream)
+
+            for _ in range(max(3, args.warmup)):
+                dec()
+            n_d = 20
+            dev_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n_d)]
+            torch.cuda.synchronize()
+            for e in dev_ev:
+                e[0].record(stream)
+                dec()
+                e[1].record(stream)
+            torch.cuda.synchronize()
+            assert attn.attn_check_status(stream) == attn.ATTN_OK
+            t_us = sum(e[0].elapsed_time(e[1]) for e in dev_ev) / n_d * 1e3
+            t_us = max_over_ranks([t_us], device=dev)[0]
+            gbs = alg_bytes / (t_us * 1e-6) / 1e9
+            kvcache[name] = {"splits": splits, "us": round(t_us, 2), "alg_bytes": alg_bytes,
+                             "gb_s": round(gbs, 1), "frac": round(gbs / hbm, 4), "calls": n_d,
+                             "kv_lens": None if lens is None else "uniform in [N/2, N] per batch entry"}
+            del wsd
+        del kc, vc
+
     # ---------------------------------------------------------------- e2e
     # Through host buffers: every step copies its inputs Q, K, V, dO from
     # pinned host memory to the device and its results O, LSE, dQ, dK, dV back.
@@ -378,6 +467,8 @@ def run_ours(args, rank, world, local_rank):
         "kernel_ms": {kname: round(t, 3) for kname, t in per_kernel.items()},
         "roofline": roofline,
         "gqa": gqa,
+        "block_sparse": sparse,
+        "kvcache": kvcache,
         "gpu_launches": 4 * args.steps,
         "clocks": clk,
         "e2e": e2e,
@@ -468,7 +559,11 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-gqa", action="store_true", help="skip the shared key/value head measurement")
+    ap.add_argument("--no-kvcache", action="store_true", help="skip the decode (key/value cache) measurement")
     ap.add_argument("--gqa-kv-heads", type=int, default=8)
+    ap.add_argument("--no-sparse", action="store_true", help="skip the block-sparse measurement")
+    ap.add_argument("--sparse-window", type=int, default=16)
+    ap.add_argument("--sparse-sink", type=int, default=2)
     ap.add_argument("--cpu-rows", type=int, default=16384)
     ap.add_argument("--ref-rows", type=int, default=8192)
     ap.add_argument("--batch", type=int, default=0, help="override B (profiling captures only)")

@@ -30,9 +30,12 @@ ATTN_ERR_LAUNCH = -5
 ATTN_ERR_TIMEOUT = -6
 ATTN_ERR_DEVICE = -7
 
-EXPORTED = ("attn_fwd", "attn_fwd_gqa", "attn_bwd", "attn_bwd_gqa", "attn_bwd_workspace_bytes",
+EXPORTED = ("attn_fwd", "attn_fwd_gqa", "attn_fwd_blocksparse", "attn_bwd", "attn_bwd_gqa", "attn_bwd_blocksparse",
+            "attn_bwd_workspace_bytes", "attn_fwd_kvcache", "attn_fwd_kvcache_splits",
+            "attn_fwd_kvcache_workspace_bytes",
             "attn_bwd_preprocess", "attn_bwd_dkdv",
             "attn_bwd_dq", "attn_bwd_static_workspace", "attn_check_status", "attn_last_error",
+            "attn_selftest_wait_timeout",
             "attn_status_string")
 
 # Size of the library-owned workspace used by attn_bwd_static_workspace (bytes).
@@ -67,6 +70,18 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.attn_bwd_gqa.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i32, f32, vp,
                                  ctypes.c_size_t, vp]
     lib.attn_bwd_gqa.restype = i32
+    lib.attn_fwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i32, f32, vp]
+    lib.attn_fwd_blocksparse.restype = i32
+    lib.attn_bwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i32, f32,
+                                         vp, ctypes.c_size_t, vp]
+    lib.attn_bwd_blocksparse.restype = i32
+    lib.attn_fwd_kvcache.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i32, f32, i64, vp,
+                                     ctypes.c_size_t, vp]
+    lib.attn_fwd_kvcache.restype = i32
+    lib.attn_fwd_kvcache_splits.argtypes = [i64] * 7
+    lib.attn_fwd_kvcache_splits.restype = i64
+    lib.attn_fwd_kvcache_workspace_bytes.argtypes = [i64] * 7
+    lib.attn_fwd_kvcache_workspace_bytes.restype = ctypes.c_size_t
     lib.attn_bwd_workspace_bytes.argtypes = [i64, i64, i64, i64]
     lib.attn_bwd_workspace_bytes.restype = ctypes.c_size_t
     lib.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, f32, vp,
@@ -80,6 +95,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.attn_bwd_dq.restype = i32
     lib.attn_bwd_static_workspace.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, f32, vp]
     lib.attn_bwd_static_workspace.restype = i32
+    lib.attn_selftest_wait_timeout.argtypes = [vp]
+    lib.attn_selftest_wait_timeout.restype = i32
     lib.attn_check_status.argtypes = [vp]
     lib.attn_check_status.restype = i32
     lib.attn_last_error.argtypes = []
@@ -180,6 +197,89 @@ def attn_bwd_gqa(Q, K, V, O, dO, LSE, dQ, dK, dV, causal: bool, scale: float, wo
         raise AttnError(st, "attn_bwd_gqa")
 
 
+def _check_mask(mask, B, H, N):
+    nt = (N + 127) // 128
+    if not mask.is_cuda or mask.dtype != torch.uint8 or not mask.is_contiguous() or \
+            tuple(mask.shape) != (B, H, nt, nt):
+        raise ValueError(f"block_mask must be a contiguous CUDA uint8 tensor of shape {(B, H, nt, nt)}")
+
+
+def attn_fwd_blocksparse(Q, K, V, O, LSE, block_mask, causal: bool, scale: float, stream=None) -> None:
+    """attn_fwd over the 128x128 blocks selected by block_mask (B, H, ceil(N/128), ceil(N/128))."""
+    _check_bhnd("Q", Q)
+    _check_bhnd("O", O, Q.shape)
+    Hk = _check_kv("K", K, Q.shape)
+    if _check_kv("V", V, Q.shape) != Hk:
+        raise ValueError("K and V must have the same number of heads")
+    _check_lse(LSE, Q.shape)
+    B, H, N, d = Q.shape
+    _check_mask(block_mask, B, H, N)
+    st = load_library().attn_fwd_blocksparse(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE), _ptr(block_mask), B, H,
+                                             Hk, N, d, int(bool(causal)), float(scale), _stream_handle(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd_blocksparse")
+
+
+def attn_bwd_blocksparse(Q, K, V, O, dO, LSE, block_mask, dQ, dK, dV, causal: bool, scale: float, workspace,
+                         stream=None) -> None:
+    """Backward of attn_fwd_blocksparse."""
+    _check_bhnd("Q", Q)
+    for n, t in (("O", O), ("dO", dO), ("dQ", dQ)):
+        _check_bhnd(n, t, Q.shape)
+    Hk = _check_kv("K", K, Q.shape)
+    for n, t in (("V", V), ("dK", dK), ("dV", dV)):
+        if _check_kv(n, t, Q.shape) != Hk:
+            raise ValueError(f"{n} must have the same number of heads as K")
+    _check_lse(LSE, Q.shape)
+    B, H, N, d = Q.shape
+    _check_mask(block_mask, B, H, N)
+    wp, wb = _ws(workspace)
+    st = load_library().attn_bwd_blocksparse(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(dO), _ptr(LSE),
+                                             _ptr(block_mask), _ptr(dQ), _ptr(dK), _ptr(dV), B, H, Hk, N, d,
+                                             int(bool(causal)), float(scale), wp, wb, _stream_handle(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_bwd_blocksparse")
+
+
+def attn_fwd_kvcache_splits(B: int, H: int, H_kv: int, Nq: int, Nk: int, d: int, num_splits: int = 0) -> int:
+    return int(load_library().attn_fwd_kvcache_splits(B, H, H_kv, Nq, Nk, d, num_splits))
+
+
+def attn_fwd_kvcache_workspace_bytes(B: int, H: int, H_kv: int, Nq: int, Nk: int, d: int,
+                                     num_splits: int = 0) -> int:
+    return int(load_library().attn_fwd_kvcache_workspace_bytes(B, H, H_kv, Nq, Nk, d, num_splits))
+
+
+def attn_fwd_kvcache(Q, K, V, O, LSE, kv_lens, causal: bool, scale: float, num_splits: int = 0, workspace=None,
+                     stream=None) -> None:
+    """O, LSE <- attention of Q (B, H, Nq, d) against the cache K, V (B, H_kv, Nk, d).
+
+    kv_lens: int32 CUDA tensor (B,) of valid cache lengths, or None (all Nk).
+    workspace: CUDA tensor of at least attn_fwd_kvcache_workspace_bytes() bytes
+    when more than one split is used (None allowed with one split).
+    """
+    _check_bhnd("Q", Q)
+    _check_bhnd("O", O, Q.shape)
+    _check_lse(LSE, Q.shape)
+    B, H, Nq, d = Q.shape
+    for name, t in (("K", K), ("V", V)):
+        if not t.is_cuda or t.dtype != torch.bfloat16 or t.dim() != 4 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor of shape (B, H_kv, Nk, d)")
+    if K.shape != V.shape or K.shape[0] != B or K.shape[3] != d or K.shape[1] < 1 or H % K.shape[1] != 0:
+        raise ValueError(f"K, V have shapes {tuple(K.shape)}, {tuple(V.shape)}; expected (B, H_kv, Nk, d)")
+    Hk, Nk = K.shape[1], K.shape[2]
+    if kv_lens is not None and (not kv_lens.is_cuda or kv_lens.dtype != torch.int32 or tuple(kv_lens.shape) != (B,)
+                                or not kv_lens.is_contiguous()):
+        raise ValueError("kv_lens must be a contiguous CUDA int32 tensor of shape (B,)")
+    wp, wb = (ctypes.c_void_p(None), 0) if workspace is None else _ws(workspace)
+    st = load_library().attn_fwd_kvcache(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE),
+                                         ctypes.c_void_p(None) if kv_lens is None else _ptr(kv_lens),
+                                         B, H, Hk, Nq, Nk, d, int(bool(causal)), float(scale), int(num_splits),
+                                         wp, wb, _stream_handle(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd_kvcache")
+
+
 def attn_bwd_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
     return int(load_library().attn_bwd_workspace_bytes(B, H, N, d))
 
@@ -257,6 +357,13 @@ def attn_bwd_dq(Q, K, V, dO, dQ, causal: bool, scale: float, workspace, stream=N
                                     int(bool(causal)), float(scale), wp, wb, _stream_handle(stream))
     if st != ATTN_OK:
         raise AttnError(st, "attn_bwd_dq")
+
+
+def attn_selftest_wait_timeout(stream=None) -> None:
+    """Enqueue the failure-path self-test (a bounded wait that runs out)."""
+    st = load_library().attn_selftest_wait_timeout(_stream_handle(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_selftest_wait_timeout")
 
 
 def attn_check_status(stream=None) -> int:

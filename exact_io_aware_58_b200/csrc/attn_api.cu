@@ -6,6 +6,7 @@
 // the caller's workspace, and the only device state is the status word
 // g_attn_status (a static __device__ variable).
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstdio>
@@ -17,6 +18,7 @@
 #include "../../include/attn.h"
 #include "attn_bwd.cuh"
 #include "attn_fwd.cuh"
+#include "attn_kvcache.cuh"
 
 namespace {
 
@@ -46,9 +48,9 @@ EncodeTiledFn encode_fn() {
 }
 
 // 3-D map over a BHND bf16 tensor viewed as [B*H][N][d]; box = 64 columns x
-// 128 rows x 1 head, 128-byte swizzle.  Rows past N read as zeros; stores
+// box_rows rows x 1 head, 128-byte swizzle.  Rows past N read as zeros; stores
 // past N are dropped.
-bool make_map(CUtensorMap* m, const void* base, int64_t bh, int64_t n, int64_t d) {
+bool make_map(CUtensorMap* m, const void* base, int64_t bh, int64_t n, int64_t d, int box_rows = 128) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) {
     fail(ATTN_ERR_LAUNCH, "%sdriver entry point cuTensorMapEncodeTiled unavailable%lld", "", 0);
@@ -56,7 +58,7 @@ bool make_map(CUtensorMap* m, const void* base, int64_t bh, int64_t n, int64_t d
   }
   const cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(n), cuuint64_t(bh)};
   const cuuint64_t strides[2] = {cuuint64_t(d * 2), cuuint64_t(n * d * 2)};
-  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t box[3] = {64, cuuint32_t(box_rows), 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -100,31 +102,31 @@ int set_smem(const void* kern, int bytes) {
               (long long)bytes);
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool SPARSE>
 int launch_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const CUtensorMap& o,
                const attn::FwdParams& prm, int grid, cudaStream_t st) {
-  auto kern = attn::attn_fwd_kernel<D, CAUSAL>;
+  auto kern = attn::attn_fwd_kernel<D, CAUSAL, SPARSE>;
   constexpr int smem = attn::FwdCfg<D>::kSmemBytes;
   if (set_smem(reinterpret_cast<const void*>(kern), smem) != ATTN_OK) return ATTN_ERR_LAUNCH;
   kern<<<grid, attn::FwdCfg<D>::kThreads, smem, st>>>(q, k, v, o, prm);
   return launch_status();
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool SPARSE>
 int launch_dkdv(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const CUtensorMap& dO,
                 const CUtensorMap& dk, const CUtensorMap& dv, const attn::BwdParams& prm, int grid, cudaStream_t st) {
   using C = attn::BwdCfg<D>;
-  auto kern = attn::attn_bwd_dkdv_kernel<D, CAUSAL>;
+  auto kern = attn::attn_bwd_dkdv_kernel<D, CAUSAL, SPARSE>;
   if (set_smem(reinterpret_cast<const void*>(kern), C::kKV_SmemBytes) != ATTN_OK) return ATTN_ERR_LAUNCH;
   kern<<<grid, C::kThreads, C::kKV_SmemBytes, st>>>(q, k, v, dO, dk, dv, prm);
   return launch_status();
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool SPARSE>
 int launch_dq(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const CUtensorMap& dO,
               const CUtensorMap& dq, const attn::BwdParams& prm, int grid, cudaStream_t st) {
   using C = attn::BwdCfg<D>;
-  auto kern = attn::attn_bwd_dq_kernel<D, CAUSAL>;
+  auto kern = attn::attn_bwd_dq_kernel<D, CAUSAL, SPARSE>;
   if (set_smem(reinterpret_cast<const void*>(kern), C::kQ_SmemBytes) != ATTN_OK) return ATTN_ERR_LAUNCH;
   kern<<<grid, C::kThreads, C::kQ_SmemBytes, st>>>(q, k, v, dO, dq, prm);
   return launch_status();
@@ -144,6 +146,13 @@ int launch_bwd_pre(const void* O, const void* dO, const float* lse, float* ws_ls
 
 int64_t npad_of(int64_t N) { return (N + 127) / 128 * 128; }
 
+// Selects the kernel instance for head dim, causal mask and block sparsity.
+#define ATTN_DISPATCH(FN, ...)                                                                       \
+  (d == 128 ? (causal ? (sparse ? FN<128, true, true>(__VA_ARGS__) : FN<128, true, false>(__VA_ARGS__))  \
+                      : (sparse ? FN<128, false, true>(__VA_ARGS__) : FN<128, false, false>(__VA_ARGS__))) \
+            : (causal ? (sparse ? FN<64, true, true>(__VA_ARGS__) : FN<64, true, false>(__VA_ARGS__))    \
+                      : (sparse ? FN<64, false, true>(__VA_ARGS__) : FN<64, false, false>(__VA_ARGS__))))
+
 }  // namespace
 
 #define ATTN_EXPORT __attribute__((visibility("default")))
@@ -154,8 +163,8 @@ extern "C" {
 
 namespace {
 
-int fwd_impl(const void* Q, const void* K, const void* V, void* O, float* LSE, int64_t B, int64_t H, int64_t H_kv,
-             int64_t N, int64_t d, int causal, float scale, void* stream) {
+int fwd_impl(const void* Q, const void* K, const void* V, void* O, float* LSE, const uint8_t* mask, int64_t B,
+             int64_t H, int64_t H_kv, int64_t N, int64_t d, int causal, float scale, void* stream) {
   int s = check_sizes(B, H, N, d);
   if (s != ATTN_OK) return s;
   if ((s = check_heads(H, H_kv)) != ATTN_OK) return s;
@@ -176,14 +185,13 @@ int fwd_impl(const void* Q, const void* K, const void* V, void* O, float* LSE, i
   prm.h_kv = int(H_kv);
   prm.group = int(H / H_kv);
   prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.mask = mask;
+  prm.nt = int((N + 127) / 128);
+  const bool sparse = mask != nullptr;
   const int64_t grid = bh * prm.n_mblk;
   if (grid > INT32_MAX) return ATTN_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (d == 128)
-    return causal ? launch_fwd<128, true>(mq, mk, mv, mo, prm, int(grid), st)
-                  : launch_fwd<128, false>(mq, mk, mv, mo, prm, int(grid), st);
-  return causal ? launch_fwd<64, true>(mq, mk, mv, mo, prm, int(grid), st)
-                : launch_fwd<64, false>(mq, mk, mv, mo, prm, int(grid), st);
+  return ATTN_DISPATCH(launch_fwd, mq, mk, mv, mo, prm, int(grid), st);
 }
 
 }  // namespace
@@ -192,12 +200,19 @@ extern "C" {
 
 ATTN_EXPORT int attn_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int64_t B, int64_t H,
                          int64_t N, int64_t d, int causal, float scale, void* stream) {
-  return fwd_impl(Q, K, V, O, LSE, B, H, H, N, d, causal, scale, stream);
+  return fwd_impl(Q, K, V, O, LSE, nullptr, B, H, H, N, d, causal, scale, stream);
 }
 
 ATTN_EXPORT int attn_fwd_gqa(const void* Q, const void* K, const void* V, void* O, float* LSE, int64_t B, int64_t H,
                              int64_t H_kv, int64_t N, int64_t d, int causal, float scale, void* stream) {
-  return fwd_impl(Q, K, V, O, LSE, B, H, H_kv, N, d, causal, scale, stream);
+  return fwd_impl(Q, K, V, O, LSE, nullptr, B, H, H_kv, N, d, causal, scale, stream);
+}
+
+ATTN_EXPORT int attn_fwd_blocksparse(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                                     const uint8_t* block_mask, int64_t B, int64_t H, int64_t H_kv, int64_t N,
+                                     int64_t d, int causal, float scale, void* stream) {
+  if (!block_mask) return ATTN_ERR_INVALID_ARG;
+  return fwd_impl(Q, K, V, O, LSE, block_mask, B, H, H_kv, N, d, causal, scale, stream);
 }
 
 ATTN_EXPORT size_t attn_bwd_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d) {
@@ -229,8 +244,10 @@ int bwd_common_checks(int64_t B, int64_t H, int64_t N, int64_t d, const void* wo
   return ATTN_OK;
 }
 
-attn::BwdParams bwd_params(const BwdSetup& su, int64_t N, int64_t H, int64_t H_kv, float scale) {
+attn::BwdParams bwd_params(const BwdSetup& su, int64_t N, int64_t H, int64_t H_kv, float scale,
+                           const uint8_t* mask) {
   attn::BwdParams prm;
+  prm.mask = mask;
   prm.h = int(H);
   prm.h_kv = int(H_kv);
   prm.group = int(H / H_kv);
@@ -264,8 +281,8 @@ ATTN_EXPORT int attn_bwd_preprocess(const void* O, const void* dO, const float* 
 
 namespace {
 
-int dkdv_impl(const void* Q, const void* K, const void* V, const void* dO, void* dK, void* dV, int64_t B, int64_t H,
-              int64_t H_kv, int64_t N, int64_t d, int causal, float scale, const void* workspace,
+int dkdv_impl(const void* Q, const void* K, const void* V, const void* dO, void* dK, void* dV, const uint8_t* mask,
+              int64_t B, int64_t H, int64_t H_kv, int64_t N, int64_t d, int causal, float scale, const void* workspace,
               size_t workspace_bytes, void* stream) {
   BwdSetup su;
   int s = bwd_common_checks(B, H, N, d, workspace, workspace_bytes, &su);
@@ -280,19 +297,16 @@ int dkdv_impl(const void* Q, const void* K, const void* V, const void* dO, void*
   if (!make_map(&mq, Q, su.bh, N, d) || !make_map(&mk, K, bhkv, N, d) || !make_map(&mv, V, bhkv, N, d) ||
       !make_map(&mdo, dO, su.bh, N, d) || !make_map(&mdk, dK, bhkv, N, d) || !make_map(&mdv, dV, bhkv, N, d))
     return ATTN_ERR_LAUNCH;
-  const attn::BwdParams prm = bwd_params(su, N, H, H_kv, scale);
+  const attn::BwdParams prm = bwd_params(su, N, H, H_kv, scale, mask);
+  const bool sparse = mask != nullptr;
   const int grid = int(bhkv * prm.n_tiles);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (d == 128)
-    return causal ? launch_dkdv<128, true>(mq, mk, mv, mdo, mdk, mdv, prm, grid, st)
-                  : launch_dkdv<128, false>(mq, mk, mv, mdo, mdk, mdv, prm, grid, st);
-  return causal ? launch_dkdv<64, true>(mq, mk, mv, mdo, mdk, mdv, prm, grid, st)
-                : launch_dkdv<64, false>(mq, mk, mv, mdo, mdk, mdv, prm, grid, st);
+  return ATTN_DISPATCH(launch_dkdv, mq, mk, mv, mdo, mdk, mdv, prm, grid, st);
 }
 
-int dq_impl(const void* Q, const void* K, const void* V, const void* dO, void* dQ, int64_t B, int64_t H, int64_t H_kv,
-            int64_t N, int64_t d, int causal, float scale, const void* workspace, size_t workspace_bytes,
-            void* stream) {
+int dq_impl(const void* Q, const void* K, const void* V, const void* dO, void* dQ, const uint8_t* mask, int64_t B,
+            int64_t H, int64_t H_kv, int64_t N, int64_t d, int causal, float scale, const void* workspace,
+            size_t workspace_bytes, void* stream) {
   BwdSetup su;
   int s = bwd_common_checks(B, H, N, d, workspace, workspace_bytes, &su);
   if (s != ATTN_OK) return s;
@@ -305,19 +319,16 @@ int dq_impl(const void* Q, const void* K, const void* V, const void* dO, void* d
   if (!make_map(&mq, Q, su.bh, N, d) || !make_map(&mk, K, bhkv, N, d) || !make_map(&mv, V, bhkv, N, d) ||
       !make_map(&mdo, dO, su.bh, N, d) || !make_map(&mdq, dQ, su.bh, N, d))
     return ATTN_ERR_LAUNCH;
-  const attn::BwdParams prm = bwd_params(su, N, H, H_kv, scale);
+  const attn::BwdParams prm = bwd_params(su, N, H, H_kv, scale, mask);
+  const bool sparse = mask != nullptr;
   const int grid = int(su.bh * prm.n_tiles);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (d == 128)
-    return causal ? launch_dq<128, true>(mq, mk, mv, mdo, mdq, prm, grid, st)
-                  : launch_dq<128, false>(mq, mk, mv, mdo, mdq, prm, grid, st);
-  return causal ? launch_dq<64, true>(mq, mk, mv, mdo, mdq, prm, grid, st)
-                : launch_dq<64, false>(mq, mk, mv, mdo, mdq, prm, grid, st);
+  return ATTN_DISPATCH(launch_dq, mq, mk, mv, mdo, mdq, prm, grid, st);
 }
 
 int bwd_impl(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE, void* dQ,
-             void* dK, void* dV, int64_t B, int64_t H, int64_t H_kv, int64_t N, int64_t d, int causal, float scale,
-             void* workspace, size_t workspace_bytes, void* stream) {
+             void* dK, void* dV, const uint8_t* mask, int64_t B, int64_t H, int64_t H_kv, int64_t N, int64_t d,
+             int causal, float scale, void* workspace, size_t workspace_bytes, void* stream) {
   int s = check_sizes(B, H, N, d);
   if (s != ATTN_OK) return s;
   if ((s = check_heads(H, H_kv)) != ATTN_OK) return s;
@@ -329,9 +340,9 @@ int bwd_impl(const void* Q, const void* K, const void* V, const void* O, const v
   if (workspace_bytes < attn_bwd_workspace_bytes(B, H, N, d)) return ATTN_ERR_WORKSPACE;
   s = attn_bwd_preprocess(O, dO, LSE, B, H, N, d, workspace, workspace_bytes, stream);
   if (s != ATTN_OK) return s;
-  s = dkdv_impl(Q, K, V, dO, dK, dV, B, H, H_kv, N, d, causal, scale, workspace, workspace_bytes, stream);
+  s = dkdv_impl(Q, K, V, dO, dK, dV, mask, B, H, H_kv, N, d, causal, scale, workspace, workspace_bytes, stream);
   if (s != ATTN_OK) return s;
-  return dq_impl(Q, K, V, dO, dQ, B, H, H_kv, N, d, causal, scale, workspace, workspace_bytes, stream);
+  return dq_impl(Q, K, V, dO, dQ, mask, B, H, H_kv, N, d, causal, scale, workspace, workspace_bytes, stream);
 }
 
 }  // namespace
@@ -341,27 +352,179 @@ extern "C" {
 ATTN_EXPORT int attn_bwd_dkdv(const void* Q, const void* K, const void* V, const void* dO, void* dK, void* dV,
                               int64_t B, int64_t H, int64_t N, int64_t d, int causal, float scale,
                               const void* workspace, size_t workspace_bytes, void* stream) {
-  return dkdv_impl(Q, K, V, dO, dK, dV, B, H, H, N, d, causal, scale, workspace, workspace_bytes, stream);
+  return dkdv_impl(Q, K, V, dO, dK, dV, nullptr, B, H, H, N, d, causal, scale, workspace, workspace_bytes, stream);
 }
 
 ATTN_EXPORT int attn_bwd_dq(const void* Q, const void* K, const void* V, const void* dO, void* dQ, int64_t B,
                             int64_t H, int64_t N, int64_t d, int causal, float scale, const void* workspace,
                             size_t workspace_bytes, void* stream) {
-  return dq_impl(Q, K, V, dO, dQ, B, H, H, N, d, causal, scale, workspace, workspace_bytes, stream);
+  return dq_impl(Q, K, V, dO, dQ, nullptr, B, H, H, N, d, causal, scale, workspace, workspace_bytes, stream);
 }
 
 ATTN_EXPORT int attn_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
                          void* dQ, void* dK, void* dV, int64_t B, int64_t H, int64_t N, int64_t d, int causal,
                          float scale, void* workspace, size_t workspace_bytes, void* stream) {
-  return bwd_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, H, N, d, causal, scale, workspace, workspace_bytes, stream);
+  return bwd_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, nullptr, B, H, H, N, d, causal, scale, workspace, workspace_bytes,
+                  stream);
 }
 
 ATTN_EXPORT int attn_bwd_gqa(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                              const float* LSE, void* dQ, void* dK, void* dV, int64_t B, int64_t H, int64_t H_kv,
                              int64_t N, int64_t d, int causal, float scale, void* workspace, size_t workspace_bytes,
                              void* stream) {
-  return bwd_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, H_kv, N, d, causal, scale, workspace, workspace_bytes,
-                  stream);
+  return bwd_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, nullptr, B, H, H_kv, N, d, causal, scale, workspace,
+                  workspace_bytes, stream);
+}
+
+ATTN_EXPORT int attn_bwd_blocksparse(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                                     const float* LSE, const uint8_t* block_mask, void* dQ, void* dK, void* dV,
+                                     int64_t B, int64_t H, int64_t H_kv, int64_t N, int64_t d, int causal,
+                                     float scale, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!block_mask) return ATTN_ERR_INVALID_ARG;
+  return bwd_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, block_mask, B, H, H_kv, N, d, causal, scale, workspace,
+                  workspace_bytes, stream);
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Forward against a key/value cache (decode / chunked prefill), split-KV.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr int64_t kNumSMs = 148;        // B200; only the automatic split count depends on it
+constexpr int64_t kMaxSplits = 256;
+
+struct KvcShape {
+  int64_t rows = 0;        // packed query rows per key/value head
+  int64_t n_rt = 0;        // 128-row tiles of packed rows
+  int64_t tiles = 0;       // 128-row key tiles of the cache
+  int64_t total_rows = 0;  // B*H*Nq
+};
+
+int kvc_check(int64_t B, int64_t H, int64_t H_kv, int64_t Nq, int64_t Nk, int64_t d, KvcShape* sh) {
+  if (B < 1 || H < 1 || Nq < 1 || Nk < 1) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  int s = check_heads(H, H_kv);
+  if (s != ATTN_OK) return s;
+  if (B > INT32_MAX / H || Nq > (INT32_MAX - 128) / (B * H) || Nk > INT32_MAX - 256) return ATTN_ERR_INVALID_ARG;
+  sh->rows = (H / H_kv) * Nq;
+  sh->n_rt = (sh->rows + 127) / 128;
+  sh->tiles = (Nk + 127) / 128;
+  sh->total_rows = B * H * Nq;
+  return ATTN_OK;
+}
+
+// Splits: explicit counts are capped at the number of key tiles; the automatic
+// count minimises (waves of CTAs over the SMs) x (key tiles per CTA + 1), the
+// +1 standing for a CTA's fixed cost (setup, pipeline fill, partial write).
+int64_t kvc_splits(const KvcShape& sh, int64_t B, int64_t H_kv, int64_t num_splits) {
+  if (num_splits < 0) return 0;
+  const int64_t cap = std::min(sh.tiles, kMaxSplits);
+  if (num_splits > 0) return std::min(num_splits, cap);
+  const int64_t base = B * H_kv * sh.n_rt;
+  int64_t best_s = 1, best_cost = INT64_MAX;
+  for (int64_t sp = 1; sp <= cap; ++sp) {
+    const int64_t per = (sh.tiles + sp - 1) / sp;
+    const int64_t waves = (base * sp + kNumSMs - 1) / kNumSMs;
+    const int64_t cost = waves * (per + 1);
+    if (cost < best_cost) {
+      best_cost = cost;
+      best_s = sp;
+    }
+  }
+  return best_s;
+}
+
+size_t kvc_workspace(const KvcShape& sh, int64_t splits, int64_t d) {
+  if (splits <= 1) return 0;
+  return size_t(splits) * size_t(sh.total_rows) * size_t(d + 1) * sizeof(float);
+}
+
+template <int D, bool CAUSAL, bool SPLIT>
+int launch_kvc(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const attn::KvcParams& prm,
+               int grid, cudaStream_t st) {
+  auto kern = attn::attn_kvcache_kernel<D, CAUSAL, SPLIT>;
+  constexpr int smem = attn::KvcCfg<D>::kSmemBytes;
+  if (set_smem(reinterpret_cast<const void*>(kern), smem) != ATTN_OK) return ATTN_ERR_LAUNCH;
+  kern<<<grid, attn::KvcCfg<D>::kThreads, smem, st>>>(q, k, v, prm);
+  int s = launch_status();
+  if (s != ATTN_OK || !SPLIT) return s;
+  int64_t blocks = (prm.total_rows + 7) / 8;                  // 8 rows (warps) per 256-thread block
+  if (blocks > kNumSMs * 16) blocks = kNumSMs * 16;
+  attn::attn_kvcache_merge_kernel<D><<<int(blocks), 256, 0, st>>>(prm.part_o, prm.part_lse, prm.o, prm.lse,
+                                                                   prm.total_rows, prm.splits);
+  return launch_status();
+}
+
+#define ATTN_KVC_DISPATCH(...)                                                                         \
+  (d == 128 ? (causal ? (split ? launch_kvc<128, true, true>(__VA_ARGS__) : launch_kvc<128, true, false>(__VA_ARGS__)) \
+                      : (split ? launch_kvc<128, false, true>(__VA_ARGS__) : launch_kvc<128, false, false>(__VA_ARGS__))) \
+            : (causal ? (split ? launch_kvc<64, true, true>(__VA_ARGS__) : launch_kvc<64, true, false>(__VA_ARGS__)) \
+                      : (split ? launch_kvc<64, false, true>(__VA_ARGS__) : launch_kvc<64, false, false>(__VA_ARGS__))))
+
+}  // namespace
+
+extern "C" {
+
+ATTN_EXPORT int64_t attn_fwd_kvcache_splits(int64_t B, int64_t H, int64_t H_kv, int64_t Nq, int64_t Nk, int64_t d,
+                                            int64_t num_splits) {
+  KvcShape sh;
+  if (kvc_check(B, H, H_kv, Nq, Nk, d, &sh) != ATTN_OK) return 0;
+  return kvc_splits(sh, B, H_kv, num_splits);
+}
+
+ATTN_EXPORT size_t attn_fwd_kvcache_workspace_bytes(int64_t B, int64_t H, int64_t H_kv, int64_t Nq, int64_t Nk,
+                                                    int64_t d, int64_t num_splits) {
+  KvcShape sh;
+  if (kvc_check(B, H, H_kv, Nq, Nk, d, &sh) != ATTN_OK) return 0;
+  return kvc_workspace(sh, kvc_splits(sh, B, H_kv, num_splits), d);
+}
+
+ATTN_EXPORT int attn_fwd_kvcache(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                                 const int32_t* kv_lens, int64_t B, int64_t H, int64_t H_kv, int64_t Nq, int64_t Nk,
+                                 int64_t d, int causal, float scale, int64_t num_splits, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+  KvcShape sh;
+  int s = kvc_check(B, H, H_kv, Nq, Nk, d, &sh);
+  if (s != ATTN_OK) return s;
+  if ((s = check_scale(scale)) != ATTN_OK) return s;
+  const int64_t splits = kvc_splits(sh, B, H_kv, num_splits);
+  if (splits < 1) return ATTN_ERR_INVALID_ARG;
+  if (!Q || !K || !V || !O || !LSE) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE))
+    return ATTN_ERR_MISALIGNED;
+  if (kv_lens && (reinterpret_cast<uintptr_t>(kv_lens) & 3u) != 0) return ATTN_ERR_MISALIGNED;
+  const bool split = splits > 1;
+  if (split) {
+    if (!workspace) return ATTN_ERR_INVALID_ARG;
+    if (!aligned16(workspace)) return ATTN_ERR_MISALIGNED;
+    if (workspace_bytes < kvc_workspace(sh, splits, d)) return ATTN_ERR_WORKSPACE;
+  }
+  const int64_t grid = B * H_kv * sh.n_rt * splits;
+  if (grid > INT32_MAX) return ATTN_ERR_INVALID_ARG;
+  const int qbox = int(std::min<int64_t>(128, (sh.rows + 7) / 8 * 8));
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, Q, 1, sh.total_rows, d, qbox) || !make_map(&mk, K, B * H_kv, Nk, d) ||
+      !make_map(&mv, V, B * H_kv, Nk, d))
+    return ATTN_ERR_LAUNCH;
+  attn::KvcParams prm;
+  prm.o = static_cast<__nv_bfloat16*>(O);
+  prm.lse = LSE;
+  prm.part_o = split ? static_cast<float*>(workspace) : nullptr;
+  prm.part_lse = split ? static_cast<float*>(workspace) + size_t(splits) * size_t(sh.total_rows) * size_t(d) : nullptr;
+  prm.kv_lens = kv_lens;
+  prm.total_rows = sh.total_rows;
+  prm.nq = int(Nq);
+  prm.nk = int(Nk);
+  prm.h_kv = int(H_kv);
+  prm.rows = int(sh.rows);
+  prm.n_rt = int(sh.n_rt);
+  prm.splits = int(splits);
+  prm.qbox = qbox;
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return ATTN_KVC_DISPATCH(mq, mk, mv, prm, int(grid), st);
 }
 
 }  // extern "C"
@@ -428,6 +591,47 @@ ATTN_EXPORT int attn_bwd_static_workspace(const void* Q, const void* K, const vo
   if (ws == nullptr) return ATTN_ERR_DEVICE;
   return attn_bwd(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, d, causal, scale, ws,
                   size_t(ATTN_STATIC_WORKSPACE_BYTES), stream);
+}
+
+}  // extern "C"
+
+namespace {
+
+// Failure-path self-test: one CTA allocates tensor memory, waits on an
+// mbarrier that nothing ever arrives on with a short limit, takes the same
+// timeout path as the attention kernels (abort flag + status word), then
+// releases its tensor memory and returns.  No fault, trap or endless loop.
+__global__ void attn_selftest_timeout_kernel(unsigned long long timeout_ns, int* waited_ok) {
+  __shared__ uint64_t bar;
+  __shared__ uint32_t tslot;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    attn::mbar_init(&bar, 1);
+    abort_flag = 0;
+    attn::fence_barrier_init();
+  }
+  attn::tmem_alloc(&tslot, 32);
+  attn::tmem_relinquish();
+  attn::tc_fence_before();
+  __syncthreads();
+  attn::tc_fence_after();
+  const uint32_t tmem = tslot;
+  bool ok = attn::mbar_wait(&bar, 0, &abort_flag, true, timeout_ns);   // runs out after timeout_ns
+  ok = __all_sync(0xffffffffu, ok);
+  if (threadIdx.x == 0 && waited_ok) *waited_ok = ok ? 1 : 0;
+  attn::tc_fence_before();
+  __syncthreads();
+  attn::tc_fence_after();
+  attn::tmem_dealloc(tmem, 32);
+}
+
+}  // namespace
+
+extern "C" {
+
+ATTN_EXPORT int attn_selftest_wait_timeout(void* stream) {
+  attn_selftest_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(20ull * 1000 * 1000, nullptr);
+  return launch_status();
 }
 
 ATTN_EXPORT int attn_check_status(void* stream) {

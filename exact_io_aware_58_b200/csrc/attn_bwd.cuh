@@ -63,7 +63,10 @@ attn_bwd_pre_kernel(const __nv_bfloat16* __restrict__ O, const __nv_bfloat16* __
     for (int o = kTpr / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o, kTpr);
     if (sub == 0) {
       ws_d[row] = (i < n) ? acc : 0.f;
-      ws_lse2[row] = (i < n) ? lse[size_t(bh) * size_t(n) + size_t(i)] * kLog2e : INFINITY;
+      // padding rows, and rows that see no key (LSE = -inf, block-sparse), get
+      // +inf so that every recomputed probability of theirs is exactly 0
+      const float lv = (i < n) ? lse[size_t(bh) * size_t(n) + size_t(i)] : -INFINITY;
+      ws_lse2[row] = (lv == -INFINITY) ? INFINITY : lv * kLog2e;
     }
   }
 }
@@ -79,7 +82,23 @@ struct BwdParams {
   int group;              // h / h_kv
   float scale;
   float scale_log2;
+  const uint8_t* mask;    // block-sparse only: [B*H][nt][nt], 1 = query tile attends key tile
 };
+
+// Selection over a linear range [0, hi): sel(L) != 0 marks the visited items.
+// Every role scans the same bytes, so they all walk the same sequence.
+template <class F>
+__device__ __forceinline__ int sel_next(const F& sel, int L, int hi) {
+  for (++L; L < hi; ++L)
+    if (sel(L)) return L;
+  return hi;
+}
+template <class F>
+__device__ __forceinline__ int sel_count(const F& sel, int hi) {
+  int c = 0;
+  for (int L = 0; L < hi; ++L) c += sel(L) ? 1 : 0;
+  return c;
+}
 
 template <int D>
 struct BwdCfg {
@@ -148,6 +167,15 @@ __device__ __forceinline__ void tmem_acc_to_smem(uint32_t t_acc_lane, uint32_t s
   }
 }
 
+// Zero row r, 32-column chunks [chunk_lo, chunk_hi), of a 128B-swizzled bf16 tile.
+template <int D>
+__device__ __forceinline__ void zero_tile_rows(uint32_t stage_u32, int r, int chunk_lo, int chunk_hi) {
+  for (int cc = chunk_lo; cc < chunk_hi; ++cc)
+#pragma unroll
+    for (int ch = 0; ch < 4; ++ch)
+      st_shared_v4(stage_u32 + (cc >> 1) * (128 * 128) + sw128_offset(r, (cc & 1) * 4 + ch), 0u, 0u, 0u, 0u);
+}
+
 // Load 64 fp32 columns [c0, c0+64) of this thread's TMEM lane.
 __device__ __forceinline__ void tmem_ld64f(uint32_t taddr, float (&v)[64]) {
   uint32_t a[32], b[32];
@@ -165,7 +193,7 @@ __device__ __forceinline__ void tmem_ld64f(uint32_t taddr, float (&v)[64]) {
 // ---------------------------------------------------------------------------
 // dK, dV
 // ---------------------------------------------------------------------------
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool SPARSE>
 __global__ void __launch_bounds__(320, 1)
 attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -203,8 +231,15 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
   const int n0 = jt * 128;
   const int i_start = CAUSAL ? jt : 0;
   const int n_q = nt - i_start;                // query tiles per query head
-  const int n_it = prm.group * n_q;            // every query head sharing this key/value head
+  const int n_all = prm.group * n_q;           // every (query head sharing this key/value head, query tile)
   const int bq0 = (bkv / prm.h_kv) * prm.h + (bkv % prm.h_kv) * prm.group;   // first such query head
+  // Block-sparse: item L = (query head bq0 + L / n_q, query tile i_start + L % n_q) is visited
+  // only if that query tile selected this key tile.
+  const uint8_t* mcol = SPARSE ? prm.mask + jt : nullptr;
+  auto sel = [&](int L) -> bool {
+    return mcol[(size_t(bq0 + L / n_q) * nt + size_t(i_start + L % n_q)) * nt] != 0;
+  };
+  const int n_it = SPARSE ? sel_count(sel, n_all) : n_all;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < QS; ++s) {
@@ -240,15 +275,22 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
 
   if (warp == C::kWarpLoad) {
     if (lane == 0) {
-      mbar_arrive_expect_tx(kv_full, 2 * C::kTileBytes);
-      for (int b = 0; b < C::kNumBlk; ++b) {
-        tma_load_3d(&tm_k, kv_full, smem + C::kKV_OffK + b * C::kBlockBytes, b * 64, n0, bkv);
-        tma_load_3d(&tm_v, kv_full, smem + C::kKV_OffV + b * C::kBlockBytes, b * 64, n0, bkv);
+      // A key tile that no query tile selected (block-sparse) loads nothing:
+      // its K/V slots are the staging area of the zero dK/dV it writes.
+      if (n_it > 0) {
+        mbar_arrive_expect_tx(kv_full, 2 * C::kTileBytes);
+        for (int b = 0; b < C::kNumBlk; ++b) {
+          tma_load_3d(&tm_k, kv_full, smem + C::kKV_OffK + b * C::kBlockBytes, b * 64, n0, bkv);
+          tma_load_3d(&tm_v, kv_full, smem + C::kKV_OffV + b * C::kBlockBytes, b * 64, n0, bkv);
+        }
       }
       int q_issued = 0, o_issued = 0, v_issued = 0;
+      int Lsel = SPARSE ? sel_next(sel, -1, n_all) : 0;
       for (int it = 0; it < n_it; ++it) {
-        const int qi = i_start + it % n_q;
-        const int bq = bq0 + it / n_q;
+        const int L = SPARSE ? Lsel : it;
+        if (SPARSE) Lsel = sel_next(sel, Lsel, n_all);
+        const int qi = i_start + L % n_q;
+        const int bq = bq0 + L / n_q;
         {   // LSE*log2(e) and D of query tile i
           const int slot = it % VS, use = it / VS;
           if (use > 0 && !mbar_wait(&v_empty[slot], (use - 1) & 1, abort_flag)) break;
@@ -279,7 +321,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
         }
       }
       // No copy may still be landing in shared memory when the CTA leaves.
-      mbar_wait(kv_full, 0, abort_flag, false);
+      if (n_it > 0) mbar_wait(kv_full, 0, abort_flag, false);
       for (int it = max(0, q_issued - QS); it < q_issued; ++it)
         mbar_wait(&q_full[it % QS], (it / QS) & 1, abort_flag, false);
       for (int it = max(0, o_issued - OS); it < o_issued; ++it)
@@ -313,7 +355,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       auto wait_q = [&](int it) { return mbar_wait(&q_full[it % QS], (it / QS) & 1, abort_flag); };
       auto wait_o = [&](int it) { return mbar_wait(&o_full[it % OS], (it / OS) & 1, abort_flag); };
 
-      bool ok = mbar_wait(kv_full, 0, abort_flag) && wait_q(0) && wait_o(0);
+      bool ok = n_it > 0 && mbar_wait(kv_full, 0, abort_flag) && wait_q(0) && wait_o(0);
       if (ok) {
         tc_fence_after();
         issue_kmajor(C::kColA, sK, q_tile(0));    // S^T = K_j Q_i^T
@@ -360,8 +402,11 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
     const uint32_t tB = tmem + lane_base + C::kColB + 64 * g;
     const float c = prm.scale_log2;
     bool ok = true;
+    int Lsel = SPARSE ? sel_next(sel, -1, n_all) : 0;
     for (int it = 0; it < n_it; ++it) {
-      const int qi = i_start + it % n_q;
+      const int L = SPARSE ? Lsel : it;
+      if (SPARSE) Lsel = sel_next(sel, Lsel, n_all);
+      const int qi = i_start + L % n_q;
       const float* vec = reinterpret_cast<const float*>(smem + C::kKV_OffVec + (it % VS) * 2 * C::kVecBytes);
       // LSE/D vectors of this query tile (released below, after the dS reads).
       if (!(ok = mbar_wait_warp(&v_full[it % VS], (it / VS) & 1, abort_flag))) break;
@@ -420,12 +465,15 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
       mbar_arrive(ds_full);
     }
     // epilogue: group 0 writes dV (staged in the V_j slot), group 1 writes dK (in the K_j slot)
-    if (ok) ok = mbar_wait_warp(acc_full, 0, abort_flag);
+    if (ok && n_it > 0) ok = mbar_wait_warp(acc_full, 0, abort_flag);
     uint8_t* stage = smem + (g == 0 ? C::kKV_OffV : C::kKV_OffK);
     if (ok) {
       tc_fence_after();
-      tmem_acc_to_smem<D>(tmem + lane_base + (g == 0 ? C::kColAcc0 : C::kColAcc1), smem_u32(stage), r, 0, D / 32,
-                          g == 0 ? 1.f : prm.scale);
+      if (n_it > 0)
+        tmem_acc_to_smem<D>(tmem + lane_base + (g == 0 ? C::kColAcc0 : C::kColAcc1), smem_u32(stage), r, 0, D / 32,
+                            g == 0 ? 1.f : prm.scale);
+      else
+        zero_tile_rows<D>(smem_u32(stage), r, 0, D / 32);   // no query tile selected this key tile
     }
     fence_proxy_async_smem();
     named_barrier_sync(1 + g, 128);
@@ -449,7 +497,7 @@ attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_cons
 // ---------------------------------------------------------------------------
 // dQ
 // ---------------------------------------------------------------------------
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool SPARSE>
 __global__ void __launch_bounds__(320, 1)
 attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -484,7 +532,10 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
   const int bkv = (bh / prm.h) * prm.h_kv + (bh % prm.h) / prm.group;        // its key/value head
   const int it_q = nt - 1 - (blockIdx.x % nt);   // query tile; large = most work under the causal mask
   const int m0 = it_q * 128;
-  const int n_it = CAUSAL ? it_q + 1 : nt;
+  const int j_hi = CAUSAL ? it_q + 1 : nt;       // key tiles [0, j_hi) may be visible
+  const uint8_t* mrow = SPARSE ? prm.mask + (size_t(bh) * nt + it_q) * nt : nullptr;
+  auto sel = [&](int j) -> bool { return mrow[j] != 0; };
+  const int n_it = SPARSE ? sel_count(sel, j_hi) : j_hi;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < KS; ++s) {
@@ -525,14 +576,17 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       bulk_load(smem + C::kQ_OffVec, prm.ws_lse2 + voff, C::kVecBytes, q_full);
       bulk_load(smem + C::kQ_OffVec + C::kVecBytes, prm.ws_d + voff, C::kVecBytes, q_full);
       int k_issued = 0, v_issued = 0;
+      int jsel = SPARSE ? sel_next(sel, -1, j_hi) : 0;
       for (int it = 0; it < n_it; ++it) {
+        const int j = SPARSE ? jsel : it;
+        if (SPARSE) jsel = sel_next(sel, jsel, j_hi);
         {
           const int slot = it % KS, use = it / KS;
           if (use > 0 && !mbar_wait(&k_empty[slot], (use - 1) & 1, abort_flag)) break;
           mbar_arrive_expect_tx(&k_full[slot], C::kTileBytes);
           for (int b = 0; b < C::kNumBlk; ++b)
             tma_load_3d(&tm_k, &k_full[slot], smem + C::kQ_OffK + slot * C::kTileBytes + b * C::kBlockBytes, b * 64,
-                        it * 128, bkv);
+                        j * 128, bkv);
           ++k_issued;
         }
         {
@@ -541,7 +595,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
           mbar_arrive_expect_tx(&v_full[slot], C::kTileBytes);
           for (int b = 0; b < C::kNumBlk; ++b)
             tma_load_3d(&tm_v, &v_full[slot], smem + C::kQ_OffV + slot * C::kTileBytes + b * C::kBlockBytes, b * 64,
-                        it * 128, bkv);
+                        j * 128, bkv);
           ++v_issued;
         }
       }
@@ -571,7 +625,7 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
         }
       };
 
-      bool ok = mbar_wait(q_full, 0, abort_flag) && wait_k(0) && wait_v(0);
+      bool ok = n_it > 0 && mbar_wait(q_full, 0, abort_flag) && wait_k(0) && wait_v(0);
       if (ok) {
         tc_fence_after();
         issue_kmajor(C::kColA, sQ, k_tile(0));    // S = Q_i K_j^T
@@ -625,7 +679,10 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
     const float* vec = reinterpret_cast<const float*>(smem + C::kQ_OffVec);
     const float neg_lse2 = ok ? -vec[r] : 0.f;
     const float dval = ok ? vec[128 + r] : 0.f;
+    int jsel = SPARSE ? sel_next(sel, -1, j_hi) : 0;
     for (int it = 0; it < n_it && ok; ++it) {
+      const int j = SPARSE ? jsel : it;               // key tile of this iteration
+      if (SPARSE) jsel = sel_next(sel, jsel, j_hi);
       if (!(ok = mbar_wait_warp(s_full, it & 1, abort_flag))) break;
       tc_fence_after();
       float p[64];
@@ -634,8 +691,8 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       mbar_arrive(s_free);
 #pragma unroll
       for (int k = 0; k < 64; ++k) p[k] = ex2(fmaf(p[k], c, neg_lse2));
-      const int kbase = it * 128 + 64 * g;
-      const bool need_mask = (CAUSAL && it == it_q) || (kbase + 64 > n);
+      const int kbase = j * 128 + 64 * g;
+      const bool need_mask = (CAUSAL && j == it_q) || (kbase + 64 > n);
       if (need_mask) {
         int lim = n - 1 - kbase;                 // keep k <= lim
         if (CAUSAL) lim = min(lim, row - kbase);
@@ -658,13 +715,16 @@ attn_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_consta
       tc_fence_before();
       mbar_arrive(ds_full);
     }
-    if (ok) ok = mbar_wait_warp(acc_full, 0, abort_flag);
+    if (ok && n_it > 0) ok = mbar_wait_warp(acc_full, 0, abort_flag);
     uint8_t* stage = smem + C::kQ_OffQ;   // Q_i is no longer read
     if (ok) {
       tc_fence_after();
       constexpr int kChunks = D / 32;
-      tmem_acc_to_smem<D>(tmem + lane_base + C::kColAcc0, smem_u32(stage), r, g * kChunks / 2, (g + 1) * kChunks / 2,
-                          prm.scale);
+      if (n_it > 0)
+        tmem_acc_to_smem<D>(tmem + lane_base + C::kColAcc0, smem_u32(stage), r, g * kChunks / 2,
+                            (g + 1) * kChunks / 2, prm.scale);
+      else
+        zero_tile_rows<D>(smem_u32(stage), r, g * kChunks / 2, (g + 1) * kChunks / 2);   // this query tile sees no key
     }
     fence_proxy_async_smem();
     named_barrier_sync(1, 256);

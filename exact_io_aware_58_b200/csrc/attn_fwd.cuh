@@ -41,6 +41,29 @@ struct FwdParams {
   int h_kv;            // key/value heads per batch (h % h_kv == 0)
   int group;           // h / h_kv query heads share one key/value head
   float scale_log2;    // scale * log2(e)
+  const uint8_t* mask; // block-sparse only: [B*H][nt][nt], 1 = query tile attends key tile
+  int nt;              // ceil(N / 128)
+};
+
+// Key tiles selected for the (up to) two 128-row query tiles of a CTA: bit t of
+// flags(j) says query tile t attends key tile j.  Every role scans the same
+// bytes, so they all walk the same sequence of tiles.
+struct TileSelect {
+  const uint8_t* r0;
+  const uint8_t* r1;   // null when the second query tile is past N
+  __device__ __forceinline__ uint32_t flags(int j) const {
+    return (r0[j] ? 1u : 0u) | ((r1 != nullptr && r1[j]) ? 2u : 0u);
+  }
+  __device__ __forceinline__ int next(int j, int hi) const {   // first selected tile > j, or hi
+    for (++j; j < hi; ++j)
+      if (flags(j)) return j;
+    return hi;
+  }
+  __device__ __forceinline__ int count(int hi) const {
+    int c = 0;
+    for (int j = 0; j < hi; ++j) c += flags(j) ? 1 : 0;
+    return c;
+  }
 };
 
 template <int D>
@@ -64,7 +87,7 @@ struct FwdCfg {
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;   // + slack for 1024-byte alignment
 };
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool SPARSE>
 __global__ void __launch_bounds__(320, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -91,7 +114,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const int m_blk = prm.n_mblk - 1 - (blockIdx.x % prm.n_mblk);   // heaviest causal blocks first
   const int m0 = m_blk * 256;
   const int n_kv_total = (n + 127) >> 7;
-  const int nkv = CAUSAL ? min(n_kv_total, (m0 >> 7) + 2) : n_kv_total;
+  const int kv_hi = CAUSAL ? min(n_kv_total, (m0 >> 7) + 2) : n_kv_total;   // key tiles [0, kv_hi) may be visible
+  TileSelect sel{nullptr, nullptr};
+  if (SPARSE) {
+    const int qt0 = m0 >> 7;
+    sel.r0 = prm.mask + (size_t(bh) * prm.nt + qt0) * prm.nt;
+    sel.r1 = (qt0 + 1 < prm.nt) ? sel.r0 + prm.nt : nullptr;
+  }
+  const int nkv = SPARSE ? sel.count(kv_hi) : kv_hi;   // key tiles this CTA visits
 
   if (threadIdx.x == 0) {
     for (int t = 0; t < 2; ++t) {
@@ -126,7 +156,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   if (warp == C::kWarpLoad) {
     // ------------------------------------------------------------------ TMA
     if (lane == 0) {
-      for (int t = 0; t < 2; ++t) {
+      // A CTA that visits no key tile (block-sparse) loads nothing: its Q slots
+      // are the staging area of the zero output it writes.
+      for (int t = 0; t < 2 && nkv > 0; ++t) {
         mbar_arrive_expect_tx(&q_full[t], C::kTileBytes);
         for (int b = 0; b < C::kNumBlk; ++b)
           tma_load_3d(&tm_q, &q_full[t], smem + C::kOffQ + t * C::kTileBytes + b * C::kBlockBytes,
@@ -134,12 +166,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
       int issued = 0;
       bool ok = true;
+      int jsel = SPARSE ? sel.next(-1, kv_hi) : 0;
       for (int it = 0; it < 2 * nkv; ++it) {
         const int slot = it % C::kSlots;
         const int use = it / C::kSlots;
         if (use > 0 && !mbar_wait(&kv_empty[slot], (use - 1) & 1, abort_flag)) { ok = false; break; }
         const CUtensorMap* tm = (it & 1) ? &tm_v : &tm_k;
-        const int j = it >> 1;
+        const int j = SPARSE ? jsel : (it >> 1);
+        if (SPARSE && (it & 1)) jsel = sel.next(jsel, kv_hi);
         mbar_arrive_expect_tx(&kv_full[slot], C::kTileBytes);
         for (int b = 0; b < C::kNumBlk; ++b)
           tma_load_3d(tm, &kv_full[slot], smem + C::kOffKV + slot * C::kTileBytes + b * C::kBlockBytes,
@@ -148,8 +182,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       }
       (void)ok;
       // No copy may still be landing in shared memory when the CTA leaves.
-      mbar_wait(&q_full[0], 0, abort_flag, false);
-      mbar_wait(&q_full[1], 0, abort_flag, false);
+      if (nkv > 0) {
+        mbar_wait(&q_full[0], 0, abort_flag, false);
+        mbar_wait(&q_full[1], 0, abort_flag, false);
+      }
       for (int it = max(0, issued - C::kSlots); it < issued; ++it)
         mbar_wait(&kv_full[it % C::kSlots], (it / C::kSlots) & 1, abort_flag, false);
     }
@@ -189,7 +225,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                  (acc || kk > 0) ? 1u : 0u);
       };
 
-      bool ok = mbar_wait(&q_full[0], 0, abort_flag) && mbar_wait(&q_full[1], 0, abort_flag);
+      bool ok = nkv > 0 && mbar_wait(&q_full[0], 0, abort_flag) && mbar_wait(&q_full[1], 0, abort_flag);
       if (ok) {
         int ks;
         ok = wait_kv(ks);
@@ -247,8 +283,13 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     float l = 0.f;
     bool ok = true;
 
-    for (int j = 0; j < nkv; ++j) {
-      if (!(ok = mbar_wait_warp(&s_full[t], j & 1, abort_flag))) break;
+    int jsel = SPARSE ? sel.next(-1, kv_hi) : 0;
+    for (int jj = 0; jj < nkv; ++jj) {
+      // jj counts visited tiles (barrier phases); j is the key tile itself
+      const int j = SPARSE ? jsel : jj;
+      const bool tile_on = SPARSE ? ((sel.flags(j) >> t) & 1u) != 0 : true;
+      if (SPARSE) jsel = sel.next(jsel, kv_hi);
+      if (!(ok = mbar_wait_warp(&s_full[t], jj & 1, abort_flag))) break;
       tc_fence_after();
       float s[128];
       {
@@ -269,9 +310,9 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           s[96 + k] = __uint_as_float(f[k]);
         }
       }
-      const bool need_mask = (CAUSAL && (128 * j + 127 > m0 + 128 * t)) || (128 * j + 128 > n);
+      const bool need_mask = !tile_on || (CAUSAL && (128 * j + 127 > m0 + 128 * t)) || (128 * j + 128 > n);
       if (need_mask) {
-        int limit = n - 1 - 128 * j;
+        int limit = tile_on ? n - 1 - 128 * j : -1;     // a tile this query tile did not select: all masked
         if (CAUSAL) limit = min(limit, i - 128 * j);
 #pragma unroll
         for (int k = 0; k < 128; ++k)
@@ -294,7 +335,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       if (m_tile > m_ref + kRescaleLog2) {
         alpha = ex2(m_ref - m_tile);      // 0 when m_ref is still -inf
         m_ref = m_tile;
-        rescale = (j > 0);
+        rescale = (jj > 0);
       }
       l *= alpha;
       const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
@@ -333,16 +374,23 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     }
 
     // ------------------------------------------------------------ epilogue
-    if (ok) ok = mbar_wait_warp(&o_full[t], 0, abort_flag);
+    const bool any_tile = !SPARSE || nkv > 0;   // dense: every CTA visits at least one key tile
+    if (ok && any_tile) ok = mbar_wait_warp(&o_full[t], 0, abort_flag);
     uint8_t* stage = smem + C::kOffQ + t * C::kTileBytes;   // Q_t is no longer read
     if (ok) {
       tc_fence_after();
-      const float inv_l = 1.f / l;
+      // l == 0 only for rows that see no key at all (block-sparse): O = 0, LSE = -inf.
+      const float inv_l = (SPARSE && !(l > 0.f)) ? 0.f : 1.f / l;
 #pragma unroll 1
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t o[32];
-        tmem_ld32(tO + cc * 32, o);
-        tmem_ld_wait(o);
+        if (any_tile) {
+          tmem_ld32(tO + cc * 32, o);
+          tmem_ld_wait(o);
+        } else {
+#pragma unroll
+          for (int k = 0; k < 32; ++k) o[k] = 0u;
+        }
         const uint32_t blk = cc >> 1;
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
@@ -354,7 +402,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           st_shared_v4(smem_u32(stage) + blk * C::kBlockBytes + sw128_offset(r, chunk), w0, w1, w2, w3);
         }
       }
-      if (i < n) prm.lse[size_t(bh) * size_t(n) + size_t(i)] = (m_ref + __log2f(l)) * kLn2;
+      if (i < n)
+        prm.lse[size_t(bh) * size_t(n) + size_t(i)] = (SPARSE && !(l > 0.f)) ? -INFINITY : (m_ref + __log2f(l)) * kLn2;
     }
     fence_proxy_async_smem();
     named_barrier_sync(1 + t, 128);

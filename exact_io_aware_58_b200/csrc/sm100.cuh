@@ -73,7 +73,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 // `honour_abort` = false keeps waiting (still bounded) even after an abort;
 // used to drain copies that are already in flight.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          bool honour_abort = true) {
+                                          bool honour_abort = true,
+                                          unsigned long long timeout_ns = kWaitTimeoutNs) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const unsigned long long t0 = globaltimer();
@@ -81,7 +82,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (mbar_try_wait(a, parity)) return true;
     if ((it & 31u) == 0) {
       if (honour_abort && *abort_flag) return false;
-      if (globaltimer() - t0 > kWaitTimeoutNs) {
+      if (globaltimer() - t0 > timeout_ns) {
         *abort_flag = 1;
         atomicOr(&g_attn_status, kStatusTimeout);
         return false;

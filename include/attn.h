@@ -84,6 +84,64 @@ int attn_fwd_gqa(const void* Q, const void* K, const void* V, void* O, float* LS
                  void* stream);
 
 /*
+ * Forward restricted to selected blocks ("Attention and KV Compression",
+ * section "The composability point": sparse selection changes which blocks
+ * are attended, and the kernel runs on the selected blocks).
+ * block_mask: DEVICE pointer to [B*H][nt][nt] bytes, nt = ceil(N/128);
+ * block_mask[(b*H + h)*nt*nt + i*nt + j] != 0 means query rows 128i..128i+127
+ * of head (b, h) attend key rows 128j..128j+127 (further restricted to j <= i
+ * row-wise when causal).  Only selected key tiles are loaded and multiplied.
+ * A row that sees no key gets O = 0 and LSE = -inf.  Shared key/value heads
+ * as in attn_fwd_gqa (H_kv = H for plain multi-head attention).
+ */
+int attn_fwd_blocksparse(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                         const uint8_t* block_mask,
+                         int64_t B, int64_t H, int64_t H_kv, int64_t N, int64_t d, int causal,
+                         float scale, void* stream);
+
+/*
+ * Forward of Nq new query rows against a key/value cache (decode and
+ * chunked-prefill shapes: "FlashAttention -- how 100K-token attention fits in
+ * memory", section "Arithmetic intensity", where prefill and decode are the
+ * same computation in two shape regimes; the tiling and online softmax are
+ * those of attn_fwd).
+ *   Q, O    bf16 [B][H][Nq][d] row-major (device, 16-byte aligned)
+ *   K, V    bf16 [B][H_kv][Nk][d] (the cache; Nk = its capacity in rows)
+ *   LSE     fp32 [B][H][Nq] natural-log row log-sum-exp
+ *   kv_lens int32 [B] device array, or NULL: batch entry b uses cache rows
+ *           [0, L_b), L_b = kv_lens[b] (clamped to [0, Nk]); NULL means L_b = Nk.
+ *           Rows [L_b, Nk) are never weighted, whatever they hold.
+ * The new rows are the LAST Nq positions of a sequence of L_b tokens: with
+ * `causal`, position p (0-based among the Nq rows) sees cache row j iff
+ * j <= p + L_b - Nq (bottom-right alignment; Nq = Nk = L_b is attn_fwd's
+ * mask).  A row that sees no key (L_b = 0, or p + L_b - Nq < 0) gets O = 0 and
+ * LSE = -inf.  Query head h reads key/value head h / (H / H_kv).
+ * num_splits: key tiles of each (key/value head, 128 packed query rows) are
+ * cut into this many chunks, one CTA each, and the partial results are merged
+ * by their LSE; 0 picks a count that fills the GPU's 148 SMs.  With more than
+ * one split the call needs attn_fwd_kvcache_workspace_bytes() bytes of device
+ * workspace (16-byte aligned) for the fp32 partials, else ATTN_ERR_WORKSPACE;
+ * with one split `workspace` may be NULL.  Requires B*H*Nq < 2^31 - 128.
+ * Outputs must not alias inputs or the workspace.
+ */
+int attn_fwd_kvcache(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                     const int32_t* kv_lens,
+                     int64_t B, int64_t H, int64_t H_kv, int64_t Nq, int64_t Nk, int64_t d,
+                     int causal, float scale, int64_t num_splits,
+                     void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Number of key chunks attn_fwd_kvcache uses for these arguments (num_splits
+ * as passed to it, 0 = automatic), and the workspace bytes it then needs:
+ * splits * B*H*Nq * (d + 1) * 4 when splits > 1, else 0.  Both return 0 for
+ * sizes attn_fwd_kvcache would reject.
+ */
+int64_t attn_fwd_kvcache_splits(int64_t B, int64_t H, int64_t H_kv, int64_t Nq, int64_t Nk, int64_t d,
+                                int64_t num_splits);
+size_t attn_fwd_kvcache_workspace_bytes(int64_t B, int64_t H, int64_t H_kv, int64_t Nq, int64_t Nk, int64_t d,
+                                        int64_t num_splits);
+
+/*
  * Bytes of caller-provided device workspace that attn_bwd needs for these
  * sizes (two fp32 per-row vectors per head, each padded to a multiple of 128
  * rows).  Returns 0 for sizes that attn_bwd would reject.
@@ -122,6 +180,18 @@ int attn_bwd_gqa(const void* Q, const void* K, const void* V, const void* O, con
                  const float* LSE, void* dQ, void* dK, void* dV,
                  int64_t B, int64_t H, int64_t H_kv, int64_t N, int64_t d, int causal, float scale,
                  void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Backward of attn_fwd_blocksparse (same block_mask, same layouts as
+ * attn_bwd_gqa).  The dQ kernel visits only the key tiles a query tile
+ * selected; the dK/dV kernel visits only the (query head, query tile) pairs
+ * that selected its key tile.  Rows with LSE = -inf contribute nothing; key
+ * tiles that no query tile selected get dK = dV = 0.
+ */
+int attn_bwd_blocksparse(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                         const float* LSE, const uint8_t* block_mask, void* dQ, void* dK, void* dV,
+                         int64_t B, int64_t H, int64_t H_kv, int64_t N, int64_t d, int causal, float scale,
+                         void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * The three steps of attn_bwd, callable one at a time (same arguments and
@@ -185,6 +255,17 @@ int attn_bwd_static_workspace(const void* Q, const void* K, const void* V, const
                               const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
                               int64_t B, int64_t H, int64_t N, int64_t d, int causal, float scale,
                               void* stream);
+
+/*
+ * Self-test of the failure path (no counterpart on the pages: it checks the
+ * library's bounded waits).  Enqueues one small kernel that allocates tensor
+ * memory, waits on a barrier that nothing arrives on, gives up after 20 ms
+ * exactly as the attention kernels do when a wait runs out (it raises the
+ * device status word, releases its tensor memory and returns), so that the
+ * next attn_check_status() reports ATTN_ERR_TIMEOUT and the context stays
+ * usable.  Returns ATTN_OK once enqueued.  Nothing faults, traps or hangs.
+ */
+int attn_selftest_wait_timeout(void* stream);
 
 /*
  * Synchronises `stream`, then reports and clears the device status word:

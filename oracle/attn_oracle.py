@@ -50,6 +50,12 @@ __all__ = [
     "expand_kv",
     "attn_fwd_gqa",
     "attn_bwd_gqa",
+    "BLOCK",
+    "blocksparse_scores",
+    "masked_row_softmax",
+    "attn_fwd_blocksparse",
+    "attn_bwd_blocksparse",
+    "attn_fwd_kvcache",
 ]
 
 
@@ -185,3 +191,117 @@ def attn_bwd_gqa(Q, K, V, dO, scale: float, causal: bool, B: int, H: int, H_kv: 
     dK = dKe.reshape(B, H_kv, g, n, d).sum(axis=2).reshape(B * H_kv, n, d)
     dV = dVe.reshape(B, H_kv, g, n, d).sum(axis=2).reshape(B * H_kv, n, d)
     return dQ, dK, dV
+
+
+# ---------------------------------------------------------------------------
+# Block-sparse selection ("Attention and KV Compression", section "The
+# composability point": sparse selection changes which blocks are attended and
+# the kernel runs on the selected blocks).  A block mask M of shape
+# (B*H, ceil(N/T), ceil(N/T)), T = 128, marks which key tiles each query tile
+# attends; S_ij = -inf unless M[bh, i // T, j // T] (and j <= i when causal).
+# Rows left with no visible key have no softmax; their output is taken as
+# O = 0, LSE = -inf and they contribute no gradient (the reading used for
+# fully masked rows).
+# ---------------------------------------------------------------------------
+
+BLOCK = 128
+
+
+def blocksparse_scores(q, k, scale: float, causal: bool, mask_tiles: np.ndarray) -> np.ndarray:
+    """Scores of one head with the block mask (and causal mask) written in as -inf."""
+    s = head_scores(q, k, scale, causal)
+    n = s.shape[0]
+    tiles = np.arange(n) // BLOCK
+    keep = np.asarray(mask_tiles, dtype=bool)[tiles[:, None], tiles[None, :]]
+    s[~keep] = -np.inf
+    return s
+
+
+def masked_row_softmax(s: np.ndarray):
+    """row_softmax, extended to rows with no finite score: P = 0, LSE = -inf."""
+    m = np.max(s, axis=1, keepdims=True)
+    empty = ~np.isfinite(m[:, 0])
+    m_safe = np.where(empty[:, None], 0.0, m)
+    e = np.exp(s - m_safe)
+    l = np.sum(e, axis=1, keepdims=True)
+    p = np.where(empty[:, None], 0.0, e / np.where(empty[:, None], 1.0, l))
+    lse = np.where(empty, -np.inf, (m_safe + np.log(np.where(empty[:, None], 1.0, l)))[:, 0])
+    return p, lse
+
+
+def attn_fwd_blocksparse(Q, K, V, scale: float, causal: bool, mask, B: int, H: int, H_kv: int):
+    """Forward under a block mask (B*H, nt, nt); K, V have B*H_kv heads."""
+    Q = _as3(Q)
+    Ke, Ve = expand_kv(K, B, H, H_kv), expand_kv(V, B, H, H_kv)
+    bh, n, d = Q.shape
+    O = np.empty((bh, n, d))
+    LSE = np.empty((bh, n))
+    for h in range(bh):
+        p, lse = masked_row_softmax(blocksparse_scores(Q[h], Ke[h], scale, causal, mask[h]))
+        O[h] = p @ Ve[h]
+        LSE[h] = lse
+    return O, LSE
+
+
+def attn_bwd_blocksparse(Q, K, V, dO, scale: float, causal: bool, mask, B: int, H: int, H_kv: int):
+    """Backward under a block mask: dQ (B*H, N, d); dK, dV (B*H_kv, N, d)."""
+    Q, dO = _as3(Q), _as3(dO)
+    Ke, Ve = expand_kv(K, B, H, H_kv), expand_kv(V, B, H, H_kv)
+    bh, n, d = Q.shape
+    dQ = np.empty((bh, n, d))
+    dKe = np.empty((bh, n, d))
+    dVe = np.empty((bh, n, d))
+    for h in range(bh):
+        p, _ = masked_row_softmax(blocksparse_scores(Q[h], Ke[h], scale, causal, mask[h]))
+        dVe[h] = p.T @ dO[h]
+        dp = dO[h] @ Ve[h].T
+        D = np.sum(p * dp, axis=1, keepdims=True)
+        ds = p * (dp - D)
+        dQ[h] = float(scale) * (ds @ Ke[h])
+        dKe[h] = float(scale) * (ds.T @ Q[h])
+    g = H // H_kv
+    dK = dKe.reshape(B, H_kv, g, n, d).sum(axis=2).reshape(B * H_kv, n, d)
+    dV = dVe.reshape(B, H_kv, g, n, d).sum(axis=2).reshape(B * H_kv, n, d)
+    return dQ, dK, dV
+
+
+# ---------------------------------------------------------------------------
+# Decode-shaped attention against a key/value cache ("FlashAttention -- how
+# 100K-token attention fits in memory", section "Arithmetic intensity": prefill
+# and decode are the same computation in different shape regimes).  Nq new
+# query rows attend to the first L_b cached keys/values of their batch entry
+# (L_b = kv_lens[b], default Nk).  The queries are the LAST Nq positions of that
+# length-L_b sequence, so under the causal mask query p (0-based among the new
+# rows) sees key j iff j <= p + L_b - Nq (bottom-right alignment; with Nq = Nk
+# it is the square mask above).  Rows that see no key follow the fully masked
+# row reading: O = 0, LSE = -inf.  Keys past L_b do not exist for that batch
+# entry: they are sliced away before any arithmetic.
+# ---------------------------------------------------------------------------
+
+def attn_fwd_kvcache(Q, K, V, scale: float, causal: bool, B: int, H: int, H_kv: int, kv_lens=None):
+    """Q (B*H, Nq, d); K, V (B*H_kv, Nk, d); kv_lens (B,) or None -> O (B*H, Nq, d), LSE (B*H, Nq)."""
+    Q = _as3(Q)
+    Ke, Ve = expand_kv(K, B, H, H_kv), expand_kv(V, B, H, H_kv)
+    bh, nq, d = Q.shape
+    nk = Ke.shape[1]
+    lens = [nk] * B if kv_lens is None else [int(x) for x in kv_lens]
+    O = np.empty((bh, nq, d))
+    LSE = np.empty((bh, nq))
+    for h in range(bh):
+        L = lens[h // H]
+        if not 0 <= L <= nk:
+            raise ValueError("kv_lens entries must lie in [0, Nk]")
+        k, v = Ke[h, :L], Ve[h, :L]
+        s = float(scale) * (Q[h] @ k.T)                      # (Nq, L)
+        if causal:
+            p = np.arange(nq)[:, None]
+            j = np.arange(L)[None, :]
+            s[j > p + (L - nq)] = -np.inf
+        if L == 0:
+            O[h] = 0.0
+            LSE[h] = -np.inf
+            continue
+        pr, lse = masked_row_softmax(s)
+        O[h] = pr @ v
+        LSE[h] = lse
+    return O, LSE

@@ -115,3 +115,46 @@ def test_python_binding_validates_tensors():
     q = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         attn.attn_fwd(q, q, q, q, torch.zeros(1, 1, 8), False, 0.125)
+
+
+def test_kvcache_splits_and_workspace(lib):
+    # explicit counts are capped by the number of 128-row key tiles
+    assert attn.attn_fwd_kvcache_splits(1, 8, 8, 1, 1000, 128, 3) == 3
+    assert attn.attn_fwd_kvcache_splits(1, 8, 8, 1, 1000, 128, 50) == 8
+    assert attn.attn_fwd_kvcache_splits(1, 8, 8, 1, 100, 128, 0) == 1
+    # decode batch with 64 key/value heads over a 16K cache: many splits, all SMs busy
+    s = attn.attn_fwd_kvcache_splits(8, 32, 8, 1, 16384, 128, 0)
+    assert 2 <= s <= 128
+    assert attn.attn_fwd_kvcache_workspace_bytes(8, 32, 8, 1, 16384, 128, 0) == s * 8 * 32 * 1 * 129 * 4
+    # a large prefill-sized grid needs no split and no workspace
+    assert attn.attn_fwd_kvcache_splits(8, 32, 32, 512, 2048, 128, 0) == 1
+    assert attn.attn_fwd_kvcache_workspace_bytes(8, 32, 32, 512, 2048, 128, 0) == 0
+    # rejected sizes
+    assert attn.attn_fwd_kvcache_splits(1, 8, 3, 1, 100, 128, 0) == 0
+    assert attn.attn_fwd_kvcache_workspace_bytes(1, 8, 8, 1, 100, 96, 2) == 0
+    assert attn.attn_fwd_kvcache_splits(1, 8, 8, 0, 100, 128, 0) == 0
+
+
+def test_kvcache_argument_errors(lib):
+    p = [A] * 5
+
+    def call(B=1, H=4, Hk=2, Nq=1, Nk=256, d=64, scale=0.125, splits=1, ws=None, ws_bytes=0, lens=None, ptrs=None):
+        return lib.attn_fwd_kvcache(*(ptrs or p), lens, B, H, Hk, Nq, Nk, d, 1, scale, splits, ws, ws_bytes, None)
+
+    assert call(Nq=0) == attn.ATTN_ERR_INVALID_ARG
+    assert call(Nk=0) == attn.ATTN_ERR_INVALID_ARG
+    assert call(Hk=3) == attn.ATTN_ERR_INVALID_ARG
+    assert call(d=96) == attn.ATTN_ERR_UNSUPPORTED
+    assert call(scale=0.0) == attn.ATTN_ERR_INVALID_ARG
+    assert call(splits=-1) == attn.ATTN_ERR_INVALID_ARG
+    assert call(lens=ctypes.c_void_p(0x100002)) == attn.ATTN_ERR_MISALIGNED
+    for k in range(5):
+        q = [A] * 5
+        q[k] = MIS
+        assert call(ptrs=q) == attn.ATTN_ERR_MISALIGNED
+    # two splits need a workspace of the advertised size
+    need = attn.attn_fwd_kvcache_workspace_bytes(1, 4, 2, 1, 256, 64, 2)
+    assert need == 2 * 4 * 65 * 4
+    assert call(splits=2) == attn.ATTN_ERR_INVALID_ARG
+    assert call(splits=2, ws=MIS, ws_bytes=need) == attn.ATTN_ERR_MISALIGNED
+    assert call(splits=2, ws=A, ws_bytes=need - 4) == attn.ATTN_ERR_WORKSPACE

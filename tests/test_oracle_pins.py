@@ -483,3 +483,179 @@ def test_gqa_matches_torch_autograd_fp64():
     np.testing.assert_allclose(dQ, tq.grad.numpy().reshape(B * H, N, d), rtol=1e-11, atol=1e-12)
     np.testing.assert_allclose(dK, tk.grad.numpy().reshape(B * H_kv, N, d), rtol=1e-11, atol=1e-12)
     np.testing.assert_allclose(dV, tv.grad.numpy().reshape(B * H_kv, N, d), rtol=1e-11, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# Block-sparse selection
+# ---------------------------------------------------------------------------
+
+def _bs_case(B, H, Hk, N, d, seed):
+    return (_rand((B * H, N, d), seed), _rand((B * Hk, N, d), seed + 1), _rand((B * Hk, N, d), seed + 2),
+            _rand((B * H, N, d), seed + 3))
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_blocksparse_all_selected_is_dense(causal):
+    B, H, N, d = 1, 2, 300, 4
+    q, k, v, g = _bs_case(B, H, H, N, d, 400)
+    nt = -(-N // orc.BLOCK)
+    mask = np.ones((B * H, nt, nt), dtype=np.uint8)
+    O1, L1 = orc.attn_fwd_blocksparse(q, k, v, 0.3, causal, mask, B, H, H)
+    O2, L2 = orc.attn_fwd(q, k, v, 0.3, causal)
+    np.testing.assert_array_equal(O1, O2)
+    np.testing.assert_array_equal(L1, L2)
+    for x, y in zip(orc.attn_bwd_blocksparse(q, k, v, g, 0.3, causal, mask, B, H, H),
+                    orc.attn_bwd(q, k, v, g, 0.3, causal)):
+        np.testing.assert_allclose(x, y, rtol=1e-13, atol=1e-14)
+
+
+def test_blocksparse_single_block_is_dense_attention_on_that_block():
+    # each query tile selects exactly one key tile: its rows are dense attention
+    # over that tile's 128 keys alone (the plain MHA oracle on sliced K, V)
+    N, d, T = 384, 3, orc.BLOCK
+    q, k, v, _ = _bs_case(1, 1, 1, N, d, 410)
+    choice = [2, 0, 1]
+    mask = np.zeros((1, 3, 3), dtype=np.uint8)
+    for i, j in enumerate(choice):
+        mask[0, i, j] = 1
+    O, L = orc.attn_fwd_blocksparse(q, k, v, 0.5, False, mask, 1, 1, 1)
+    for i, j in enumerate(choice):
+        rows = slice(i * T, (i + 1) * T)
+        keys = slice(j * T, (j + 1) * T)
+        s = 0.5 * (q[0, rows] @ k[0, keys].T)
+        m = s.max(axis=1, keepdims=True)
+        e = np.exp(s - m)
+        np.testing.assert_allclose(O[0, rows], (e / e.sum(1, keepdims=True)) @ v[0, keys], rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(L[0, rows], (m + np.log(e.sum(1, keepdims=True)))[:, 0], rtol=1e-13)
+
+
+def test_blocksparse_empty_rows_give_zero_output_and_no_gradient():
+    N, d = 256, 4
+    q, k, v, g = _bs_case(1, 1, 1, N, d, 420)
+    mask = np.zeros((1, 2, 2), dtype=np.uint8)
+    mask[0, 1, 0] = 1                     # query tile 0 selects nothing
+    O, L = orc.attn_fwd_blocksparse(q, k, v, 0.5, True, mask, 1, 1, 1)
+    assert (O[0, :128] == 0).all() and np.isneginf(L[0, :128]).all()
+    assert np.isfinite(O[0, 128:]).all() and np.isfinite(L[0, 128:]).all()
+    dQ, dK, dV = orc.attn_bwd_blocksparse(q, k, v, g, 0.5, True, mask, 1, 1, 1)
+    assert (dQ[0, :128] == 0).all()
+    assert (dK[0, 128:] == 0).all() and (dV[0, 128:] == 0).all()   # key tile 1 is never selected
+
+
+def test_blocksparse_backward_matches_central_differences():
+    B, H, Hk, N, d, scale = 1, 2, 1, 260, 2, 0.7
+    q, k, v, g = _bs_case(B, H, Hk, N, d, 430)
+    rng = np.random.default_rng(431)
+    mask = (rng.random((B * H, 3, 3)) < 0.6).astype(np.uint8)
+    mask[0, 1, :] = 0                      # one empty query tile
+    dQ, dK, dV = orc.attn_bwd_blocksparse(q, k, v, g, scale, True, mask, B, H, Hk)
+
+    def loss(q_, k_, v_):
+        O, _ = orc.attn_fwd_blocksparse(q_, k_, v_, scale, True, mask, B, H, Hk)
+        return float(np.sum(O * g))
+
+    h = 1e-6
+    pick = [(0, 0, 0), (0, 129, 1), (0, 259, 0), (1, 200, 1), (1, 5, 0)]
+    for name, x, grad in (("q", q, dQ), ("k", k, dK), ("v", v, dV)):
+        for idx in pick:
+            if idx[0] >= x.shape[0]:
+                continue
+            a = {"q_": q, "k_": k, "v_": v}
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            a[name + "_"] = xp
+            fp = loss(**a)
+            a[name + "_"] = xm
+            fm = loss(**a)
+            assert abs((fp - fm) / (2 * h) - grad[idx]) <= 1e-6 * max(1.0, abs(grad[idx])), (name, idx)
+
+
+# ---------------------------------------------------------------------------
+# Key/value cache (decode-shaped) forward
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_kvcache_with_as_many_queries_as_keys_is_plain_attention(causal):
+    B, H, N, d = 1, 2, 37, 3
+    q, k, v, _ = _bs_case(B, H, H, N, d, 500)
+    O1, L1 = orc.attn_fwd_kvcache(q, k, v, 0.4, causal, B, H, H)
+    O2, L2 = orc.attn_fwd(q, k, v, 0.4, causal)
+    np.testing.assert_allclose(O1, O2, rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(L1, L2, rtol=1e-13, atol=1e-14)
+
+
+@pytest.mark.parametrize("nq", [1, 3, 16])
+def test_kvcache_queries_are_the_last_rows_of_the_sequence(nq):
+    # the cache holds all L keys; the new queries are the last nq rows of a
+    # length-L causal attention whose earlier query rows are arbitrary
+    L, d = 29, 4
+    q_full = _rand((1, L, d), 510)
+    k, v = _rand((1, L, d), 511), _rand((1, L, d), 512)
+    O_full, L_full = orc.attn_fwd(q_full, k, v, 0.6, True)
+    O, LSE = orc.attn_fwd_kvcache(q_full[:, L - nq:], k, v, 0.6, True, 1, 1, 1)
+    np.testing.assert_allclose(O, O_full[:, L - nq:], rtol=1e-13, atol=1e-14)
+    np.testing.assert_allclose(LSE, L_full[:, L - nq:], rtol=1e-13, atol=1e-14)
+
+
+def test_kvcache_single_query_brute_force():
+    # one query against five cached keys, every sum written out by hand
+    q = [0.3, -1.2, 0.7]
+    ks = [[1.0, 0.5, -0.2], [-0.4, 0.1, 0.9], [0.0, -1.0, 0.3], [0.8, 0.8, 0.8], [-0.5, 0.2, -0.1]]
+    vs = [[1.0, 2.0, 3.0], [-1.0, 0.0, 1.0], [0.5, 0.5, 0.5], [2.0, -2.0, 0.0], [0.0, 1.0, -1.0]]
+    scale = 0.9
+    for causal in (False, True):
+        e = [math.exp(scale * sum(a * b for a, b in zip(q, kj))) for kj in ks]
+        tot = sum(e)
+        o_ref = [sum(e[j] * vs[j][c] for j in range(5)) / tot for c in range(3)]
+        O, LSE = orc.attn_fwd_kvcache(np.array([[q]]), np.array([ks]), np.array([vs]), scale, causal, 1, 1, 1)
+        np.testing.assert_allclose(O[0, 0], o_ref, rtol=1e-14)
+        assert abs(LSE[0, 0] - math.log(tot)) < 1e-14
+
+
+def test_kvcache_lengths_truncate_the_cache():
+    # entries past kv_lens[b] are never read, even when they hold NaN
+    B, H, Hk, nq, nk, d = 3, 4, 2, 5, 40, 3
+    q = _rand((B * H, nq, d), 520)
+    k, v = _rand((B * Hk, nk, d), 521), _rand((B * Hk, nk, d), 522)
+    lens = [40, 17, 6]
+    kn, vn = k.copy(), v.copy()
+    for b, L in enumerate(lens):
+        kn[b * Hk:(b + 1) * Hk, L:] = np.nan
+        vn[b * Hk:(b + 1) * Hk, L:] = np.nan
+    for causal in (False, True):
+        O, LSE = orc.attn_fwd_kvcache(q, kn, vn, 0.5, causal, B, H, Hk, kv_lens=lens)
+        for b, L in enumerate(lens):
+            qs = slice(b * H, (b + 1) * H)
+            ks = slice(b * Hk, (b + 1) * Hk)
+            Ob, Lb = orc.attn_fwd_kvcache(q[qs], k[ks, :L], v[ks, :L], 0.5, causal, 1, H, Hk)
+            np.testing.assert_array_equal(O[qs], Ob)
+            np.testing.assert_array_equal(LSE[qs], Lb)
+
+
+def test_kvcache_group_heads_read_their_shared_head():
+    B, H, Hk, nq, nk, d = 2, 6, 2, 3, 11, 4
+    q = _rand((B * H, nq, d), 530)
+    k, v = _rand((B * Hk, nk, d), 531), _rand((B * Hk, nk, d), 532)
+    O, LSE = orc.attn_fwd_kvcache(q, k, v, 0.5, True, B, H, Hk)
+    for b in range(B):
+        for h in range(H):
+            kv = b * Hk + h // (H // Hk)
+            Oh, Lh = orc.attn_fwd_kvcache(q[b * H + h], k[kv], v[kv], 0.5, True, 1, 1, 1)
+            np.testing.assert_array_equal(O[b * H + h], Oh[0])
+            np.testing.assert_array_equal(LSE[b * H + h], Lh[0])
+
+
+def test_kvcache_shorter_cache_than_queries_leaves_empty_rows():
+    nq, d = 6, 3
+    q = _rand((1, nq, d), 540)
+    k, v = _rand((1, 10, d), 541), _rand((1, 10, d), 542)
+    O, LSE = orc.attn_fwd_kvcache(q, k, v, 0.5, True, 1, 1, 1, kv_lens=[4])
+    # rows p < nq - L see no key; row p >= nq - L sees keys 0 .. p - (nq - L)
+    assert (O[0, :2] == 0).all() and np.isneginf(LSE[0, :2]).all()
+    for p in range(2, nq):
+        s = 0.5 * (q[0, p] @ k[0, :p - 1].T)
+        e = np.exp(s - s.max())
+        np.testing.assert_allclose(O[0, p], e @ v[0, :p - 1] / e.sum(), rtol=1e-13)
+    O0, L0 = orc.attn_fwd_kvcache(q, k, v, 0.5, False, 1, 1, 1, kv_lens=[0])
+    assert (O0 == 0).all() and np.isneginf(L0).all()

@@ -54,6 +54,7 @@ KERNEL_SOURCES = {
     "bwd_pre": ("attn_bwd.cuh", "sm100.cuh"),
     "bwd_dkdv": ("attn_bwd.cuh", "sm100.cuh"),
     "bwd_dq": ("attn_bwd.cuh", "sm100.cuh"),
+    "kvcache": ("attn_kvcache.cuh", "sm100.cuh"),
 }
 
 
@@ -360,9 +361,45 @@ def run_ours(args, rank, world, local_rank):
             gbs = alg_bytes / (t_us * 1e-6) / 1e9
             kvcache[name] = {"splits": splits, "us": round(t_us, 2), "alg_bytes": alg_bytes,
                              "gb_s": round(gbs, 1), "frac": round(gbs / hbm, 4), "calls": n_d,
+                             "traffic": recorded_traffic("kvcache") if lens is None else None,
                              "kv_lens": None if lens is None else "uniform in [N/2, N] per batch entry"}
             del wsd
         del kc, vc
+
+    # ---------------------------------------------------- FP8 (E4M3) forward
+    # Same workload and FLOP count as the bf16 forward, inputs quantised per
+    # tensor to E4M3; its tensor peak is the measured bf16 peak x 2 (the
+    # nominal E4M3 : BF16 dense ratio, 4.5 : 2.25 PFLOP/s).
+    fp8 = None
+    if not args.no_fp8 and w.d == 128:
+        def q8(x):
+            ds = float(x.abs().amax()) / 448.0
+            return (x.float() / ds).to(torch.float8_e4m3fn), ds
+
+        (qf, dq8), (kf, dk8), (vf, dv8) = q8(q), q8(k), q8(v)
+
+        def fp8_fwd():
+            attn.attn_fwd_fp8(qf, kf, vf, o, lse, causal, scale, dq8, dk8, dv8, stream)
+
+        for _ in range(args.warmup):
+            fp8_fwd()
+        n_f = max(3, min(args.steps, 5))
+        fev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n_f)]
+        torch.cuda.synchronize()
+        for e in fev:
+            e[0].record(stream)
+            fp8_fwd()
+            e[1].record(stream)
+        torch.cuda.synchronize()
+        assert attn.attn_check_status(stream) == attn.ATTN_OK
+        tf = sum(e[0].elapsed_time(e[1]) for e in fev) / n_f
+        tf = max_over_ranks([tf], device=dev)[0]
+        fp8_tf = aggregate_tflops(f_fwd, world, tf)
+        fp8 = {"workload": "long_batch forward on E4M3 Q, K, V (per-tensor scales)", "ms_fwd": round(tf, 3),
+               "fwd_tflops": round(fp8_tf, 2), "peak": round(2 * burst, 1),
+               "peak_kind": f"2 x bf16_tflops ({peaks_src}), nominal E4M3:BF16 ratio",
+               "frac": round(fp8_tf / (2 * burst), 4), "steps": n_f}
+        del qf, kf, vf
 
     # ---------------------------------------------------------------- e2e
     # Through host buffers: every step copies its inputs Q, K, V, dO from
@@ -469,6 +506,7 @@ def run_ours(args, rank, world, local_rank):
         "gqa": gqa,
         "block_sparse": sparse,
         "kvcache": kvcache,
+        "fp8": fp8,
         "gpu_launches": 4 * args.steps,
         "clocks": clk,
         "e2e": e2e,
@@ -560,6 +598,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-gqa", action="store_true", help="skip the shared key/value head measurement")
     ap.add_argument("--no-kvcache", action="store_true", help="skip the decode (key/value cache) measurement")
+    ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 forward measurement")
     ap.add_argument("--gqa-kv-heads", type=int, default=8)
     ap.add_argument("--no-sparse", action="store_true", help="skip the block-sparse measurement")
     ap.add_argument("--sparse-window", type=int, default=16)

@@ -31,7 +31,7 @@ ATTN_ERR_TIMEOUT = -6
 ATTN_ERR_DEVICE = -7
 
 EXPORTED = ("attn_fwd", "attn_fwd_gqa", "attn_fwd_blocksparse", "attn_bwd", "attn_bwd_gqa", "attn_bwd_blocksparse",
-            "attn_bwd_workspace_bytes", "attn_fwd_kvcache", "attn_fwd_kvcache_splits",
+            "attn_bwd_workspace_bytes", "attn_fwd_fp8", "attn_fwd_kvcache", "attn_fwd_kvcache_splits",
             "attn_fwd_kvcache_workspace_bytes",
             "attn_bwd_preprocess", "attn_bwd_dkdv",
             "attn_bwd_dq", "attn_bwd_static_workspace", "attn_check_status", "attn_last_error",
@@ -75,6 +75,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.attn_bwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i32, f32,
                                          vp, ctypes.c_size_t, vp]
     lib.attn_bwd_blocksparse.restype = i32
+    lib.attn_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i32, f32, f32, f32, f32, vp]
+    lib.attn_fwd_fp8.restype = i32
     lib.attn_fwd_kvcache.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i32, f32, i64, vp,
                                      ctypes.c_size_t, vp]
     lib.attn_fwd_kvcache.restype = i32
@@ -239,6 +241,30 @@ def attn_bwd_blocksparse(Q, K, V, O, dO, LSE, block_mask, dQ, dK, dV, causal: bo
                                              int(bool(causal)), float(scale), wp, wb, _stream_handle(stream))
     if st != ATTN_OK:
         raise AttnError(st, "attn_bwd_blocksparse")
+
+
+def attn_fwd_fp8(Q8, K8, V8, O, LSE, causal: bool, scale: float, q_descale: float, k_descale: float,
+                 v_descale: float, stream=None) -> None:
+    """O (bf16), LSE <- attention of the dequantised E4M3 tensors descale * X8.
+
+    Q8 (B, H, N, 128) and K8, V8 (B, H_kv, N, 128) are torch.float8_e4m3fn
+    (or uint8 holding E4M3 codes) CUDA tensors; O is bf16 (B, H, N, 128).
+    """
+    for name, t in (("Q8", Q8), ("K8", K8), ("V8", V8)):
+        if not t.is_cuda or t.dtype not in (torch.float8_e4m3fn, torch.uint8) or t.dim() != 4 \
+                or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA float8_e4m3fn (or uint8) tensor of rank 4")
+    _check_bhnd("O", O, Q8.shape)
+    _check_lse(LSE, Q8.shape)
+    B, H, N, d = Q8.shape
+    if K8.shape != V8.shape or K8.shape[0] != B or K8.shape[2] != N or K8.shape[3] != d or K8.shape[1] < 1 \
+            or H % K8.shape[1] != 0:
+        raise ValueError(f"K8, V8 have shapes {tuple(K8.shape)}, {tuple(V8.shape)}; expected (B, H_kv, N, d)")
+    st = load_library().attn_fwd_fp8(_ptr(Q8), _ptr(K8), _ptr(V8), _ptr(O), _ptr(LSE), B, H, K8.shape[1], N, d,
+                                     int(bool(causal)), float(scale), float(q_descale), float(k_descale),
+                                     float(v_descale), _stream_handle(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd_fp8")
 
 
 def attn_fwd_kvcache_splits(B: int, H: int, H_kv: int, Nq: int, Nk: int, d: int, num_splits: int = 0) -> int:

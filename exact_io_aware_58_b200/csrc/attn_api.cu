@@ -18,6 +18,7 @@
 #include "../../include/attn.h"
 #include "attn_bwd.cuh"
 #include "attn_fwd.cuh"
+#include "attn_fwd_fp8.cuh"
 #include "attn_kvcache.cuh"
 
 namespace {
@@ -61,6 +62,28 @@ bool make_map(CUtensorMap* m, const void* base, int64_t bh, int64_t n, int64_t d
   const cuuint32_t box[3] = {64, cuuint32_t(box_rows), 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    fail(ATTN_ERR_LAUNCH, "%scuTensorMapEncodeTiled returned CUresult %lld", "", (long long)r);
+    return false;
+  }
+  return true;
+}
+
+// 3-D map over an E4M3 (byte) BHND tensor with d = 128: box = one 128-byte
+// row x 128 rows x 1 head, 128-byte swizzle.  Rows past N read as zeros.
+bool make_map_u8(CUtensorMap* m, const void* base, int64_t bh, int64_t n, int64_t d) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) {
+    fail(ATTN_ERR_LAUNCH, "%sdriver entry point cuTensorMapEncodeTiled unavailable%lld", "", 0);
+    return false;
+  }
+  const cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(n), cuuint64_t(bh)};
+  const cuuint64_t strides[2] = {cuuint64_t(d), cuuint64_t(n * d)};
+  const cuuint32_t box[3] = {128, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
@@ -383,6 +406,63 @@ ATTN_EXPORT int attn_bwd_blocksparse(const void* Q, const void* K, const void* V
   if (!block_mask) return ATTN_ERR_INVALID_ARG;
   return bwd_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, block_mask, B, H, H_kv, N, d, causal, scale, workspace,
                   workspace_bytes, stream);
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Forward on FP8 (E4M3) inputs with per-tensor dequantisation factors.
+// ---------------------------------------------------------------------------
+namespace {
+
+template <bool CAUSAL>
+int launch_fp8(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const attn::Fp8Params& prm,
+               int grid, cudaStream_t st) {
+  auto kern = attn::attn_fwd_fp8_kernel<CAUSAL>;
+  constexpr int smem = attn::Fp8Cfg::kSmemBytes;
+  if (set_smem(reinterpret_cast<const void*>(kern), smem) != ATTN_OK) return ATTN_ERR_LAUNCH;
+  kern<<<grid, attn::Fp8Cfg::kThreads, smem, st>>>(q, k, v, prm);
+  return launch_status();
+}
+
+bool positive_finite(float x) { return std::isfinite(x) && x > 0.f; }
+
+}  // namespace
+
+extern "C" {
+
+ATTN_EXPORT int attn_fwd_fp8(const void* Q8, const void* K8, const void* V8, void* O, float* LSE, int64_t B,
+                             int64_t H, int64_t H_kv, int64_t N, int64_t d, int causal, float scale,
+                             float q_descale, float k_descale, float v_descale, void* stream) {
+  int s = check_sizes(B, H, N, d);
+  if (s != ATTN_OK) return s;
+  if (d != 128) return fail(ATTN_ERR_UNSUPPORTED, "%sattn_fwd_fp8 supports d = 128 only (got %lld)", "", (long long)d);
+  if ((s = check_heads(H, H_kv)) != ATTN_OK) return s;
+  if ((s = check_scale(scale)) != ATTN_OK) return s;
+  if (!positive_finite(q_descale) || !positive_finite(k_descale) || !positive_finite(v_descale))
+    return ATTN_ERR_INVALID_ARG;
+  if (!Q8 || !K8 || !V8 || !O || !LSE) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(Q8) || !aligned16(K8) || !aligned16(V8) || !aligned16(O) || !aligned16(LSE))
+    return ATTN_ERR_MISALIGNED;
+  const int64_t bh = B * H, bhkv = B * H_kv;
+  CUtensorMap mq, mk, mv;
+  if (!make_map_u8(&mq, Q8, bh, N, d) || !make_map_u8(&mk, K8, bhkv, N, d) || !make_map_u8(&mv, V8, bhkv, N, d))
+    return ATTN_ERR_LAUNCH;
+  attn::Fp8Params prm;
+  prm.o = static_cast<__nv_bfloat16*>(O);
+  prm.lse = LSE;
+  prm.n = int(N);
+  prm.n_mblk = int((N + 255) / 256);
+  prm.h = int(H);
+  prm.h_kv = int(H_kv);
+  prm.group = int(H / H_kv);
+  prm.c = float(double(scale) * double(q_descale) * double(k_descale) * 1.4426950408889634);
+  prm.v_descale = v_descale;
+  if (!std::isfinite(prm.c) || !(prm.c > 0.f)) return ATTN_ERR_INVALID_ARG;
+  const int64_t grid = bh * prm.n_mblk;
+  if (grid > INT32_MAX) return ATTN_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return causal ? launch_fp8<true>(mq, mk, mv, prm, int(grid), st) : launch_fp8<false>(mq, mk, mv, prm, int(grid), st);
 }
 
 }  // extern "C"

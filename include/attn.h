@@ -100,6 +100,27 @@ int attn_fwd_blocksparse(const void* Q, const void* K, const void* V, void* O, f
                          float scale, void* stream);
 
 /*
+ * Forward on FP8 inputs ("Attention and KV Compression", section "What it
+ * does and does not change": later versions add narrower numeric formats;
+ * the computation is unchanged).
+ *   Q8       uint8 [B][H][N][128]   E4M3 codes (OCP FP8 E4M3: bias 7, no inf)
+ *   K8, V8   uint8 [B][H_kv][N][128]
+ *   O        bf16  [B][H][N][128],  LSE fp32 [B][H][N] (natural log)
+ * The attention is that of attn_fwd_gqa on the dequantised tensors
+ * Q = q_descale * Q8, K = k_descale * K8, V = v_descale * V8 (each descale
+ * finite and > 0).  QK^T and PV run on the E4M3 tensor-core path with fp32
+ * accumulation; the products Q8 K8^T are exact, and the row max, row sum and
+ * LSE are fp32.  P is rounded to E4M3 for the PV product (each p changes by at
+ * most 2^-4 of itself or 2^-10 absolute, p <= 2^8), so per row
+ * |O - O_exact| <= v_descale * max|V8| * (2^-4 + n_visible * 2^-10 / l) where
+ * l = sum_j exp(S_ij - max_j S_ij), plus the bf16 rounding of O.
+ * d must be 128 (else ATTN_ERR_UNSUPPORTED).  Other rules as attn_fwd.
+ */
+int attn_fwd_fp8(const void* Q8, const void* K8, const void* V8, void* O, float* LSE,
+                 int64_t B, int64_t H, int64_t H_kv, int64_t N, int64_t d, int causal, float scale,
+                 float q_descale, float k_descale, float v_descale, void* stream);
+
+/*
  * Forward of Nq new query rows against a key/value cache (decode and
  * chunked-prefill shapes: "FlashAttention -- how 100K-token attention fits in
  * memory", section "Arithmetic intensity", where prefill and decode are the

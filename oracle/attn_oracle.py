@@ -56,6 +56,8 @@ __all__ = [
     "attn_fwd_blocksparse",
     "attn_bwd_blocksparse",
     "attn_fwd_kvcache",
+    "e4m3_decode",
+    "attn_fwd_fp8",
 ]
 
 
@@ -305,3 +307,38 @@ def attn_fwd_kvcache(Q, K, V, scale: float, causal: bool, B: int, H: int, H_kv: 
         O[h] = pr @ v
         LSE[h] = lse
     return O, LSE
+
+
+# ---------------------------------------------------------------------------
+# Narrower input format: FP8 E4M3 ("Attention and KV Compression", section
+# "What it does and does not change": later versions add support for narrower
+# numeric formats; the computation itself is unchanged).  Each of Q, K, V is
+# given as E4M3 codes plus one per-tensor dequantisation factor; the attention
+# is the plain definition above applied to the dequantised values
+# X = descale_X * decode(X8).
+# ---------------------------------------------------------------------------
+
+def e4m3_decode(codes) -> np.ndarray:
+    """E4M3 byte codes -> float64 values, from the format's definition.
+
+    1 sign bit, 4 exponent bits (bias 7), 3 mantissa bits; exponent field 0
+    holds subnormals m/8 * 2^-6; exponent 15 with mantissa 7 is NaN (the only
+    special code: no infinities), so the largest finite magnitude is
+    1.75 * 2^8 = 448.
+    """
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 0x7).astype(np.float64)
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 7.0))
+    mag = np.where((e == 15) & ((c & 0x7) == 7), np.nan, mag)
+    return sign * mag
+
+
+def attn_fwd_fp8(Q8, K8, V8, q_descale: float, k_descale: float, v_descale: float, scale: float, causal: bool,
+                 B: int, H: int, H_kv: int):
+    """Forward on E4M3 inputs: Q8 (B*H, N, d), K8, V8 (B*H_kv, N, d) uint8 codes."""
+    Q = float(q_descale) * e4m3_decode(Q8)
+    K = float(k_descale) * e4m3_decode(K8)
+    V = float(v_descale) * e4m3_decode(V8)
+    return attn_fwd_gqa(Q, K, V, scale, causal, B, H, H_kv)

@@ -158,3 +158,21 @@ def test_kvcache_argument_errors(lib):
     assert call(splits=2) == attn.ATTN_ERR_INVALID_ARG
     assert call(splits=2, ws=MIS, ws_bytes=need) == attn.ATTN_ERR_MISALIGNED
     assert call(splits=2, ws=A, ws_bytes=need - 4) == attn.ATTN_ERR_WORKSPACE
+
+
+def test_fp8_argument_errors(lib):
+    p = [A] * 5
+
+    def call(d=128, dq=1.0, dk=1.0, dv=1.0, ptrs=None, Hk=2):
+        return lib.attn_fwd_fp8(*(ptrs or p), 1, 4, Hk, 256, d, 1, 0.125, dq, dk, dv, None)
+
+    assert call(d=64) == attn.ATTN_ERR_UNSUPPORTED
+    assert call(Hk=3) == attn.ATTN_ERR_INVALID_ARG
+    for bad in (0.0, -1.0, float("inf"), float("nan")):
+        assert call(dq=bad) == attn.ATTN_ERR_INVALID_ARG
+        assert call(dk=bad) == attn.ATTN_ERR_INVALID_ARG
+        assert call(dv=bad) == attn.ATTN_ERR_INVALID_ARG
+    for k in range(5):
+        q = [A] * 5
+        q[k] = MIS
+        assert call(ptrs=q) == attn.ATTN_ERR_MISALIGNED

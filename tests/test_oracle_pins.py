@@ -659,3 +659,45 @@ def test_kvcache_shorter_cache_than_queries_leaves_empty_rows():
         np.testing.assert_allclose(O[0, p], e @ v[0, :p - 1] / e.sum(), rtol=1e-13)
     O0, L0 = orc.attn_fwd_kvcache(q, k, v, 0.5, False, 1, 1, 1, kv_lens=[0])
     assert (O0 == 0).all() and np.isneginf(L0).all()
+
+
+# ---------------------------------------------------------------------------
+# FP8 (E4M3) inputs
+# ---------------------------------------------------------------------------
+
+def test_e4m3_decode_matches_torch_for_every_code():
+    import torch
+    codes = np.arange(256, dtype=np.uint8)
+    ours = orc.e4m3_decode(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    nan = np.isnan(ref)
+    assert (np.isnan(ours) == nan).all() and nan.sum() == 2          # 0x7F and 0xFF
+    np.testing.assert_array_equal(ours[~nan], ref[~nan])
+
+
+def test_e4m3_decode_landmarks():
+    d = orc.e4m3_decode
+    assert d([0x38])[0] == 1.0                  # exponent field 7 = bias, mantissa 0
+    assert d([0x7E])[0] == 448.0                # largest finite
+    assert d([0x01])[0] == 2.0 ** -9            # smallest subnormal
+    assert d([0x08])[0] == 2.0 ** -6            # smallest normal
+    assert d([0xB8])[0] == -1.0
+    assert d([0x00])[0] == 0.0 and np.signbit(d([0x80])[0])
+
+
+def test_fp8_forward_is_attention_on_dequantised_values():
+    # codes chosen so the dequantised tensors are known exactly: code 0x38 + k
+    # (k < 8) is 1 + k/8, and every descale is a power of two
+    rng = np.random.default_rng(600)
+    B, H, Hk, N, d = 1, 2, 1, 20, 4
+    q8 = (0x38 + rng.integers(0, 8, (B * H, N, d))).astype(np.uint8)
+    k8 = (0x30 + rng.integers(0, 8, (B * Hk, N, d))).astype(np.uint8)     # 0x30 + k = (1 + k/8) / 2
+    v8 = (0xB8 + rng.integers(0, 8, (B * Hk, N, d))).astype(np.uint8)     # negative values
+    Qd = 0.5 * (1 + (q8 - 0x38) / 8.0)
+    Kd = 4.0 * 0.5 * (1 + (k8 - 0x30) / 8.0)
+    Vd = 0.25 * -(1 + (v8 - 0xB8) / 8.0)
+    for causal in (False, True):
+        O, L = orc.attn_fwd_fp8(q8, k8, v8, 0.5, 4.0, 0.25, 0.3, causal, B, H, Hk)
+        O2, L2 = orc.attn_fwd_gqa(Qd, Kd, Vd, 0.3, causal, B, H, Hk)
+        np.testing.assert_allclose(O, O2, rtol=1e-14)
+        np.testing.assert_allclose(L, L2, rtol=1e-14)

@@ -472,7 +472,7 @@ ATTN_EXPORT int attn_fwd_fp8(const void* Q8, const void* K8, const void* V8, voi
 // ---------------------------------------------------------------------------
 namespace {
 
-constexpr int64_t kNumSMs = 148;        // B200; only the automatic split count depends on it
+constexpr int64_t kNumSMs = 148;   // B200: sizes the persistent grid and the automatic split count
 constexpr int64_t kMaxSplits = 256;
 
 struct KvcShape {
@@ -496,8 +496,9 @@ int kvc_check(int64_t B, int64_t H, int64_t H_kv, int64_t Nq, int64_t Nk, int64_
 }
 
 // Splits: explicit counts are capped at the number of key tiles; the automatic
-// count minimises (waves of CTAs over the SMs) x (key tiles per CTA + 1), the
-// +1 standing for a CTA's fixed cost (setup, pipeline fill, partial write).
+// count minimises (work items per SM, rounded up) x (key tiles per item +
+// 1/4), the 1/4 standing for an item's fixed cost in the persistent kernel
+// (its partial write and the merge traffic).
 int64_t kvc_splits(const KvcShape& sh, int64_t B, int64_t H_kv, int64_t num_splits) {
   if (num_splits < 0) return 0;
   const int64_t cap = std::min(sh.tiles, kMaxSplits);
@@ -507,7 +508,7 @@ int64_t kvc_splits(const KvcShape& sh, int64_t B, int64_t H_kv, int64_t num_spli
   for (int64_t sp = 1; sp <= cap; ++sp) {
     const int64_t per = (sh.tiles + sp - 1) / sp;
     const int64_t waves = (base * sp + kNumSMs - 1) / kNumSMs;
-    const int64_t cost = waves * (per + 1);
+    const int64_t cost = waves * (4 * per + 1);
     if (cost < best_cost) {
       best_cost = cost;
       best_s = sp;
@@ -581,8 +582,9 @@ ATTN_EXPORT int attn_fwd_kvcache(const void* Q, const void* K, const void* V, vo
     if (!aligned16(workspace)) return ATTN_ERR_MISALIGNED;
     if (workspace_bytes < kvc_workspace(sh, splits, d)) return ATTN_ERR_WORKSPACE;
   }
-  const int64_t grid = B * H_kv * sh.n_rt * splits;
-  if (grid > INT32_MAX) return ATTN_ERR_INVALID_ARG;
+  const int64_t n_items = B * H_kv * sh.n_rt * splits;
+  if (n_items > INT32_MAX) return ATTN_ERR_INVALID_ARG;
+  const int64_t grid = std::min<int64_t>(n_items, kNumSMs);     // persistent: one CTA per SM
   const int qbox = int(std::min<int64_t>(128, (sh.rows + 7) / 8 * 8));
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, Q, 1, sh.total_rows, d, qbox) || !make_map(&mk, K, B * H_kv, Nk, d) ||
@@ -602,6 +604,7 @@ ATTN_EXPORT int attn_fwd_kvcache(const void* Q, const void* K, const void* V, vo
   prm.n_rt = int(sh.n_rt);
   prm.splits = int(splits);
   prm.qbox = qbox;
+  prm.n_items = int(n_items);
   prm.scale_log2 = scale * 1.4426950408889634f;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return ATTN_KVC_DISPATCH(mq, mk, mv, prm, int(grid), st);

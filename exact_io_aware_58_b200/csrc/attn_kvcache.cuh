@@ -9,20 +9,21 @@
 // key and value is used by only a handful of query rows, so the kernel is bound
 // by reading the cache from HBM, not by the tensor cores.
 //
-// B200 mapping (one CTA = one 128-row tile of PACKED query rows x one chunk of
-// key tiles, 192 threads, one CTA per SM):
+// B200 mapping (work item = one 128-row tile of PACKED query rows x one chunk
+// of key tiles; a persistent grid of one 192-thread CTA per SM walks the items):
 //   * The g = H / H_kv query heads that share a key/value head, and their Nq
 //     rows each, are packed into the rows of one MMA tile: packed row r is head
 //     kvh*g + r / Nq, position r % Nq.  In a BHND tensor these rows are
 //     contiguous, so one TMA box loads them and every cached tile is read once
 //     per packed tile instead of once per query head.
 //   * Split-KV: the key tiles of a (kv head, row tile) are cut into `splits`
-//     contiguous chunks, one CTA each, so that a decode batch with few heads
-//     still covers all SMs.  Each CTA writes an fp32 partial O (normalised by
+//     contiguous chunks, one work item each, so that a decode batch with few
+//     heads still spreads its cache over all SMs.  Each CTA writes an fp32 partial O (normalised by
 //     its own row sum) and its partial LSE; attn_kvcache_merge_kernel combines
 //     them (O = sum_s exp(LSE_s - LSE) O_s, LSE = log sum_s exp LSE_s).  With
-//     one split the CTA writes the bf16 output directly.
-//   * warp 5 TMA producer (Q once, then K_j / V_j through a ring), warp 4 MMA
+//     one split the item writes the bf16 output directly.
+//   * warp 5 TMA producer (each item's Q into one of two buffers, then its
+//     K_j / V_j through a ring that runs on across items), warp 4 MMA
 //     issuer, warps 0-3 softmax with one query row per thread.  S is double
 //     buffered in TMEM, so S(j+1) runs on the tensor core while the softmax of
 //     tile j runs; P(j) is written back over the upper half of S(j) and read
@@ -59,6 +60,7 @@ struct KvcParams {
   int n_rt;              // 128-row packed tiles per key/value head
   int splits;            // key chunks per (kv head, row tile)
   int qbox;              // rows of the query TMA box: min(128, rows rounded up to 8)
+  int n_items;           // work items = B*H_kv * n_rt * splits
   float scale_log2;      // scale * log2(e)
 };
 
@@ -74,15 +76,56 @@ struct KvcCfg {
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
   static constexpr uint32_t kColPOff = 64;
-  static constexpr int kOffQ = 0;
-  static constexpr int kOffKV = kTileBytes;
+  static constexpr int kOffQ = 0;                        // two query buffers (next item's Q loads early)
+  static constexpr int kOffKV = 2 * kTileBytes;
   static constexpr int kOffBar = kOffKV + kSlots * kTileBytes;
-  // q_full, kv_full[S], kv_empty[S], s_full[2], p_full[2], pv_done, o_full, drain
-  static constexpr int kNumBars = 1 + 2 * kSlots + 2 + 2 + 3;
+  // q_full[2], q_empty[2], kv_full[S], kv_empty[S], s_full[2], p_full[2], pv_done, o_full, o_free, drain
+  static constexpr int kNumBars = 4 + 2 * kSlots + 4 + 4;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
 };
 
+// One work item = (key/value head, 128-row packed query tile, key chunk).
+struct KvcItem {
+  int bkv;       // b * H_kv + key/value head
+  int split;
+  int r0;        // first packed row of the tile
+  int r_valid;   // packed rows that exist in the tile
+  int L;         // valid cache rows of this batch entry
+  int j_lo;      // first key tile of the chunk
+  int nkv;       // key tiles in the chunk (0: nothing to read)
+};
+
+__device__ __forceinline__ KvcItem kvc_item(const KvcParams& prm, int w, bool causal) {
+  KvcItem it;
+  it.split = w % prm.splits;
+  const int rt = (w / prm.splits) % prm.n_rt;
+  it.bkv = w / (prm.splits * prm.n_rt);
+  const int b = it.bkv / prm.h_kv;
+  it.r0 = 128 * rt;
+  it.r_valid = min(128, prm.rows - it.r0);
+  int L = prm.kv_lens ? prm.kv_lens[b] : prm.nk;
+  it.L = min(max(L, 0), prm.nk);
+  // Largest key index any row of the tile may see -> key tiles [0, kv_hi).
+  int lim_max = it.L - 1;
+  if (causal) {
+    const int r1 = it.r0 + it.r_valid - 1;
+    const int p_max = (it.r0 / prm.nq == r1 / prm.nq) ? (r1 % prm.nq) : (prm.nq - 1);
+    lim_max = min(lim_max, p_max + it.L - prm.nq);
+  }
+  const int kv_hi = lim_max < 0 ? 0 : (lim_max >> 7) + 1;
+  const int chunk = (kv_hi + prm.splits - 1) / prm.splits;
+  it.j_lo = min(kv_hi, it.split * chunk);
+  it.nkv = min(kv_hi, it.j_lo + chunk) - it.j_lo;
+  return it;
+}
+
+// Persistent: CTA c takes work items c, c + gridDim.x, ...  Every role walks
+// the same item sequence and skips the same empty items, and the barrier
+// phases run on across items, so the K/V stream never drains between items:
+// the next item's Q and first key tiles load while the current item's last
+// tiles are still being consumed, and its first S products run while the
+// softmax warps write the current item's output.
 template <int D, bool CAUSAL, bool SPLIT>
 __global__ void __launch_bounds__(192, 1)
 attn_kvcache_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -92,64 +135,49 @@ attn_kvcache_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
   uint64_t* q_full = bars;
-  uint64_t* kv_full = q_full + 1;
+  uint64_t* q_empty = q_full + 2;
+  uint64_t* kv_full = q_empty + 2;
   uint64_t* kv_empty = kv_full + C::kSlots;
   uint64_t* s_full = kv_empty + C::kSlots;
   uint64_t* p_full = s_full + 2;
   uint64_t* pv_done = p_full + 2;
   uint64_t* o_full = pv_done + 1;
-  uint64_t* drain = o_full + 1;
+  uint64_t* o_free = o_full + 1;
+  uint64_t* drain = o_free + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int split = blockIdx.x % prm.splits;
-  const int rt = (blockIdx.x / prm.splits) % prm.n_rt;
-  const int bkv = blockIdx.x / (prm.splits * prm.n_rt);      // b * H_kv + kv head
-  const int b = bkv / prm.h_kv;
-  const int r0 = 128 * rt;                                    // first packed row of the tile
-  const int r_valid = min(128, prm.rows - r0);                // packed rows that exist
-  int L = prm.kv_lens ? prm.kv_lens[b] : prm.nk;
-  L = min(max(L, 0), prm.nk);
-  const int shift = L - prm.nq;                               // bottom-right causal offset
-
-  // Largest key index any row of this tile may see -> key tiles [0, kv_hi).
-  int lim_max = L - 1;
-  if (CAUSAL) {
-    const int r1 = r0 + r_valid - 1;
-    const int p_max = (r0 / prm.nq == r1 / prm.nq) ? (r1 % prm.nq) : (prm.nq - 1);
-    lim_max = min(lim_max, p_max + shift);
-  }
-  const int kv_hi = lim_max < 0 ? 0 : (lim_max >> 7) + 1;
-  const int chunk = (kv_hi + prm.splits - 1) / prm.splits;
-  const int j_lo = min(kv_hi, split * chunk);
-  const int nkv = min(kv_hi, j_lo + chunk) - j_lo;             // key tiles this CTA visits
 
   if (threadIdx.x == 0) {
-    mbar_init(q_full, 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&q_full[t], 1);
+      mbar_init(&q_empty[t], 1);
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_full[t], 128);
+    }
     for (int s = 0; s < C::kSlots; ++s) {
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
     }
-    for (int t = 0; t < 2; ++t) {
-      mbar_init(&s_full[t], 1);
-      mbar_init(&p_full[t], 128);
-    }
     mbar_init(pv_done, 1);
     mbar_init(o_full, 1);
+    mbar_init(o_free, 128);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp < 4 && prm.qbox < 128) {
-    // Query rows past the packed rows are never loaded: clear them so the
-    // padding rows of the MMA see zeros rather than stale shared memory.
+    // Query rows past the packed rows are never loaded: clear them (in both
+    // query buffers) so the padding rows of the MMA see zeros.
     const int r = threadIdx.x;
     if (r >= prm.qbox) {
-      for (int blk = 0; blk < C::kNumBlk; ++blk)
-        for (int ch = 0; ch < 8; ++ch)
-          st_shared_v4(smem_u32(smem + C::kOffQ + blk * C::kBlockBytes) + r * 128 + ch * 16, 0u, 0u, 0u, 0u);
+      for (int qb = 0; qb < 2; ++qb)
+        for (int blk = 0; blk < C::kNumBlk; ++blk)
+          for (int ch = 0; ch < 8; ++ch)
+            st_shared_v4(smem_u32(smem + C::kOffQ + qb * C::kTileBytes + blk * C::kBlockBytes) + r * 128 + ch * 16,
+                         0u, 0u, 0u, 0u);
     }
     fence_proxy_async_smem();
   }
@@ -166,241 +194,280 @@ attn_kvcache_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const int n_items = prm.n_items;
 
   if (warp == C::kWarpLoad) {
     // ------------------------------------------------------------------ TMA
-    if (lane == 0 && nkv > 0) {
-      mbar_arrive_expect_tx(q_full, uint32_t(prm.qbox * 128 * C::kNumBlk));
-      for (int blk = 0; blk < C::kNumBlk; ++blk)
-        tma_load_3d(&tm_q, q_full, smem + C::kOffQ + blk * C::kBlockBytes, blk * 64,
-                    bkv * prm.rows + r0, 0);
-      int issued = 0;
-      for (int it = 0; it < 2 * nkv; ++it) {
-        const int slot = it % C::kSlots;
-        const int use = it / C::kSlots;
-        if (use > 0 && !mbar_wait(&kv_empty[slot], (use - 1) & 1, abort_flag)) break;
-        const CUtensorMap* tm = (it & 1) ? &tm_v : &tm_k;
-        mbar_arrive_expect_tx(&kv_full[slot], C::kTileBytes);
+    if (lane == 0) {
+      int qi = 0, it = 0;
+      bool ok = true;
+      for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
+        const KvcItem I = kvc_item(prm, w, CAUSAL);
+        if (I.nkv == 0) continue;
+        const int qb = qi & 1;
+        if (qi >= 2 && !(ok = mbar_wait(&q_empty[qb], uint32_t(((qi >> 1) - 1) & 1), abort_flag))) break;
+        mbar_arrive_expect_tx(&q_full[qb], uint32_t(prm.qbox * 128 * C::kNumBlk));
         for (int blk = 0; blk < C::kNumBlk; ++blk)
-          tma_load_3d(tm, &kv_full[slot], smem + C::kOffKV + slot * C::kTileBytes + blk * C::kBlockBytes,
-                      blk * 64, 128 * (j_lo + (it >> 1)), bkv);
-        ++issued;
+          tma_load_3d(&tm_q, &q_full[qb], smem + C::kOffQ + qb * C::kTileBytes + blk * C::kBlockBytes, blk * 64,
+                      I.bkv * prm.rows + I.r0, 0);
+        ++qi;
+        for (int t = 0; t < 2 * I.nkv; ++t) {
+          const int slot = it % C::kSlots;
+          const int use = it / C::kSlots;
+          if (use > 0 && !(ok = mbar_wait(&kv_empty[slot], uint32_t((use - 1) & 1), abort_flag))) break;
+          mbar_arrive_expect_tx(&kv_full[slot], C::kTileBytes);
+          const CUtensorMap* tm = (t & 1) ? &tm_v : &tm_k;
+          for (int blk = 0; blk < C::kNumBlk; ++blk)
+            tma_load_3d(tm, &kv_full[slot], smem + C::kOffKV + slot * C::kTileBytes + blk * C::kBlockBytes,
+                        blk * 64, 128 * (I.j_lo + (t >> 1)), I.bkv);
+          ++it;
+        }
       }
       // No copy may still be landing in shared memory when the CTA leaves.
-      mbar_wait(q_full, 0, abort_flag, false);
-      for (int it = max(0, issued - C::kSlots); it < issued; ++it)
-        mbar_wait(&kv_full[it % C::kSlots], (it / C::kSlots) & 1, abort_flag, false);
+      for (int q = max(0, qi - 2); q < qi; ++q) mbar_wait(&q_full[q & 1], uint32_t((q >> 1) & 1), abort_flag, false);
+      for (int k = max(0, it - C::kSlots); k < it; ++k)
+        mbar_wait(&kv_full[k % C::kSlots], uint32_t((k / C::kSlots) & 1), abort_flag, false);
     }
     __syncwarp();
   } else if (warp == C::kWarpMma) {
     // ------------------------------------------------------------------ MMA
-    if (lane == 0 && nkv > 0) {
+    if (lane == 0) {
       constexpr uint32_t kIdescS = idesc_bf16(128, 128, false, false);
       constexpr uint32_t kIdescPV = idesc_bf16(128, D, false, true);
-      const uint32_t sQ = smem_u32(smem + C::kOffQ);
       const uint32_t sKV = smem_u32(smem + C::kOffKV);
-      auto slot_of = [](int item) { return item % C::kSlots; };
-      auto parity_of = [](int item) { return uint32_t((item / C::kSlots) & 1); };
-      auto issue_s = [&](int jj) {           // S(jj) = Q K_jj^T into buffer jj % 2
-        const uint32_t b0 = sKV + slot_of(2 * jj) * C::kTileBytes;
-        const uint32_t dt = tmem + ((jj & 1) ? C::kColS1 : C::kColS0);
+      int qi = 0, it = 0, sc = 0, oi = 0;
+      bool ok = true;
+      bool issued_any = false;
+      for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
+        const KvcItem I = kvc_item(prm, w, CAUSAL);
+        if (I.nkv == 0) continue;
+        const int qb = qi & 1;
+        const uint32_t sQ = smem_u32(smem + C::kOffQ + qb * C::kTileBytes);
+        if (!(ok = mbar_wait(&q_full[qb], uint32_t((qi >> 1) & 1), abort_flag))) break;
+        for (int jj = 0; jj <= I.nkv && ok; ++jj) {
+          if (jj < I.nkv) {
+            // S of this tile overwrites the buffer of the P two tiles back,
+            // whose PV was issued before it.
+            const int kit = it + 2 * jj;
+            if (!(ok = mbar_wait(&kv_full[kit % C::kSlots], uint32_t((kit / C::kSlots) & 1), abort_flag))) break;
+            tc_fence_after();
+            const uint32_t b0 = sKV + (kit % C::kSlots) * C::kTileBytes;
+            const uint32_t dt = tmem + (((sc + jj) & 1) ? C::kColS1 : C::kColS0);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * C::kBlockBytes + (kk & 3) * 32;
-          mma_ss(dt, smem_desc_sw128(sQ + off, 16, 1024), smem_desc_sw128(b0 + off, 16, 1024), kIdescS,
-                 kk > 0 ? 1u : 0u);
-        }
-      };
-      auto issue_pv = [&](int jj) {          // O += P(jj) V_jj
-        const uint32_t b0 = sKV + slot_of(2 * jj + 1) * C::kTileBytes;
-        const uint32_t at = tmem + ((jj & 1) ? C::kColS1 : C::kColS0) + C::kColPOff;
+            for (int kk = 0; kk < D / 16; ++kk) {
+              const uint32_t off = (kk >> 2) * C::kBlockBytes + (kk & 3) * 32;
+              mma_ss(dt, smem_desc_sw128(sQ + off, 16, 1024), smem_desc_sw128(b0 + off, 16, 1024), kIdescS,
+                     kk > 0 ? 1u : 0u);
+            }
+            issued_any = true;
+            mma_commit(&s_full[(sc + jj) & 1]);
+            mma_commit(&kv_empty[kit % C::kSlots]);
+            if (jj == I.nkv - 1) mma_commit(&q_empty[qb]);
+          }
+          if (jj > 0) {
+            const int pj = jj - 1;
+            const int ps = sc + pj;
+            if (!(ok = mbar_wait(&p_full[ps & 1], uint32_t((ps >> 1) & 1), abort_flag))) break;
+            // The first PV of an item overwrites O: the previous item's
+            // epilogue must have read it.
+            if (pj == 0 && oi > 0 && !(ok = mbar_wait(o_free, uint32_t((oi - 1) & 1), abort_flag))) break;
+            const int vit = it + 2 * pj + 1;
+            if (!(ok = mbar_wait(&kv_full[vit % C::kSlots], uint32_t((vit / C::kSlots) & 1), abort_flag))) break;
+            tc_fence_after();
+            const uint32_t b0 = sKV + (vit % C::kSlots) * C::kTileBytes;
+            const uint32_t at = tmem + ((ps & 1) ? C::kColS1 : C::kColS0) + C::kColPOff;
 #pragma unroll
-        for (int kk = 0; kk < 128 / 16; ++kk)
-          mma_ts(tmem + C::kColO, at + kk * 8, smem_desc_sw128(b0 + kk * 2048, C::kBlockBytes, 1024), kIdescPV,
-                 (jj > 0 || kk > 0) ? 1u : 0u);
-      };
-
-      bool ok = mbar_wait(q_full, 0, abort_flag);
-      for (int jj = 0; jj <= nkv && ok; ++jj) {
-        if (jj < nkv) {
-          // S(jj) overwrites the buffer of P(jj-2), whose PV was issued before.
-          if (!(ok = mbar_wait(&kv_full[slot_of(2 * jj)], parity_of(2 * jj), abort_flag))) break;
-          tc_fence_after();
-          issue_s(jj);
-          mma_commit(&s_full[jj & 1]);
-          mma_commit(&kv_empty[slot_of(2 * jj)]);
+            for (int kk = 0; kk < 128 / 16; ++kk)
+              mma_ts(tmem + C::kColO, at + kk * 8, smem_desc_sw128(b0 + kk * 2048, C::kBlockBytes, 1024), kIdescPV,
+                     (pj > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(&kv_empty[vit % C::kSlots]);
+            mma_commit(pj == I.nkv - 1 ? o_full : pv_done);
+          }
         }
-        if (jj > 0) {
-          const int pj = jj - 1;
-          if (!(ok = mbar_wait(&p_full[pj & 1], uint32_t((pj >> 1) & 1), abort_flag))) break;
-          if (!(ok = mbar_wait(&kv_full[slot_of(2 * pj + 1)], parity_of(2 * pj + 1), abort_flag))) break;
-          tc_fence_after();
-          issue_pv(pj);
-          mma_commit(&kv_empty[slot_of(2 * pj + 1)]);
-          mma_commit(pj == nkv - 1 ? o_full : pv_done);
-        }
+        it += 2 * I.nkv;
+        sc += I.nkv;
+        ++qi;
+        ++oi;
       }
       // Every MMA issued so far must finish before tensor memory is released.
-      mma_commit(drain);
-      mbar_wait(drain, 0, abort_flag, false);
+      if (issued_any) {
+        mma_commit(drain);
+        mbar_wait(drain, 0, abort_flag, false);
+      }
     }
     __syncwarp();
   } else {
     // -------------------------------------------------------------- softmax
     const int r = warp * 32 + lane;           // row inside the tile = TMEM lane
-    const int rp = r0 + r;                    // packed row
-    const bool row_ok = r < r_valid;
-    const bool warp_on = warp * 32 < r_valid;
-    const int p = rp % prm.nq;
-    int lim = L - 1;                          // last key this row sees
-    if (CAUSAL) lim = min(lim, p + shift);
     const uint32_t lane_base = uint32_t(warp * 32) << 16;
     const uint32_t tO = tmem + lane_base + C::kColO;
     const float c = prm.scale_log2;
-    float m_ref = -INFINITY;
-    float l = 0.f;
+    int it = 0, sc = 0, pvb = 0, oi = 0;
     bool ok = true;
 
-    for (int jj = 0; jj < nkv; ++jj) {
-      const int j = j_lo + jj;
-      const uint32_t tS = tmem + lane_base + ((jj & 1) ? C::kColS1 : C::kColS0);
-      if (!(ok = mbar_wait_warp(&s_full[jj & 1], uint32_t((jj >> 1) & 1), abort_flag))) break;
-      tc_fence_after();
-      // Cache rows past L inside this key tile: clear their V rows (all 128
-      // threads, one key row each) so that P = 0 meets V = 0 there.
-      if (128 * j + 128 > L && L < prm.nk) {
-        const int item = 2 * jj + 1;
-        if (!(ok = mbar_wait_warp(&kv_full[item % C::kSlots], uint32_t((item / C::kSlots) & 1), abort_flag))) break;
-        if (128 * j + r >= L) {
-          uint8_t* vt = smem + C::kOffKV + (item % C::kSlots) * C::kTileBytes;
-          for (int blk = 0; blk < C::kNumBlk; ++blk)
-            for (int ch = 0; ch < 8; ++ch)
-              st_shared_v4(smem_u32(vt + blk * C::kBlockBytes) + r * 128 + ch * 16, 0u, 0u, 0u, 0u);
-        }
-        fence_proxy_async_smem();
-      }
-      if (warp_on) {
-        float s[128];
-        {
-          uint32_t a[32], bb[32], e[32], f[32];
-          tmem_ld32(tS + 0, a);
-          tmem_ld32(tS + 32, bb);
-          tmem_ld32(tS + 64, e);
-          tmem_ld32(tS + 96, f);
-          tmem_ld_wait(a);
-          reg_fence32(bb);
-          reg_fence32(e);
-          reg_fence32(f);
-#pragma unroll
-          for (int k = 0; k < 32; ++k) {
-            s[k] = __uint_as_float(a[k]);
-            s[32 + k] = __uint_as_float(bb[k]);
-            s[64 + k] = __uint_as_float(e[k]);
-            s[96 + k] = __uint_as_float(f[k]);
-          }
-        }
-        const int limit = row_ok ? lim - 128 * j : -1;     // padding rows: everything masked
-        if (__any_sync(0xffffffffu, limit < 127)) {
-#pragma unroll
-          for (int k = 0; k < 128; ++k)
-            if (k > limit) s[k] = -INFINITY;
-        }
-        float mxp[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) mxp[u] = s[u];
-#pragma unroll
-        for (int k = 8; k < 128; k += 8)
-#pragma unroll
-          for (int u = 0; u < 8; ++u) mxp[u] = fmaxf(mxp[u], s[k + u]);
-        const float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
-                               fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
-        const float m_tile = mx * c;
-        float alpha = 1.f;
-        bool rescale = false;
-        if (m_tile > m_ref + kKvcRescaleLog2) {
-          alpha = ex2(m_ref - m_tile);
-          m_ref = m_tile;
-          rescale = (jj > 0);
-        }
-        l *= alpha;
-        const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
-        float sump[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            const float p0 = ex2(fmaf(s[32 * q + 2 * k], c, neg_m));
-            const float p1 = ex2(fmaf(s[32 * q + 2 * k + 1], c, neg_m));
-            sump[k & 3] += p0 + p1;
-            pk[k] = pack_bf16x2(p0, p1);
-          }
-          tmem_st16(tS + C::kColPOff + 16 * q, pk);
-        }
-        l += (sump[0] + sump[1]) + (sump[2] + sump[3]);
-        if (__any_sync(0xffffffffu, rescale)) {
-          // O holds the sum through tile jj-2 for sure; wait for PV(jj-1).
-          if (!(ok = mbar_wait_warp(pv_done, uint32_t((jj - 1) & 1), abort_flag))) break;
-          tc_fence_after();
-          const float a = rescale ? alpha : 1.f;
-#pragma unroll 1
-          for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t o[32];
-            tmem_ld32(tO + cc * 32, o);
-            tmem_ld_wait(o);
-#pragma unroll
-            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * a);
-            tmem_st32(tO + cc * 32, o);
-          }
-        }
-        tmem_st_wait();
-      }
-      tc_fence_before();
-      mbar_arrive(&p_full[jj & 1]);
-    }
+    for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
+      const KvcItem I = kvc_item(prm, w, CAUSAL);
+      const int rp = I.r0 + r;                // packed row
+      const bool row_ok = r < I.r_valid;
+      const bool warp_on = warp * 32 < I.r_valid;
+      int lim = I.L - 1;                      // last key this row sees
+      if (CAUSAL) lim = min(lim, rp % prm.nq + I.L - prm.nq);
+      float m_ref = -INFINITY;
+      float l = 0.f;
 
-    // ------------------------------------------------------------ epilogue
-    if (ok && nkv > 0 && warp_on) ok = mbar_wait_warp(o_full, 0, abort_flag);
-    if (ok && warp_on) {
+      for (int jj = 0; jj < I.nkv; ++jj) {
+        const int j = I.j_lo + jj;
+        const int sb = (sc + jj) & 1;
+        const uint32_t tS = tmem + lane_base + (sb ? C::kColS1 : C::kColS0);
+        if (!(ok = mbar_wait_warp(&s_full[sb], uint32_t(((sc + jj) >> 1) & 1), abort_flag))) break;
+        tc_fence_after();
+        // Cache rows past L inside this key tile: clear their V rows (all 128
+        // threads, one key row each) so that P = 0 meets V = 0 there.
+        if (128 * j + 128 > I.L && I.L < prm.nk) {
+          const int vit = it + 2 * jj + 1;
+          if (!(ok = mbar_wait_warp(&kv_full[vit % C::kSlots], uint32_t((vit / C::kSlots) & 1), abort_flag))) break;
+          if (128 * j + r >= I.L) {
+            uint8_t* vt = smem + C::kOffKV + (vit % C::kSlots) * C::kTileBytes;
+            for (int blk = 0; blk < C::kNumBlk; ++blk)
+              for (int ch = 0; ch < 8; ++ch)
+                st_shared_v4(smem_u32(vt + blk * C::kBlockBytes) + r * 128 + ch * 16, 0u, 0u, 0u, 0u);
+          }
+          fence_proxy_async_smem();
+        }
+        if (warp_on) {
+          float s[128];
+          {
+            uint32_t a[32], bb[32], e[32], f[32];
+            tmem_ld32(tS + 0, a);
+            tmem_ld32(tS + 32, bb);
+            tmem_ld32(tS + 64, e);
+            tmem_ld32(tS + 96, f);
+            tmem_ld_wait(a);
+            reg_fence32(bb);
+            reg_fence32(e);
+            reg_fence32(f);
+#pragma unroll
+            for (int k = 0; k < 32; ++k) {
+              s[k] = __uint_as_float(a[k]);
+              s[32 + k] = __uint_as_float(bb[k]);
+              s[64 + k] = __uint_as_float(e[k]);
+              s[96 + k] = __uint_as_float(f[k]);
+            }
+          }
+          const int limit = row_ok ? lim - 128 * j : -1;     // padding rows: everything masked
+          if (__any_sync(0xffffffffu, limit < 127)) {
+#pragma unroll
+            for (int k = 0; k < 128; ++k)
+              if (k > limit) s[k] = -INFINITY;
+          }
+          float mxp[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) mxp[u] = s[u];
+#pragma unroll
+          for (int k = 8; k < 128; k += 8)
+#pragma unroll
+            for (int u = 0; u < 8; ++u) mxp[u] = fmaxf(mxp[u], s[k + u]);
+          const float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
+                                 fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
+          const float m_tile = mx * c;
+          float alpha = 1.f;
+          bool rescale = false;
+          if (m_tile > m_ref + kKvcRescaleLog2) {
+            alpha = ex2(m_ref - m_tile);
+            m_ref = m_tile;
+            rescale = (jj > 0);
+          }
+          l *= alpha;
+          const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
+          float sump[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+              const float p0 = ex2(fmaf(s[32 * q + 2 * k], c, neg_m));
+              const float p1 = ex2(fmaf(s[32 * q + 2 * k + 1], c, neg_m));
+              sump[k & 3] += p0 + p1;
+              pk[k] = pack_bf16x2(p0, p1);
+            }
+            tmem_st16(tS + C::kColPOff + 16 * q, pk);
+          }
+          l += (sump[0] + sump[1]) + (sump[2] + sump[3]);
+          if (__any_sync(0xffffffffu, rescale)) {
+            // O holds this item's sum through tile jj-2 for sure; wait for PV(jj-1).
+            if (!(ok = mbar_wait_warp(pv_done, uint32_t((pvb + jj - 1) & 1), abort_flag))) break;
+            tc_fence_after();
+            const float a = rescale ? alpha : 1.f;
+#pragma unroll 1
+            for (int cc = 0; cc < D / 32; ++cc) {
+              uint32_t o[32];
+              tmem_ld32(tO + cc * 32, o);
+              tmem_ld_wait(o);
+#pragma unroll
+              for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * a);
+              tmem_st32(tO + cc * 32, o);
+            }
+          }
+          tmem_st_wait();
+        }
+        tc_fence_before();
+        mbar_arrive(&p_full[sb]);
+      }
+      if (!ok) break;
+
+      // ---------------------------------------------------------- epilogue
+      if (I.nkv > 0 && warp_on && !(ok = mbar_wait_warp(o_full, uint32_t(oi & 1), abort_flag))) break;
       tc_fence_after();
       const bool has = l > 0.f;                // false: the row saw no key in this chunk
       const float inv_l = has ? 1.f / l : 0.f;
-      const long long row = (long long)bkv * prm.rows + rp;   // flat B*H*Nq row
+      const long long row = (long long)I.bkv * prm.rows + rp;   // flat B*H*Nq row
+      if (warp_on) {
 #pragma unroll 1
-      for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t o[32];
-        if (nkv > 0) {
-          tmem_ld32(tO + cc * 32, o);
-          tmem_ld_wait(o);
-        } else {
-#pragma unroll
-          for (int k = 0; k < 32; ++k) o[k] = 0u;
-        }
-        if (row_ok) {
-          if (SPLIT) {
-            float4* dst = reinterpret_cast<float4*>(prm.part_o + ((long long)split * prm.total_rows + row) * D + cc * 32);
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-              dst[k] = make_float4(__uint_as_float(o[4 * k]) * inv_l, __uint_as_float(o[4 * k + 1]) * inv_l,
-                                   __uint_as_float(o[4 * k + 2]) * inv_l, __uint_as_float(o[4 * k + 3]) * inv_l);
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          if (I.nkv > 0) {
+            tmem_ld32(tO + cc * 32, o);
+            tmem_ld_wait(o);
           } else {
-            uint4* dst = reinterpret_cast<uint4*>(prm.o + row * D + cc * 32);
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-              dst[k] = make_uint4(
-                  pack_bf16x2(__uint_as_float(o[8 * k + 0]) * inv_l, __uint_as_float(o[8 * k + 1]) * inv_l),
-                  pack_bf16x2(__uint_as_float(o[8 * k + 2]) * inv_l, __uint_as_float(o[8 * k + 3]) * inv_l),
-                  pack_bf16x2(__uint_as_float(o[8 * k + 4]) * inv_l, __uint_as_float(o[8 * k + 5]) * inv_l),
-                  pack_bf16x2(__uint_as_float(o[8 * k + 6]) * inv_l, __uint_as_float(o[8 * k + 7]) * inv_l));
+            for (int k = 0; k < 32; ++k) o[k] = 0u;
+          }
+          if (row_ok) {
+            if (SPLIT) {
+              float4* dst =
+                  reinterpret_cast<float4*>(prm.part_o + ((long long)I.split * prm.total_rows + row) * D + cc * 32);
+#pragma unroll
+              for (int k = 0; k < 8; ++k)
+                dst[k] = make_float4(__uint_as_float(o[4 * k]) * inv_l, __uint_as_float(o[4 * k + 1]) * inv_l,
+                                     __uint_as_float(o[4 * k + 2]) * inv_l, __uint_as_float(o[4 * k + 3]) * inv_l);
+            } else {
+              uint4* dst = reinterpret_cast<uint4*>(prm.o + row * D + cc * 32);
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                dst[k] = make_uint4(
+                    pack_bf16x2(__uint_as_float(o[8 * k + 0]) * inv_l, __uint_as_float(o[8 * k + 1]) * inv_l),
+                    pack_bf16x2(__uint_as_float(o[8 * k + 2]) * inv_l, __uint_as_float(o[8 * k + 3]) * inv_l),
+                    pack_bf16x2(__uint_as_float(o[8 * k + 4]) * inv_l, __uint_as_float(o[8 * k + 5]) * inv_l),
+                    pack_bf16x2(__uint_as_float(o[8 * k + 6]) * inv_l, __uint_as_float(o[8 * k + 7]) * inv_l));
+            }
           }
         }
+        if (row_ok) {
+          const float lse = has ? (m_ref + __log2f(l)) * kKvcLn2 : -INFINITY;
+          if (SPLIT)
+            prm.part_lse[(long long)I.split * prm.total_rows + row] = lse;
+          else
+            prm.lse[row] = lse;
+        }
       }
-      if (row_ok) {
-        const float lse = has ? (m_ref + __log2f(l)) * kKvcLn2 : -INFINITY;
-        if (SPLIT)
-          prm.part_lse[(long long)split * prm.total_rows + row] = lse;
-        else
-          prm.lse[row] = lse;
+      if (I.nkv > 0) {
+        // O has been read: the next item's first PV may overwrite it.
+        tc_fence_before();
+        mbar_arrive(o_free);
+        it += 2 * I.nkv;
+        sc += I.nkv;
+        pvb += I.nkv - 1;
+        ++oi;
       }
     }
   }

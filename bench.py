@@ -364,6 +364,18 @@ def run_ours(args, rank, world, local_rank):
                              "traffic": recorded_traffic("kvcache") if lens is None else None,
                              "kv_lens": None if lens is None else "uniform in [N/2, N] per batch entry"}
             del wsd
+        if not args.no_cpu_baseline and rank == 0:
+            # the oracle (as it stands) on batch entry 0 of the full-cache decode
+            import numpy as np
+            from oracle import attn_oracle as orc
+            h64 = lambda t: t.float().cpu().numpy().astype(np.float64).reshape(-1, t.shape[2], t.shape[3])
+            Qh, Kh, Vh = h64(qd[0:1]), h64(kc[0:1]), h64(vc[0:1])
+            t = time.perf_counter()
+            orc.attn_fwd_kvcache(Qh, Kh, Vh, scale, causal, 1, w.H, hk)
+            dt = time.perf_counter() - t
+            b1 = hk * w.N * w.d * 2 * 2
+            kvcache["cpu_oracle"] = {"value": round(b1 / dt / 1e9, 3), "unit": "GB/s", "seconds": round(dt, 3),
+                                     "kind": "oracle", "sample": "batch entry 0 of the full-cache decode, fp64 numpy"}
         del kc, vc
 
     # ---------------------------------------------------- FP8 (E4M3) forward
@@ -399,6 +411,18 @@ def run_ours(args, rank, world, local_rank):
                "fwd_tflops": round(fp8_tf, 2), "peak": round(2 * burst, 1),
                "peak_kind": f"2 x bf16_tflops ({peaks_src}), nominal E4M3:BF16 ratio",
                "frac": round(fp8_tf / (2 * burst), 4), "steps": n_f}
+        if not args.no_cpu_baseline and rank == 0:
+            # the oracle on the causal prefix of head (0, 0): first 4096 rows and keys
+            import numpy as np
+            from oracle import attn_oracle as orc
+            rows = 4096
+            c8 = lambda t: t[0, 0, :rows].view(torch.uint8).cpu().numpy()[None]
+            t = time.perf_counter()
+            orc.attn_fwd_fp8(c8(qf), c8(kf), c8(vf), dq8, dk8, dv8, scale, causal, 1, 1, 1)
+            dt = time.perf_counter() - t
+            fp8["cpu_oracle"] = {"value": round(4.0 * rows * rows * w.d / 2 / dt / 1e12, 6), "unit": "TFLOP/s",
+                                 "seconds": round(dt, 3), "kind": "oracle",
+                                 "sample": f"causal prefix of head (0,0): first {rows} rows, forward, fp64 numpy"}
         del qf, kf, vf
 
     # ---------------------------------------------------------------- e2e

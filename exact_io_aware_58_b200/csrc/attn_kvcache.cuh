@@ -70,14 +70,15 @@ struct KvcCfg {
   static constexpr int kBlockBytes = 128 * 128;          // [128][64] bf16 column block
   static constexpr int kNumBlk = D / 64;
   static constexpr int kSlots = (D == 128) ? 4 : 8;      // K/V ring: two key tiles ahead
+  static constexpr int kQBufs = 2;                       // query buffers (next item's Q loads early)
   static constexpr int kThreads = 192;
   static constexpr int kWarpMma = 4;
   static constexpr int kWarpLoad = 5;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
   static constexpr uint32_t kColPOff = 64;
-  static constexpr int kOffQ = 0;                        // two query buffers (next item's Q loads early)
-  static constexpr int kOffKV = 2 * kTileBytes;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffKV = kQBufs * kTileBytes;
   static constexpr int kOffBar = kOffKV + kSlots * kTileBytes;
   // q_full[2], q_empty[2], kv_full[S], kv_empty[S], s_full[2], p_full[2], pv_done, o_full, o_free, drain
   static constexpr int kNumBars = 4 + 2 * kSlots + 4 + 4;
@@ -173,7 +174,7 @@ attn_kvcache_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     // query buffers) so the padding rows of the MMA see zeros.
     const int r = threadIdx.x;
     if (r >= prm.qbox) {
-      for (int qb = 0; qb < 2; ++qb)
+      for (int qb = 0; qb < C::kQBufs; ++qb)
         for (int blk = 0; blk < C::kNumBlk; ++blk)
           for (int ch = 0; ch < 8; ++ch)
             st_shared_v4(smem_u32(smem + C::kOffQ + qb * C::kTileBytes + blk * C::kBlockBytes) + r * 128 + ch * 16,
@@ -204,8 +205,8 @@ attn_kvcache_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
         const KvcItem I = kvc_item(prm, w, CAUSAL);
         if (I.nkv == 0) continue;
-        const int qb = qi & 1;
-        if (qi >= 2 && !(ok = mbar_wait(&q_empty[qb], uint32_t(((qi >> 1) - 1) & 1), abort_flag))) break;
+        const int qb = qi % C::kQBufs;
+        if (qi >= C::kQBufs && !(ok = mbar_wait(&q_empty[qb], uint32_t((qi / C::kQBufs - 1) & 1), abort_flag))) break;
         mbar_arrive_expect_tx(&q_full[qb], uint32_t(prm.qbox * 128 * C::kNumBlk));
         for (int blk = 0; blk < C::kNumBlk; ++blk)
           tma_load_3d(&tm_q, &q_full[qb], smem + C::kOffQ + qb * C::kTileBytes + blk * C::kBlockBytes, blk * 64,
@@ -224,7 +225,8 @@ attn_kvcache_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         }
       }
       // No copy may still be landing in shared memory when the CTA leaves.
-      for (int q = max(0, qi - 2); q < qi; ++q) mbar_wait(&q_full[q & 1], uint32_t((q >> 1) & 1), abort_flag, false);
+      for (int q = max(0, qi - C::kQBufs); q < qi; ++q)
+        mbar_wait(&q_full[q % C::kQBufs], uint32_t((q / C::kQBufs) & 1), abort_flag, false);
       for (int k = max(0, it - C::kSlots); k < it; ++k)
         mbar_wait(&kv_full[k % C::kSlots], uint32_t((k / C::kSlots) & 1), abort_flag, false);
     }
@@ -241,9 +243,9 @@ attn_kvcache_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
         const KvcItem I = kvc_item(prm, w, CAUSAL);
         if (I.nkv == 0) continue;
-        const int qb = qi & 1;
+        const int qb = qi % C::kQBufs;
         const uint32_t sQ = smem_u32(smem + C::kOffQ + qb * C::kTileBytes);
-        if (!(ok = mbar_wait(&q_full[qb], uint32_t((qi >> 1) & 1), abort_flag))) break;
+        if (!(ok = mbar_wait(&q_full[qb], uint32_t((qi / C::kQBufs) & 1), abort_flag))) break;
         for (int jj = 0; jj <= I.nkv && ok; ++jj) {
           if (jj < I.nkv) {
             // S of this tile overwrites the buffer of the P two tiles back,

@@ -55,6 +55,7 @@ KERNEL_SOURCES = {
     "bwd_dkdv": ("attn_bwd.cuh", "sm100.cuh"),
     "bwd_dq": ("attn_bwd.cuh", "sm100.cuh"),
     "kvcache": ("attn_kvcache.cuh", "sm100.cuh"),
+    "fp8": ("attn_fwd_fp8.cuh", "sm100.cuh"),
 }
 
 
@@ -410,7 +411,7 @@ def run_ours(args, rank, world, local_rank):
         fp8 = {"workload": "long_batch forward on E4M3 Q, K, V (per-tensor scales)", "ms_fwd": round(tf, 3),
                "fwd_tflops": round(fp8_tf, 2), "peak": round(2 * burst, 1),
                "peak_kind": f"2 x bf16_tflops ({peaks_src}), nominal E4M3:BF16 ratio",
-               "frac": round(fp8_tf / (2 * burst), 4), "steps": n_f}
+               "frac": round(fp8_tf / (2 * burst), 4), "steps": n_f, "traffic": recorded_traffic("fp8")}
         if not args.no_cpu_baseline and rank == 0:
             # the oracle on the causal prefix of head (0, 0): first 4096 rows and keys
             import numpy as np

@@ -69,8 +69,8 @@ struct KvcCfg {
   static constexpr int kTileBytes = 128 * D * 2;
   static constexpr int kBlockBytes = 128 * 128;          // [128][64] bf16 column block
   static constexpr int kNumBlk = D / 64;
-  static constexpr int kSlots = (D == 128) ? 4 : 8;      // K/V ring: two key tiles ahead
-  static constexpr int kQBufs = 2;                       // query buffers (next item's Q loads early)
+  static constexpr int kSlots = (D == 128) ? 6 : 12;     // K/V ring: three key tiles ahead
+  static constexpr int kQBufs = 1;                       // query buffers
   static constexpr int kThreads = 192;
   static constexpr int kWarpMma = 4;
   static constexpr int kWarpLoad = 5;

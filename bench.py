@@ -348,16 +348,18 @@ def run_ours(args, rank, world, local_rank):
 
             for _ in range(max(3, args.warmup)):
                 dec()
-            n_d = 20
-            dev_ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n_d)]
+            # One event pair around back-to-back calls: a call is ~0.1 ms of GPU
+            # work, so per-call event pairs would also time the host's launch gap.
+            n_d = 50
+            ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             torch.cuda.synchronize()
-            for e in dev_ev:
-                e[0].record(stream)
+            ev0.record(stream)
+            for _ in range(n_d):
                 dec()
-                e[1].record(stream)
+            ev1.record(stream)
             torch.cuda.synchronize()
             assert attn.attn_check_status(stream) == attn.ATTN_OK
-            t_us = sum(e[0].elapsed_time(e[1]) for e in dev_ev) / n_d * 1e3
+            t_us = ev0.elapsed_time(ev1) / n_d * 1e3
             t_us = max_over_ranks([t_us], device=dev)[0]
             gbs = alg_bytes / (t_us * 1e-6) / 1e9
             kvcache[name] = {"splits": splits, "us": round(t_us, 2), "alg_bytes": alg_bytes,

@@ -517,15 +517,23 @@ int64_t kvc_splits(const KvcShape& sh, int64_t B, int64_t H_kv, int64_t num_spli
   return best_s;
 }
 
+// With at most 32 packed query rows per key/value head the kernel replicates
+// them into all four TMEM lane quarters and splits every key tile four ways,
+// so each key chunk yields four partials.
+bool kvc_replicated(const KvcShape& sh) { return sh.rows <= 32; }
+
+int64_t kvc_partials(const KvcShape& sh, int64_t splits) { return splits * (kvc_replicated(sh) ? 4 : 1); }
+
 size_t kvc_workspace(const KvcShape& sh, int64_t splits, int64_t d) {
-  if (splits <= 1) return 0;
-  return size_t(splits) * size_t(sh.total_rows) * size_t(d + 1) * sizeof(float);
+  const int64_t parts = kvc_partials(sh, splits);
+  if (parts <= 1) return 0;
+  return size_t(parts) * size_t(sh.total_rows) * size_t(d + 1) * sizeof(float);
 }
 
-template <int D, bool CAUSAL, bool SPLIT>
+template <int D, bool CAUSAL, bool SPLIT, bool REPL>
 int launch_kvc(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const attn::KvcParams& prm,
                int grid, cudaStream_t st) {
-  auto kern = attn::attn_kvcache_kernel<D, CAUSAL, SPLIT>;
+  auto kern = attn::attn_kvcache_kernel<D, CAUSAL, SPLIT, REPL>;
   constexpr int smem = attn::KvcCfg<D>::kSmemBytes;
   if (set_smem(reinterpret_cast<const void*>(kern), smem) != ATTN_OK) return ATTN_ERR_LAUNCH;
   kern<<<grid, attn::KvcCfg<D>::kThreads, smem, st>>>(q, k, v, prm);
@@ -534,15 +542,17 @@ int launch_kvc(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
   int64_t blocks = (prm.total_rows + 7) / 8;                  // 8 rows (warps) per 256-thread block
   if (blocks > kNumSMs * 16) blocks = kNumSMs * 16;
   attn::attn_kvcache_merge_kernel<D><<<int(blocks), 256, 0, st>>>(prm.part_o, prm.part_lse, prm.o, prm.lse,
-                                                                   prm.total_rows, prm.splits);
+                                                                   prm.total_rows, prm.splits * (REPL ? 4 : 1));
   return launch_status();
 }
 
-#define ATTN_KVC_DISPATCH(...)                                                                         \
-  (d == 128 ? (causal ? (split ? launch_kvc<128, true, true>(__VA_ARGS__) : launch_kvc<128, true, false>(__VA_ARGS__)) \
-                      : (split ? launch_kvc<128, false, true>(__VA_ARGS__) : launch_kvc<128, false, false>(__VA_ARGS__))) \
-            : (causal ? (split ? launch_kvc<64, true, true>(__VA_ARGS__) : launch_kvc<64, true, false>(__VA_ARGS__)) \
-                      : (split ? launch_kvc<64, false, true>(__VA_ARGS__) : launch_kvc<64, false, false>(__VA_ARGS__))))
+template <int D, bool CAUSAL>
+int dispatch_kvc(bool split, bool repl, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                 const attn::KvcParams& prm, int grid, cudaStream_t st) {
+  if (repl) return launch_kvc<D, CAUSAL, true, true>(q, k, v, prm, grid, st);
+  return split ? launch_kvc<D, CAUSAL, true, false>(q, k, v, prm, grid, st)
+               : launch_kvc<D, CAUSAL, false, false>(q, k, v, prm, grid, st);
+}
 
 }  // namespace
 
@@ -576,7 +586,9 @@ ATTN_EXPORT int attn_fwd_kvcache(const void* Q, const void* K, const void* V, vo
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE))
     return ATTN_ERR_MISALIGNED;
   if (kv_lens && (reinterpret_cast<uintptr_t>(kv_lens) & 3u) != 0) return ATTN_ERR_MISALIGNED;
-  const bool split = splits > 1;
+  const bool repl = kvc_replicated(sh);
+  const int64_t parts = kvc_partials(sh, splits);
+  const bool split = parts > 1;
   if (split) {
     if (!workspace) return ATTN_ERR_INVALID_ARG;
     if (!aligned16(workspace)) return ATTN_ERR_MISALIGNED;
@@ -594,7 +606,7 @@ ATTN_EXPORT int attn_fwd_kvcache(const void* Q, const void* K, const void* V, vo
   prm.o = static_cast<__nv_bfloat16*>(O);
   prm.lse = LSE;
   prm.part_o = split ? static_cast<float*>(workspace) : nullptr;
-  prm.part_lse = split ? static_cast<float*>(workspace) + size_t(splits) * size_t(sh.total_rows) * size_t(d) : nullptr;
+  prm.part_lse = split ? static_cast<float*>(workspace) + size_t(parts) * size_t(sh.total_rows) * size_t(d) : nullptr;
   prm.kv_lens = kv_lens;
   prm.total_rows = sh.total_rows;
   prm.nq = int(Nq);
@@ -607,7 +619,11 @@ ATTN_EXPORT int attn_fwd_kvcache(const void* Q, const void* K, const void* V, vo
   prm.n_items = int(n_items);
   prm.scale_log2 = scale * 1.4426950408889634f;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  return ATTN_KVC_DISPATCH(mq, mk, mv, prm, int(grid), st);
+  if (d == 128)
+    return causal ? dispatch_kvc<128, true>(split, repl, mq, mk, mv, prm, int(grid), st)
+                  : dispatch_kvc<128, false>(split, repl, mq, mk, mv, prm, int(grid), st);
+  return causal ? dispatch_kvc<64, true>(split, repl, mq, mk, mv, prm, int(grid), st)
+                : dispatch_kvc<64, false>(split, repl, mq, mk, mv, prm, int(grid), st);
 }
 
 }  // extern "C"

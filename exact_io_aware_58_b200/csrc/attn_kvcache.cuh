@@ -29,6 +29,16 @@
 //     tile j runs; P(j) is written back over the upper half of S(j) and read
 //     from TMEM by the PV MMA.  Warps whose 32 rows are all padding only keep
 //     the barrier protocol.
+//   * Few packed rows (at most 32, e.g. decode with up to 32 query heads per
+//     key/value head): the rows are loaded into all four TMEM lane quarters
+//     (four copies of the query box), so every lane quarter computes the same
+//     scores, and warp w keeps an online softmax over key columns
+//     [32w, 32w + 32) of each tile only.  Its P goes to its own 16 packed
+//     columns of a dedicated P buffer whose other columns stay zero, so the
+//     PV product of lane quarter w sums over its key subset alone: four
+//     independent partials per item, merged with the split-KV partials.  The
+//     per-warp softmax work per key tile drops fourfold, which is what keeps
+//     the cache stream, not the softmax, the limit.
 //   * Causal masking is bottom-right aligned: the new rows are the last Nq
 //     positions of a sequence of L = kv_lens[b] tokens, so position p sees key
 //     j iff j <= p + L - Nq.  Rows that see no key get O = 0 and LSE = -inf.
@@ -77,6 +87,7 @@ struct KvcCfg {
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
   static constexpr uint32_t kColPOff = 64;
+  static constexpr uint32_t kColP0 = 384, kColP1 = 448;   // replicated mode: P buffers of their own
   static constexpr int kOffQ = 0;
   static constexpr int kOffKV = kQBufs * kTileBytes;
   static constexpr int kOffBar = kOffKV + kSlots * kTileBytes;
@@ -127,11 +138,12 @@ __device__ __forceinline__ KvcItem kvc_item(const KvcParams& prm, int w, bool ca
 // the next item's Q and first key tiles load while the current item's last
 // tiles are still being consumed, and its first S products run while the
 // softmax warps write the current item's output.
-template <int D, bool CAUSAL, bool SPLIT>
+template <int D, bool CAUSAL, bool SPLIT, bool REPL>
 __global__ void __launch_bounds__(192, 1)
 attn_kvcache_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const KvcParams prm) {
   using C = KvcCfg<D>;
+  static_assert(!REPL || SPLIT, "the replicated mode always writes partials");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
@@ -169,11 +181,11 @@ attn_kvcache_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp < 4 && prm.qbox < 128) {
-    // Query rows past the packed rows are never loaded: clear them (in both
-    // query buffers) so the padding rows of the MMA see zeros.
+  if (warp < 4 && prm.qbox < (REPL ? 32 : 128)) {
+    // Query rows past the packed rows are never loaded: clear them (in every
+    // query buffer) so the padding rows of the MMA see zeros.
     const int r = threadIdx.x;
-    if (r >= prm.qbox) {
+    if ((REPL ? (r & 31) : r) >= prm.qbox) {
       for (int qb = 0; qb < C::kQBufs; ++qb)
         for (int blk = 0; blk < C::kNumBlk; ++blk)
           for (int ch = 0; ch < 8; ++ch)
@@ -196,6 +208,19 @@ attn_kvcache_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int n_items = prm.n_items;
+  if (REPL && warp < 4) {
+    // Replicated mode: each lane quarter writes P only in its own 16 packed
+    // columns of a P buffer; the other columns of its lanes stay zero.
+    uint32_t z[32];
+#pragma unroll
+    for (int k = 0; k < 32; ++k) z[k] = 0u;
+    const uint32_t lb = uint32_t(warp * 32) << 16;
+    tmem_st32(tmem + lb + C::kColP0, z);
+    tmem_st32(tmem + lb + C::kColP0 + 32, z);
+    tmem_st32(tmem + lb + C::kColP1, z);
+    tmem_st32(tmem + lb + C::kColP1 + 32, z);
+    tmem_st_wait();
+  }
 
   if (warp == C::kWarpLoad) {
     // ------------------------------------------------------------------ TMA
@@ -207,10 +232,13 @@ attn_kvcache_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         if (I.nkv == 0) continue;
         const int qb = qi % C::kQBufs;
         if (qi >= C::kQBufs && !(ok = mbar_wait(&q_empty[qb], uint32_t((qi / C::kQBufs - 1) & 1), abort_flag))) break;
-        mbar_arrive_expect_tx(&q_full[qb], uint32_t(prm.qbox * 128 * C::kNumBlk));
-        for (int blk = 0; blk < C::kNumBlk; ++blk)
-          tma_load_3d(&tm_q, &q_full[qb], smem + C::kOffQ + qb * C::kTileBytes + blk * C::kBlockBytes, blk * 64,
-                      I.bkv * prm.rows + I.r0, 0);
+        constexpr int kCopies = REPL ? 4 : 1;   // replicated mode: the rows in every TMEM lane quarter
+        mbar_arrive_expect_tx(&q_full[qb], uint32_t(kCopies * prm.qbox * 128 * C::kNumBlk));
+        for (int cp = 0; cp < kCopies; ++cp)
+          for (int blk = 0; blk < C::kNumBlk; ++blk)
+            tma_load_3d(&tm_q, &q_full[qb],
+                        smem + C::kOffQ + qb * C::kTileBytes + blk * C::kBlockBytes + cp * 32 * 128, blk * 64,
+                        I.bkv * prm.rows + I.r0, 0);
         ++qi;
         for (int t = 0; t < 2 * I.nkv; ++t) {
           const int slot = it % C::kSlots;
@@ -277,7 +305,8 @@ attn_kvcache_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if (!(ok = mbar_wait(&kv_full[vit % C::kSlots], uint32_t((vit / C::kSlots) & 1), abort_flag))) break;
             tc_fence_after();
             const uint32_t b0 = sKV + (vit % C::kSlots) * C::kTileBytes;
-            const uint32_t at = tmem + ((ps & 1) ? C::kColS1 : C::kColS0) + C::kColPOff;
+            const uint32_t at = REPL ? tmem + ((ps & 1) ? C::kColP1 : C::kColP0)
+                                     : tmem + ((ps & 1) ? C::kColS1 : C::kColS0) + C::kColPOff;
 #pragma unroll
             for (int kk = 0; kk < 128 / 16; ++kk)
               mma_ts(tmem + C::kColO, at + kk * 8, smem_desc_sw128(b0 + kk * 2048, C::kBlockBytes, 1024), kIdescPV,
@@ -300,7 +329,11 @@ attn_kvcache_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     __syncwarp();
   } else {
     // -------------------------------------------------------------- softmax
-    const int r = warp * 32 + lane;           // row inside the tile = TMEM lane
+    // Replicated mode: every lane quarter holds the same packed rows (lane =
+    // row) and warp w takes key columns [32w, 32w + 32) of each tile: four
+    // independent online softmaxes over disjoint key subsets, merged as four
+    // partials per key chunk.
+    const int r = REPL ? lane : warp * 32 + lane;   // row inside the tile
     const uint32_t lane_base = uint32_t(warp * 32) << 16;
     const uint32_t tO = tmem + lane_base + C::kColO;
     const float c = prm.scale_log2;
@@ -311,7 +344,7 @@ attn_kvcache_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       const KvcItem I = kvc_item(prm, w, CAUSAL);
       const int rp = I.r0 + r;                // packed row
       const bool row_ok = r < I.r_valid;
-      const bool warp_on = warp * 32 < I.r_valid;
+      const bool warp_on = REPL || warp * 32 < I.r_valid;
       int lim = I.L - 1;                      // last key this row sees
       if (CAUSAL) lim = min(lim, rp % prm.nq + I.L - prm.nq);
       float m_ref = -INFINITY;
@@ -328,15 +361,74 @@ attn_kvcache_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         if (128 * j + 128 > I.L && I.L < prm.nk) {
           const int vit = it + 2 * jj + 1;
           if (!(ok = mbar_wait_warp(&kv_full[vit % C::kSlots], uint32_t((vit / C::kSlots) & 1), abort_flag))) break;
-          if (128 * j + r >= I.L) {
+          const int kr = warp * 32 + lane;     // key row of the V tile cleared by this thread
+          if (128 * j + kr >= I.L) {
             uint8_t* vt = smem + C::kOffKV + (vit % C::kSlots) * C::kTileBytes;
             for (int blk = 0; blk < C::kNumBlk; ++blk)
               for (int ch = 0; ch < 8; ++ch)
-                st_shared_v4(smem_u32(vt + blk * C::kBlockBytes) + r * 128 + ch * 16, 0u, 0u, 0u, 0u);
+                st_shared_v4(smem_u32(vt + blk * C::kBlockBytes) + kr * 128 + ch * 16, 0u, 0u, 0u, 0u);
           }
           fence_proxy_async_smem();
         }
-        if (warp_on) {
+        if (REPL) {
+          float s[32];
+          {
+            uint32_t a[32];
+            tmem_ld32(tS + 32 * warp, a);
+            tmem_ld_wait(a);
+#pragma unroll
+            for (int k = 0; k < 32; ++k) s[k] = __uint_as_float(a[k]);
+          }
+          const int limit = row_ok ? lim - 128 * j - 32 * warp : -1;
+          if (__any_sync(0xffffffffu, limit < 31)) {
+#pragma unroll
+            for (int k = 0; k < 32; ++k)
+              if (k > limit) s[k] = -INFINITY;
+          }
+          float mxp[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) mxp[u] = s[u];
+#pragma unroll
+          for (int k = 4; k < 32; k += 4)
+#pragma unroll
+            for (int u = 0; u < 4; ++u) mxp[u] = fmaxf(mxp[u], s[k + u]);
+          const float m_tile = fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])) * c;
+          float alpha = 1.f;
+          bool rescale = false;
+          if (m_tile > m_ref + kKvcRescaleLog2) {
+            alpha = ex2(m_ref - m_tile);
+            m_ref = m_tile;
+            rescale = (jj > 0);
+          }
+          l *= alpha;
+          const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
+          float sump[4] = {0.f, 0.f, 0.f, 0.f};
+          uint32_t pk[16];
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            const float p0 = ex2(fmaf(s[2 * k], c, neg_m));
+            const float p1 = ex2(fmaf(s[2 * k + 1], c, neg_m));
+            sump[k & 3] += p0 + p1;
+            pk[k] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(tmem + lane_base + (sb ? C::kColP1 : C::kColP0) + 16 * warp, pk);
+          l += (sump[0] + sump[1]) + (sump[2] + sump[3]);
+          if (__any_sync(0xffffffffu, rescale)) {
+            if (!(ok = mbar_wait_warp(pv_done, uint32_t((pvb + jj - 1) & 1), abort_flag))) break;
+            tc_fence_after();
+            const float a = rescale ? alpha : 1.f;
+#pragma unroll 1
+            for (int cc = 0; cc < D / 32; ++cc) {
+              uint32_t o[32];
+              tmem_ld32(tO + cc * 32, o);
+              tmem_ld_wait(o);
+#pragma unroll
+              for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * a);
+              tmem_st32(tO + cc * 32, o);
+            }
+          }
+          tmem_st_wait();
+        } else if (warp_on) {
           float s[128];
           {
             uint32_t a[32], bb[32], e[32], f[32];
@@ -423,6 +515,7 @@ attn_kvcache_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       const bool has = l > 0.f;                // false: the row saw no key in this chunk
       const float inv_l = has ? 1.f / l : 0.f;
       const long long row = (long long)I.bkv * prm.rows + rp;   // flat B*H*Nq row
+      const int part = REPL ? I.split * 4 + warp : I.split;      // partial written by this thread
       if (warp_on) {
 #pragma unroll 1
         for (int cc = 0; cc < D / 32; ++cc) {
@@ -436,8 +529,7 @@ attn_kvcache_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           }
           if (row_ok) {
             if (SPLIT) {
-              float4* dst =
-                  reinterpret_cast<float4*>(prm.part_o + ((long long)I.split * prm.total_rows + row) * D + cc * 32);
+              float4* dst = reinterpret_cast<float4*>(prm.part_o + ((long long)part * prm.total_rows + row) * D + cc * 32);
 #pragma unroll
               for (int k = 0; k < 8; ++k)
                 dst[k] = make_float4(__uint_as_float(o[4 * k]) * inv_l, __uint_as_float(o[4 * k + 1]) * inv_l,
@@ -457,7 +549,7 @@ attn_kvcache_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         if (row_ok) {
           const float lse = has ? (m_ref + __log2f(l)) * kKvcLn2 : -INFINITY;
           if (SPLIT)
-            prm.part_lse[(long long)I.split * prm.total_rows + row] = lse;
+            prm.part_lse[(long long)part * prm.total_rows + row] = lse;
           else
             prm.lse[row] = lse;
         }

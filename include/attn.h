@@ -138,11 +138,15 @@ int attn_fwd_fp8(const void* Q8, const void* K8, const void* V8, void* O, float*
  * mask).  A row that sees no key (L_b = 0, or p + L_b - Nq < 0) gets O = 0 and
  * LSE = -inf.  Query head h reads key/value head h / (H / H_kv).
  * num_splits: key tiles of each (key/value head, 128 packed query rows) are
- * cut into this many chunks, one CTA each, and the partial results are merged
- * by their LSE; 0 picks a count that fills the GPU's 148 SMs.  With more than
- * one split the call needs attn_fwd_kvcache_workspace_bytes() bytes of device
- * workspace (16-byte aligned) for the fp32 partials, else ATTN_ERR_WORKSPACE;
- * with one split `workspace` may be NULL.  Requires B*H*Nq < 2^31 - 128.
+ * cut into this many chunks (work items of a persistent grid) and the partial
+ * results are merged by their LSE; 0 picks a count that fills the GPU's 148
+ * SMs.  When (H / H_kv) * Nq <= 32 the packed rows are replicated into all
+ * four TMEM lane quarters and every key tile is split four ways, so each chunk
+ * yields four partials.  Whenever there is more than one partial the call
+ * needs attn_fwd_kvcache_workspace_bytes() bytes of device workspace
+ * (16-byte aligned) for the fp32 partials, else ATTN_ERR_WORKSPACE (or
+ * ATTN_ERR_INVALID_ARG for NULL); when that function returns 0, `workspace`
+ * may be NULL.  Requires B*H*Nq < 2^31 - 128.
  * Outputs must not alias inputs or the workspace.
  */
 int attn_fwd_kvcache(const void* Q, const void* K, const void* V, void* O, float* LSE,
@@ -154,8 +158,9 @@ int attn_fwd_kvcache(const void* Q, const void* K, const void* V, void* O, float
 /*
  * Number of key chunks attn_fwd_kvcache uses for these arguments (num_splits
  * as passed to it, 0 = automatic), and the workspace bytes it then needs:
- * splits * B*H*Nq * (d + 1) * 4 when splits > 1, else 0.  Both return 0 for
- * sizes attn_fwd_kvcache would reject.
+ * partials * B*H*Nq * (d + 1) * 4 with partials = splits * (4 if
+ * (H / H_kv) * Nq <= 32 else 1), or 0 when there is a single partial.  Both
+ * return 0 for sizes attn_fwd_kvcache would reject.
  */
 int64_t attn_fwd_kvcache_splits(int64_t B, int64_t H, int64_t H_kv, int64_t Nq, int64_t Nk, int64_t d,
                                 int64_t num_splits);

@@ -125,7 +125,12 @@ def test_kvcache_splits_and_workspace(lib):
     # decode batch with 64 key/value heads over a 16K cache: many splits, all SMs busy
     s = attn.attn_fwd_kvcache_splits(8, 32, 8, 1, 16384, 128, 0)
     assert 2 <= s <= 128
-    assert attn.attn_fwd_kvcache_workspace_bytes(8, 32, 8, 1, 16384, 128, 0) == s * 8 * 32 * 1 * 129 * 4
+    # 4 packed rows per key/value head: replicated into the four lane quarters, four partials per chunk
+    assert attn.attn_fwd_kvcache_workspace_bytes(8, 32, 8, 1, 16384, 128, 0) == 4 * s * 8 * 32 * 1 * 129 * 4
+    # 40 packed rows: one partial per chunk; a single chunk needs no workspace
+    assert attn.attn_fwd_kvcache_workspace_bytes(1, 8, 2, 10, 1000, 64, 3) == 3 * 8 * 10 * 65 * 4
+    assert attn.attn_fwd_kvcache_workspace_bytes(1, 8, 2, 10, 1000, 64, 1) == 0
+    assert attn.attn_fwd_kvcache_workspace_bytes(1, 8, 2, 1, 1000, 64, 1) == 4 * 8 * 1 * 65 * 4
     # a large prefill-sized grid needs no split and no workspace
     assert attn.attn_fwd_kvcache_splits(8, 32, 32, 512, 2048, 128, 0) == 1
     assert attn.attn_fwd_kvcache_workspace_bytes(8, 32, 32, 512, 2048, 128, 0) == 0
@@ -154,7 +159,7 @@ def test_kvcache_argument_errors(lib):
         assert call(ptrs=q) == attn.ATTN_ERR_MISALIGNED
     # two splits need a workspace of the advertised size
     need = attn.attn_fwd_kvcache_workspace_bytes(1, 4, 2, 1, 256, 64, 2)
-    assert need == 2 * 4 * 65 * 4
+    assert need == 4 * 2 * 4 * 65 * 4          # 2 packed rows: four partials per chunk
     assert call(splits=2) == attn.ATTN_ERR_INVALID_ARG
     assert call(splits=2, ws=MIS, ws_bytes=need) == attn.ATTN_ERR_MISALIGNED
     assert call(splits=2, ws=A, ws_bytes=need - 4) == attn.ATTN_ERR_WORKSPACE

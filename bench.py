@@ -598,7 +598,7 @@ def run_reference(args):
         "metric": METRIC,
         "value": round(value, 6),
         "unit": "TFLOP/s",
-        "n_gpus": 0,
+        "n_gpus": args.gpus,          # the launch it belongs to; the work itself runs on host cores
         "steps": args.steps,
         "warmup": args.warmup,
         "ms_per_step": round(ms, 1),

@@ -474,6 +474,7 @@ namespace {
 
 constexpr int64_t kNumSMs = 148;   // B200: sizes the persistent grid and the automatic split count
 constexpr int64_t kMaxSplits = 256;
+static_assert(kMaxSplits * 4 <= attn::kKvcMaxParts, "the merge kernel holds every partial's LSE in shared memory");
 
 struct KvcShape {
   int64_t rows = 0;        // packed query rows per key/value head
@@ -539,8 +540,8 @@ int launch_kvc(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
   kern<<<grid, attn::KvcCfg<D>::kThreads, smem, st>>>(q, k, v, prm);
   int s = launch_status();
   if (s != ATTN_OK || !SPLIT) return s;
-  int64_t blocks = (prm.total_rows + 7) / 8;                  // 8 rows (warps) per 256-thread block
-  if (blocks > kNumSMs * 16) blocks = kNumSMs * 16;
+  int64_t blocks = prm.total_rows;                            // one 256-thread block per row
+  if (blocks > kNumSMs * 8) blocks = kNumSMs * 8;
   attn::attn_kvcache_merge_kernel<D><<<int(blocks), 256, 0, st>>>(prm.part_o, prm.part_lse, prm.o, prm.lse,
                                                                    prm.total_rows, prm.splits * (REPL ? 4 : 1));
   return launch_status();

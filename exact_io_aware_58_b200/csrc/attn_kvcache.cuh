@@ -575,53 +575,90 @@ attn_kvcache_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   }
 }
 
-// Combines the split-KV partials of each row: one warp per row.
+// Combines the split-KV partials of each row: one 256-thread block per row
+// (grid-stride).  The partials' LSEs go through shared memory once; each of
+// the 8 warps then accumulates every 8th partial (all its loads independent,
+// so they are in flight together), and the warps' sums are added in shared
+// memory.  Every partial row is written by the main kernel (zeros where a
+// chunk saw no key), so no load is conditional.
+constexpr int kKvcMaxParts = 1024;
+
 template <int D>
 __global__ void __launch_bounds__(256)
 attn_kvcache_merge_kernel(const float* __restrict__ part_o, const float* __restrict__ part_lse,
-                          __nv_bfloat16* __restrict__ o, float* __restrict__ lse, long long total_rows, int splits) {
+                          __nv_bfloat16* __restrict__ o, float* __restrict__ lse, long long total_rows, int parts) {
   constexpr int kPer = D / 32;                 // columns per lane
+  __shared__ float s_lse[kKvcMaxParts];
+  __shared__ float s_acc[8][D];
+  __shared__ float s_red[8];
+  __shared__ float s_sum[8];
+  const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
-  for (long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); row < total_rows;
-       row += warps) {
+  for (long long row = blockIdx.x; row < total_rows; row += gridDim.x) {
     float mx = -INFINITY;
-    for (int s = lane; s < splits; s += 32) mx = fmaxf(mx, part_lse[(long long)s * total_rows + row]);
+    for (int s = threadIdx.x; s < parts; s += 256) {
+      const float v = part_lse[(long long)s * total_rows + row];
+      s_lse[s] = v;
+      mx = fmaxf(mx, v);
+    }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    if (lane == 0) s_red[warp] = mx;
+    __syncthreads();
+    mx = s_red[0];
+#pragma unroll
+    for (int w = 1; w < 8; ++w) mx = fmaxf(mx, s_red[w]);
     float acc[kPer];
 #pragma unroll
     for (int k = 0; k < kPer; ++k) acc[k] = 0.f;
     float sum = 0.f;
     if (mx != -INFINITY) {
-      for (int s = 0; s < splits; ++s) {
-        const float ls = part_lse[(long long)s * total_rows + row];
-        if (ls == -INFINITY) continue;         // the chunk saw no key for this row
-        const float w = expf(ls - mx);
+#pragma unroll 4
+      for (int s = warp; s < parts; s += 8) {
+        const float ls = s_lse[s];
+        const float w = (ls == -INFINITY) ? 0.f : expf(ls - mx);
         sum += w;
         const float* src = part_o + ((long long)s * total_rows + row) * D + lane * kPer;
         if constexpr (kPer == 4) {
-          const float4 v = *reinterpret_cast<const float4*>(src);
-          acc[0] = fmaf(w, v.x, acc[0]);
-          acc[1] = fmaf(w, v.y, acc[1]);
-          acc[2] = fmaf(w, v.z, acc[2]);
-          acc[3] = fmaf(w, v.w, acc[3]);
+          const float4 t = *reinterpret_cast<const float4*>(src);
+          acc[0] = fmaf(w, t.x, acc[0]);
+          acc[1] = fmaf(w, t.y, acc[1]);
+          acc[2] = fmaf(w, t.z, acc[2]);
+          acc[3] = fmaf(w, t.w, acc[3]);
         } else {
-          const float2 v = *reinterpret_cast<const float2*>(src);
-          acc[0] = fmaf(w, v.x, acc[0]);
-          acc[1] = fmaf(w, v.y, acc[1]);
+          const float2 t = *reinterpret_cast<const float2*>(src);
+          acc[0] = fmaf(w, t.x, acc[0]);
+          acc[1] = fmaf(w, t.y, acc[1]);
         }
       }
     }
-    const float inv = sum > 0.f ? 1.f / sum : 0.f;
-    __nv_bfloat16* dst = o + row * D + lane * kPer;
-    if constexpr (kPer == 4) {
-      *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(acc[0] * inv, acc[1] * inv),
-                                                  pack_bf16x2(acc[2] * inv, acc[3] * inv));
-    } else {
-      *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) s_acc[warp][lane * kPer + k] = acc[k];
+    if (lane == 0) s_sum[warp] = sum;
+    __syncthreads();
+    if (warp == 0) {
+      float tot = 0.f;
+#pragma unroll
+      for (int w = 0; w < 8; ++w) tot += s_sum[w];
+      float out[kPer];
+#pragma unroll
+      for (int k = 0; k < kPer; ++k) {
+        float a = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) a += s_acc[w][lane * kPer + k];
+        out[k] = a;
+      }
+      const float inv = tot > 0.f ? 1.f / tot : 0.f;
+      __nv_bfloat16* dst = o + row * D + lane * kPer;
+      if constexpr (kPer == 4) {
+        *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(out[0] * inv, out[1] * inv),
+                                                    pack_bf16x2(out[2] * inv, out[3] * inv));
+      } else {
+        *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(out[0] * inv, out[1] * inv);
+      }
+      if (lane == 0) lse[row] = tot > 0.f ? mx + logf(tot) : -INFINITY;
     }
-    if (lane == 0) lse[row] = sum > 0.f ? mx + logf(sum) : -INFINITY;
+    __syncthreads();   // shared memory is reused by the next row
   }
 }
 

@@ -31,7 +31,7 @@ ATTN_ERR_TIMEOUT = -6
 ATTN_ERR_DEVICE = -7
 
 EXPORTED = ("attn_fwd", "attn_fwd_gqa", "attn_fwd_blocksparse", "attn_bwd", "attn_bwd_gqa", "attn_bwd_blocksparse",
-            "attn_bwd_workspace_bytes", "attn_fwd_fp8", "attn_fwd_kvcache", "attn_fwd_kvcache_splits",
+            "attn_bwd_workspace_bytes", "attn_fwd_fp8", "attn_fwd_kvcache", "attn_fwd_kvcache_fp8", "attn_fwd_kvcache_splits",
             "attn_fwd_kvcache_workspace_bytes",
             "attn_bwd_preprocess", "attn_bwd_dkdv",
             "attn_bwd_dq", "attn_bwd_static_workspace", "attn_check_status", "attn_last_error",
@@ -80,6 +80,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.attn_fwd_kvcache.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i32, f32, i64, vp,
                                      ctypes.c_size_t, vp]
     lib.attn_fwd_kvcache.restype = i32
+    lib.attn_fwd_kvcache_fp8.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i32, f32, f32, f32,
+                                         i64, vp, ctypes.c_size_t, vp]
+    lib.attn_fwd_kvcache_fp8.restype = i32
     lib.attn_fwd_kvcache_splits.argtypes = [i64] * 7
     lib.attn_fwd_kvcache_splits.restype = i64
     lib.attn_fwd_kvcache_workspace_bytes.argtypes = [i64] * 7
@@ -304,6 +307,34 @@ def attn_fwd_kvcache(Q, K, V, O, LSE, kv_lens, causal: bool, scale: float, num_s
                                          wp, wb, _stream_handle(stream))
     if st != ATTN_OK:
         raise AttnError(st, "attn_fwd_kvcache")
+
+
+def attn_fwd_kvcache_fp8(Q, K8, V8, O, LSE, kv_lens, causal: bool, scale: float, k_descale: float,
+                         v_descale: float, num_splits: int = 0, workspace=None, stream=None) -> None:
+    """attn_fwd_kvcache with an E4M3 cache: K8, V8 (B, H_kv, Nk, 128) float8_e4m3fn or uint8 CUDA tensors."""
+    _check_bhnd("Q", Q)
+    _check_bhnd("O", O, Q.shape)
+    _check_lse(LSE, Q.shape)
+    B, H, Nq, d = Q.shape
+    for name, t in (("K8", K8), ("V8", V8)):
+        if not t.is_cuda or t.dtype not in (torch.float8_e4m3fn, torch.uint8) or t.dim() != 4 \
+                or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA float8_e4m3fn (or uint8) tensor of rank 4")
+    if K8.shape != V8.shape or K8.shape[0] != B or K8.shape[3] != d or K8.shape[1] < 1 or H % K8.shape[1] != 0:
+        raise ValueError(f"K8, V8 have shapes {tuple(K8.shape)}, {tuple(V8.shape)}; expected (B, H_kv, Nk, d)")
+    if kv_lens is not None and (not kv_lens.is_cuda or kv_lens.dtype != torch.int32 or tuple(kv_lens.shape) != (B,)
+                                or not kv_lens.is_contiguous()):
+        raise ValueError("kv_lens must be a contiguous CUDA int32 tensor of shape (B,)")
+    if workspace is None:
+        raise ValueError("attn_fwd_kvcache_fp8 needs a workspace (attn_fwd_kvcache_workspace_bytes)")
+    wp, wb = _ws(workspace)
+    st = load_library().attn_fwd_kvcache_fp8(_ptr(Q), _ptr(K8), _ptr(V8), _ptr(O), _ptr(LSE),
+                                             ctypes.c_void_p(None) if kv_lens is None else _ptr(kv_lens),
+                                             B, H, K8.shape[1], Nq, K8.shape[2], d, int(bool(causal)), float(scale),
+                                             float(k_descale), float(v_descale), int(num_splits), wp, wb,
+                                             _stream_handle(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd_kvcache_fp8")
 
 
 def attn_bwd_workspace_bytes(B: int, H: int, N: int, d: int) -> int:

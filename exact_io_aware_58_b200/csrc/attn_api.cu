@@ -20,6 +20,7 @@
 #include "attn_fwd.cuh"
 #include "attn_fwd_fp8.cuh"
 #include "attn_kvcache.cuh"
+#include "attn_kvcache_fp8.cuh"
 
 namespace {
 
@@ -625,6 +626,92 @@ ATTN_EXPORT int attn_fwd_kvcache(const void* Q, const void* K, const void* V, vo
                   : dispatch_kvc<128, false>(split, repl, mq, mk, mv, prm, int(grid), st);
   return causal ? dispatch_kvc<64, true>(split, repl, mq, mk, mv, prm, int(grid), st)
                 : dispatch_kvc<64, false>(split, repl, mq, mk, mv, prm, int(grid), st);
+}
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode against an FP8 (E4M3) key/value cache.
+// ---------------------------------------------------------------------------
+namespace {
+
+template <bool CAUSAL>
+int launch_kvc8(const CUtensorMap& q, const CUtensorMap& k8, const CUtensorMap& v8, const attn::KvcParams& prm,
+                float v_descale, int grid, cudaStream_t st) {
+  auto kern = attn::attn_kvcache_fp8_kernel<CAUSAL>;
+  constexpr int smem = attn::Kvc8Cfg::kSmemBytes;
+  if (set_smem(reinterpret_cast<const void*>(kern), smem) != ATTN_OK) return ATTN_ERR_LAUNCH;
+  kern<<<grid, attn::Kvc8Cfg::kThreads, smem, st>>>(q, k8, v8, prm, v_descale);
+  int s = launch_status();
+  if (s != ATTN_OK) return s;
+  int64_t blocks = prm.total_rows;
+  if (blocks > kNumSMs * 8) blocks = kNumSMs * 8;
+  attn::attn_kvcache_merge_kernel<128><<<int(blocks), 256, 0, st>>>(prm.part_o, prm.part_lse, prm.o, prm.lse,
+                                                                     prm.total_rows, prm.splits * 4);
+  return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+ATTN_EXPORT int attn_fwd_kvcache_fp8(const void* Q, const void* K8, const void* V8, void* O, float* LSE,
+                                     const int32_t* kv_lens, int64_t B, int64_t H, int64_t H_kv, int64_t Nq,
+                                     int64_t Nk, int64_t d, int causal, float scale, float k_descale,
+                                     float v_descale, int64_t num_splits, void* workspace, size_t workspace_bytes,
+                                     void* stream) {
+  KvcShape sh;
+  int s = kvc_check(B, H, H_kv, Nq, Nk, d, &sh);
+  if (s != ATTN_OK) return s;
+  if (d != 128)
+    return fail(ATTN_ERR_UNSUPPORTED, "%sattn_fwd_kvcache_fp8 supports d = 128 only (got %lld)", "", (long long)d);
+  if (!kvc_replicated(sh))
+    return fail(ATTN_ERR_UNSUPPORTED,
+                "%sattn_fwd_kvcache_fp8 takes at most 32 query rows per key/value head ((H / H_kv) * Nq = %lld)", "",
+                (long long)sh.rows);
+  if ((s = check_scale(scale)) != ATTN_OK) return s;
+  if (!(std::isfinite(k_descale) && k_descale > 0.f) || !(std::isfinite(v_descale) && v_descale > 0.f))
+    return ATTN_ERR_INVALID_ARG;
+  const int64_t splits = kvc_splits(sh, B, H_kv, num_splits);
+  if (splits < 1) return ATTN_ERR_INVALID_ARG;
+  if (!Q || !K8 || !V8 || !O || !LSE || !workspace) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K8) || !aligned16(V8) || !aligned16(O) || !aligned16(LSE) || !aligned16(workspace))
+    return ATTN_ERR_MISALIGNED;
+  if (kv_lens && (reinterpret_cast<uintptr_t>(kv_lens) & 3u) != 0) return ATTN_ERR_MISALIGNED;
+  if (workspace_bytes < kvc_workspace(sh, splits, d)) return ATTN_ERR_WORKSPACE;
+  const int64_t n_items = B * H_kv * sh.n_rt * splits;
+  if (n_items > INT32_MAX) return ATTN_ERR_INVALID_ARG;
+  const int64_t grid = std::min<int64_t>(n_items, kNumSMs);
+  const int qbox = int((sh.rows + 7) / 8 * 8);
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, Q, 1, sh.total_rows, d, qbox) || !make_map_u8(&mk, K8, B * H_kv, Nk, d) ||
+      !make_map_u8(&mv, V8, B * H_kv, Nk, d))
+    return ATTN_ERR_LAUNCH;
+  const int64_t parts = kvc_partials(sh, splits);
+  attn::KvcParams prm;
+  prm.o = static_cast<__nv_bfloat16*>(O);
+  prm.lse = LSE;
+  prm.part_o = static_cast<float*>(workspace);
+  prm.part_lse = static_cast<float*>(workspace) + size_t(parts) * size_t(sh.total_rows) * size_t(d);
+  prm.kv_lens = kv_lens;
+  prm.total_rows = sh.total_rows;
+  prm.nq = int(Nq);
+  prm.nk = int(Nk);
+  prm.h_kv = int(H_kv);
+  prm.rows = int(sh.rows);
+  prm.n_rt = int(sh.n_rt);
+  prm.splits = int(splits);
+  prm.qbox = qbox;
+  prm.n_items = int(n_items);
+  // The widened tiles hold 2^-8 times the E4M3 values (see the kernel): the
+  // factor goes into the exp2 argument and into the final 1/l.
+  prm.scale_log2 = float(double(scale) * double(k_descale) * 256.0 * 1.4426950408889634);
+  const float v_scale = float(double(v_descale) * 256.0);
+  if (!std::isfinite(prm.scale_log2) || !(prm.scale_log2 > 0.f) || !std::isfinite(v_scale))
+    return ATTN_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return causal ? launch_kvc8<true>(mq, mk, mv, prm, v_scale, int(grid), st)
+                : launch_kvc8<false>(mq, mk, mv, prm, v_scale, int(grid), st);
 }
 
 }  // extern "C"

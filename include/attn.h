@@ -156,6 +156,28 @@ int attn_fwd_kvcache(const void* Q, const void* K, const void* V, void* O, float
                      void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * attn_fwd_kvcache with the cache stored in FP8: K8, V8 are uint8 [B][H_kv][Nk][128]
+ * E4M3 codes with per-tensor dequantisation factors k_descale, v_descale (finite,
+ * > 0); the result is attn_fwd_kvcache's on K = k_descale * K8, V = v_descale * V8
+ * (every E4M3 value times 2^-8 is exactly an f16 value, so the cache is widened
+ * on chip without rounding; the query tile is converted to f16 on chip, which is
+ * exact for bf16 values of magnitude 2^-14 .. 65504 -- larger |Q| elements are
+ * outside this entry point's domain, smaller ones round to f16's subnormal
+ * grid, an absolute error below 2^-25 -- and the arithmetic is otherwise that
+ * of the bf16 path: fp32 scores and statistics, P rounded to f16).  Reading half
+ * the bytes per cached row is the point: decode reads the whole cache every
+ * step.  Q, O bf16 and LSE, kv_lens, causal alignment, num_splits as in
+ * attn_fwd_kvcache.  Restrictions: d = 128 and (H / H_kv) * Nq <= 32 (decode
+ * shapes), else ATTN_ERR_UNSUPPORTED.  The workspace is always needed, sized by
+ * attn_fwd_kvcache_workspace_bytes() with the same arguments.
+ */
+int attn_fwd_kvcache_fp8(const void* Q, const void* K8, const void* V8, void* O, float* LSE,
+                         const int32_t* kv_lens,
+                         int64_t B, int64_t H, int64_t H_kv, int64_t Nq, int64_t Nk, int64_t d,
+                         int causal, float scale, float k_descale, float v_descale, int64_t num_splits,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Number of key chunks attn_fwd_kvcache uses for these arguments (num_splits
  * as passed to it, 0 = automatic), and the workspace bytes it then needs:
  * partials * B*H*Nq * (d + 1) * 4 with partials = splits * (4 if

@@ -58,6 +58,7 @@ __all__ = [
     "attn_fwd_kvcache",
     "e4m3_decode",
     "attn_fwd_fp8",
+    "attn_fwd_kvcache_fp8",
 ]
 
 
@@ -342,3 +343,11 @@ def attn_fwd_fp8(Q8, K8, V8, q_descale: float, k_descale: float, v_descale: floa
     K = float(k_descale) * e4m3_decode(K8)
     V = float(v_descale) * e4m3_decode(V8)
     return attn_fwd_gqa(Q, K, V, scale, causal, B, H, H_kv)
+
+
+def attn_fwd_kvcache_fp8(Q, K8, V8, k_descale: float, v_descale: float, scale: float, causal: bool,
+                         B: int, H: int, H_kv: int, kv_lens=None):
+    """Decode against an E4M3 cache: attn_fwd_kvcache on K = k_descale * decode(K8), V = v_descale * decode(V8)."""
+    K = float(k_descale) * e4m3_decode(K8)
+    V = float(v_descale) * e4m3_decode(V8)
+    return attn_fwd_kvcache(Q, K, V, scale, causal, B, H, H_kv, kv_lens=kv_lens)

@@ -181,3 +181,26 @@ def test_fp8_argument_errors(lib):
         q = [A] * 5
         q[k] = MIS
         assert call(ptrs=q) == attn.ATTN_ERR_MISALIGNED
+
+
+def test_kvcache_fp8_argument_errors(lib):
+    p = [A] * 5
+    ws_ok = attn.attn_fwd_kvcache_workspace_bytes(1, 4, 2, 1, 256, 128, 2)
+
+    def call(H=4, Hk=2, Nq=1, d=128, kd=1.0, vd=1.0, ws=A, ws_bytes=None, ptrs=None):
+        wb = ws_ok if ws_bytes is None else ws_bytes
+        return lib.attn_fwd_kvcache_fp8(*(ptrs or p), None, 1, H, Hk, Nq, 256, d, 1, 0.125, kd, vd, 2, ws, wb,
+                                        None)
+
+    assert call(d=64) == attn.ATTN_ERR_UNSUPPORTED
+    assert call(H=64, Hk=1) == attn.ATTN_ERR_UNSUPPORTED        # 64 packed rows per key/value head
+    assert call(Nq=17) == attn.ATTN_ERR_UNSUPPORTED             # 2 * 17 = 34 > 32
+    for bad in (0.0, -2.0, float("nan")):
+        assert call(kd=bad) == attn.ATTN_ERR_INVALID_ARG
+        assert call(vd=bad) == attn.ATTN_ERR_INVALID_ARG
+    assert call(ws=None) == attn.ATTN_ERR_INVALID_ARG
+    assert call(ws_bytes=ws_ok - 4) == attn.ATTN_ERR_WORKSPACE
+    for k in range(5):
+        q = [A] * 5
+        q[k] = MIS
+        assert call(ptrs=q) == attn.ATTN_ERR_MISALIGNED

@@ -701,3 +701,19 @@ def test_fp8_forward_is_attention_on_dequantised_values():
         O2, L2 = orc.attn_fwd_gqa(Qd, Kd, Vd, 0.3, causal, B, H, Hk)
         np.testing.assert_allclose(O, O2, rtol=1e-14)
         np.testing.assert_allclose(L, L2, rtol=1e-14)
+
+
+def test_kvcache_fp8_is_kvcache_on_the_dequantised_cache():
+    # codes 0x38 + k (k < 8) decode to 1 + k/8; the descales are powers of two,
+    # so the dequantised cache is known exactly without the decoder
+    rng = np.random.default_rng(610)
+    B, H, Hk, nq, nk, d = 2, 4, 2, 1, 9, 3
+    q = _rand((B * H, nq, d), 611)
+    k8 = (0x38 + rng.integers(0, 8, (B * Hk, nk, d))).astype(np.uint8)
+    v8 = (0xB8 + rng.integers(0, 8, (B * Hk, nk, d))).astype(np.uint8)
+    Kd = 0.25 * (1 + (k8 - 0x38) / 8.0)
+    Vd = 2.0 * -(1 + (v8 - 0xB8) / 8.0)
+    O, L = orc.attn_fwd_kvcache_fp8(q, k8, v8, 0.25, 2.0, 0.7, True, B, H, Hk, kv_lens=[9, 4])
+    O2, L2 = orc.attn_fwd_kvcache(q, Kd, Vd, 0.7, True, B, H, Hk, kv_lens=[9, 4])
+    np.testing.assert_allclose(O, O2, rtol=1e-14)
+    np.testing.assert_allclose(L, L2, rtol=1e-14)

@@ -12,16 +12,17 @@
 // kernel (work item = key/value head x key chunk, up to 32 packed query rows
 // replicated over the four TMEM lane quarters, warp w of the softmax owning
 // key columns [32w, 32w+32), four partials per item merged by LSE), with one
-// change: the cache tiles arrive as E4M3 bytes (TMA, 16 KB per tile) and the
-// four softmax warps widen them into one f16 K tile and one f16 V tile in
-// shared memory with integer operations only (exactly: every E4M3 value times
-// 2^-8 is an f16 value, normal or subnormal; the 2^8 goes into the scales).
-// The MMAs run as kind::f16 with f16 operands: the query tile is converted
-// from bf16 to f16 in shared memory once per work item (exact for |q| in the
-// f16 range, up to 65504) and P is packed as f16.  K_{j+1} is widened as soon as S_j
-// has completed (so S_{j+1} runs during the softmax of tile j), V_j once PV_{j-1}
-// has completed.  dk is folded into the exp2 argument and dv into the final
-// 1/l.  Cache rows past the valid length are widened as zeros in V.  d = 128.
+// change: the cache tiles arrive as E4M3 bytes (TMA, 16 KB per tile) and eight
+// dedicated widening warps turn them into one f16 K tile and one f16 V tile
+// in shared memory with integer operations only (exactly: every E4M3 value
+// times 2^-8 is an f16 value, normal or subnormal; the 2^8 goes into the
+// scales).  The MMAs run as kind::f16 with f16 operands: the widening warps
+// also convert each work item's query tile from bf16 to f16 in shared memory
+// (exact for |q| in [2^-14, 65504]) and the softmax packs P as f16.
+// K_{j+1} is widened as soon as S_j has completed, V_j once PV_{j-1} has
+// completed, so the widening of one tile overlaps the softmax of the previous
+// one.  dk is folded into the exp2 argument and dv into the final 1/l.  Cache
+// rows past the valid length are widened as zeros in V.  d = 128.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -34,14 +35,17 @@ namespace attn {
 
 struct Kvc8Cfg {
   static constexpr int D = 128;
-  static constexpr int kTileBytes = 128 * D * 2;       // bf16 tiles (Q, widened K, widened V)
+  static constexpr int kTileBytes = 128 * D * 2;       // 16-bit tiles (Q, widened K, widened V)
   static constexpr int kTile8Bytes = 128 * D;          // E4M3 tile: 128 rows x 128 bytes
   static constexpr int kBlockBytes = 128 * 128;
   static constexpr int kNumBlk = D / 64;
   static constexpr int kSlots = 6;                     // E4M3 ring: three key tiles ahead
-  static constexpr int kThreads = 192;
   static constexpr int kWarpMma = 4;
   static constexpr int kWarpLoad = 5;
+  static constexpr int kWarpWiden0 = 6;                // warps 6 .. 6 + kWidenWarps - 1
+  static constexpr int kWidenWarps = 8;
+  static constexpr int kWidenThreads = 32 * kWidenWarps;
+  static constexpr int kThreads = 32 * kWarpWiden0 + kWidenThreads;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256;
   static constexpr uint32_t kColP0 = 384, kColP1 = 448;
@@ -51,11 +55,12 @@ struct Kvc8Cfg {
   static constexpr int kOffVb = kOffKb + kTileBytes;
   static constexpr int kOffBar = kOffVb + kTileBytes;
   // q_full, q_empty, ring_full[S], ring_empty[S], s_full[2], p_full[2], pv_done, o_full, o_free,
-  // kb_full, vb_full, drain, q_ready
-  static constexpr int kNumBars = 2 + 2 * kSlots + 2 + 2 + 3 + 2 + 1 + 1;
+  // kb_full, kb_free, vb_full, vb_free, drain, q_ready
+  static constexpr int kNumBars = 2 + 2 * kSlots + 2 + 2 + 3 + 4 + 1 + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
 };
+static_assert(Kvc8Cfg::kSmemBytes <= 227 * 1024, "shared memory");
 
 __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
   uint4 v;
@@ -64,13 +69,16 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
 }
 
 // Two E4M3 codes (bytes 0 and 2 of x, bytes 1 and 3 zero) -> one f16x2 word
-// holding 2^-8 times their values, with integer operations only: the code
+// holding 2^-8 times their values, with integer operations only.  The code
 // s.eeee.mmm placed at f16 bits 15 / 13..10 / 9..7 is the f16 number
 // 2^(e-15) * 1.mmm (or 0.mmm * 2^-14 for e = 0), i.e. exactly 2^-8 times the
-// E4M3 value 2^(e-7) * 1.mmm (0.mmm * 2^-6).  The factor 2^8 is folded into
-// the dequantisation scales.  (The E4M3 NaN code reads as 2^-8 * 480.)
+// E4M3 value 2^(e-7) * 1.mmm (0.mmm * 2^-6).  Shifting the code left by 7
+// puts eeee.mmm in place and the sign at bit 14; adding the sign bit once
+// more first carries it to bit 15 (a code plus its sign bit is at most 0x17F,
+// so nothing crosses into the other half).  The factor 2^8 is folded into the
+// dequantisation scales.  (The E4M3 NaN code reads as 2^-8 * 480.)
 __device__ __forceinline__ uint32_t e4m3_pair_to_f16x2(uint32_t x) {
-  return ((x & 0x007F007Fu) << 7) | ((x & 0x00800080u) << 8);
+  return (x + (x & 0x00800080u)) << 7;
 }
 
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
@@ -84,14 +92,21 @@ __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool a_mn_major, 
          (uint32_t(N >> 3) << 17) | (uint32_t(M >> 4) << 24);
 }
 
-// Widen one 128 x 128 E4M3 tile (128-byte swizzled rows) into a bf16 tile
-// (two [128][64] column blocks, 128-byte swizzle), all 128 threads: 8 lanes
-// per row, 16 rows per pass.  Rows >= zero_from are written as zeros.
-__device__ __forceinline__ void widen_tile(uint32_t src8, uint32_t dstb, int tid, int zero_from) {
-  const int c = tid & 7;                 // 16-byte chunk of the E4M3 row = elements 16c..16c+15
+// Widen one 128 x 128 E4M3 tile (128-byte swizzled rows) into an f16 tile
+// (two [128][64] column blocks, 128-byte swizzle) with the kWidenThreads
+// widening threads: 8 lanes per row (lane c reads bytes 16c..16c+15), 32 rows
+// per pass.  Rows >= zero_from are written as zeros.  Lane c's 16 values are
+// two 16-byte chunks of column block c / 4; lanes c < 4 store their even
+// chunk first and lanes c >= 4 their odd chunk first, so the eight lanes of
+// one row hit eight different bank groups in each store.
+__device__ __forceinline__ void widen_tile(uint32_t src8, uint32_t dstb, int t, int zero_from) {
+  const int c = t & 7;
+  const uint32_t blk = dstb + (c >> 2) * Kvc8Cfg::kBlockBytes;
+  const uint32_t ch = (c & 3) * 2;
+  const bool odd_first = c >= 4;
 #pragma unroll 2
-  for (int pass = 0; pass < 8; ++pass) {
-    const int row = pass * 16 + (tid >> 3);
+  for (int pass = 0; pass < 128 * 8 / Kvc8Cfg::kWidenThreads; ++pass) {
+    const int row = pass * (Kvc8Cfg::kWidenThreads / 8) + (t >> 3);
     const uint4 v = ld_shared_v4(src8 + row * 128 + ((c ^ (row & 7)) << 4));
     uint32_t w[8];
     const uint32_t in[4] = {v.x, v.y, v.z, v.w};
@@ -104,15 +119,42 @@ __device__ __forceinline__ void widen_tile(uint32_t src8, uint32_t dstb, int tid
 #pragma unroll
       for (int k = 0; k < 8; ++k) w[k] = 0u;
     }
-    const uint32_t blk = dstb + (c >> 2) * 16384;
-    const uint32_t ch = (c & 3) * 2;
-    st_shared_v4(blk + sw128_offset(row, ch), w[0], w[1], w[2], w[3]);
-    st_shared_v4(blk + sw128_offset(row, ch + 1), w[4], w[5], w[6], w[7]);
+    const uint32_t a0 = blk + sw128_offset(row, ch);
+    const uint32_t a1 = blk + sw128_offset(row, ch + 1);
+    if (odd_first) {
+      st_shared_v4(a1, w[4], w[5], w[6], w[7]);
+      st_shared_v4(a0, w[0], w[1], w[2], w[3]);
+    } else {
+      st_shared_v4(a0, w[0], w[1], w[2], w[3]);
+      st_shared_v4(a1, w[4], w[5], w[6], w[7]);
+    }
+  }
+}
+
+// The query tile (bf16, [128][64] column blocks, 128-byte swizzle) -> f16 in
+// place, by the widening threads: 16-byte chunk q = pass * kWidenThreads + t
+// is chunk q % 8 of column block (q / 8) % 2 of row q / 16, so the eight lanes
+// of a row read and write eight different bank groups.  Rows that are padding
+// in every lane quarter are zeros already and are skipped.
+__device__ __forceinline__ void convert_q_tile(uint32_t sq, int t, int qbox) {
+#pragma unroll 2
+  for (int pass = 0; pass < 128 * 16 / Kvc8Cfg::kWidenThreads; ++pass) {
+    const int q = pass * Kvc8Cfg::kWidenThreads + t;
+    const int row = q >> 4;
+    if ((row & 31) >= qbox) continue;
+    const uint32_t a = sq + ((q >> 3) & 1) * Kvc8Cfg::kBlockBytes + row * 128 + (q & 7) * 16;
+    const uint4 v = ld_shared_v4(a);
+    const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o4[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+      o4[k] = pack_f16x2(__uint_as_float(in[k] << 16), __uint_as_float(in[k] & 0xFFFF0000u));
+    st_shared_v4(a, o4[0], o4[1], o4[2], o4[3]);
   }
 }
 
 template <bool CAUSAL>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(Kvc8Cfg::kThreads, 1)
 attn_kvcache_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k8,
                         const __grid_constant__ CUtensorMap tm_v8, const KvcParams prm, const float v_descale) {
   using C = Kvc8Cfg;
@@ -129,9 +171,11 @@ attn_kvcache_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
   uint64_t* pv_done = p_full + 2;
   uint64_t* o_full = pv_done + 1;
   uint64_t* o_free = o_full + 1;
-  uint64_t* kb_full = o_free + 1;
-  uint64_t* vb_full = kb_full + 1;
-  uint64_t* drain = vb_full + 1;
+  uint64_t* kb_full = o_free + 1;          // the f16 K tile holds the next key tile
+  uint64_t* kb_free = kb_full + 1;         // the S product reading it has completed
+  uint64_t* vb_full = kb_free + 1;
+  uint64_t* vb_free = vb_full + 1;         // the PV product reading it has completed
+  uint64_t* drain = vb_free + 1;
   uint64_t* q_ready = drain + 1;           // the query tile has been converted to f16
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
@@ -144,7 +188,7 @@ attn_kvcache_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
     mbar_init(q_empty, 1);
     for (int s = 0; s < C::kSlots; ++s) {
       mbar_init(&ring_full[s], 1);
-      mbar_init(&ring_empty[s], 128);      // released by the widening threads
+      mbar_init(&ring_empty[s], C::kWidenWarps);   // one arrival per widening warp
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&s_full[t], 1);
@@ -153,14 +197,18 @@ attn_kvcache_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
     mbar_init(pv_done, 1);
     mbar_init(o_full, 1);
     mbar_init(o_free, 128);
-    mbar_init(kb_full, 128);
-    mbar_init(vb_full, 128);
+    mbar_init(kb_full, C::kWidenWarps);
+    mbar_init(kb_free, 1);
+    mbar_init(vb_full, C::kWidenWarps);
+    mbar_init(vb_free, 1);
     mbar_init(drain, 1);
-    mbar_init(q_ready, 128);
+    mbar_init(q_ready, C::kWidenWarps);
     *abort_flag = 0;
     fence_barrier_init();
   }
   if (warp < 4 && prm.qbox < 32) {
+    // Query rows that are padding in every lane quarter are never loaded:
+    // zero them once.
     const int r = threadIdx.x;
     if ((r & 31) >= prm.qbox)
       for (int blk = 0; blk < C::kNumBlk; ++blk)
@@ -243,7 +291,9 @@ attn_kvcache_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
         if (!(ok = mbar_wait(q_ready, uint32_t(qi & 1), abort_flag))) break;
         for (int jj = 0; jj <= I.nkv && ok; ++jj) {
           if (jj < I.nkv) {
-            // K_jj widened into the bf16 K tile (global tile count sc + jj)
+            // K_jj widened into the f16 K tile (global key tile count sc + jj).
+            // S buffer (sc + jj) & 1 was last read by the softmax of tile
+            // jj - 2, whose P was waited for before PV_{jj-2} was issued.
             if (!(ok = mbar_wait(kb_full, uint32_t((sc + jj) & 1), abort_flag))) break;
             tc_fence_after();
             const uint32_t dt = tmem + (((sc + jj) & 1) ? C::kColS1 : C::kColS0);
@@ -255,6 +305,7 @@ attn_kvcache_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
             }
             issued_any = true;
             mma_commit(&s_full[(sc + jj) & 1]);
+            mma_commit(kb_free);
             if (jj == I.nkv - 1) mma_commit(q_empty);
           }
           if (jj > 0) {
@@ -270,6 +321,7 @@ attn_kvcache_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
               mma_ts(tmem + C::kColO, at + kk * 8, smem_desc_sw128(sVb + kk * 2048, C::kBlockBytes, 1024), kIdescPV,
                      (pj > 0 || kk > 0) ? 1u : 0u);
             mma_commit(pj == I.nkv - 1 ? o_full : pv_done);
+            mma_commit(vb_free);
           }
         }
         sc += I.nkv;
@@ -282,28 +334,75 @@ attn_kvcache_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       }
     }
     __syncwarp();
-  } else {
-    // ------------------------------------------ widening + softmax (warps 0-3)
-    const int tid = threadIdx.x;              // 0..127: widening lane
-    const int r = lane;                       // packed row (replicated in every lane quarter)
-    const uint32_t lane_base = uint32_t(warp * 32) << 16;
-    const uint32_t tO = tmem + lane_base + C::kColO;
+  } else if (warp >= C::kWarpWiden0) {
+    // ------------------------------------------------ widening (8 warps)
+    // Per work item: the query tile to f16, then K_0, then K_{jj+1} and V_jj
+    // for every key tile jj (K first: S_{jj+1} waits for it, while PV_jj
+    // also waits for the softmax of tile jj).  kc / vc count the K / V tiles
+    // widened over all items; tile kc may overwrite the K tile once the S
+    // product of tile kc - 1 has completed (kb_free), likewise V with PV.
+    const int t = threadIdx.x - 32 * C::kWarpWiden0;
     const uint32_t sRing = smem_u32(smem + C::kOffRing);
     const uint32_t sKb = smem_u32(smem + C::kOffKb);
     const uint32_t sVb = smem_u32(smem + C::kOffVb);
-    const float c = prm.scale_log2;           // includes dk
-    int it = 0, sc = 0, pvb = 0, oi = 0;
+    int it = 0, kc = 0, vc = 0, qi = 0;
     bool ok = true;
 
-    // Widen ring item `item` into dst; the ring slot is then released.
-    auto widen = [&](int item, uint32_t dst, int zero_from) -> bool {
+    // Widen ring item `item` into dst and release its ring slot; then signal
+    // `full`.  Every thread fences its own shared-memory writes for the
+    // tensor core's (async) proxy before its warp's single arrival.
+    auto widen = [&](int item, uint32_t dst, int zero_from, uint64_t* full) -> bool {
       const int slot = item % C::kSlots;
       if (!mbar_wait_warp(&ring_full[slot], uint32_t((item / C::kSlots) & 1), abort_flag)) return false;
-      widen_tile(sRing + slot * C::kTile8Bytes, dst, tid, zero_from);
+      widen_tile(sRing + slot * C::kTile8Bytes, dst, t, zero_from);
       fence_proxy_async_smem();
-      mbar_arrive(&ring_empty[slot]);
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&ring_empty[slot]);
+        mbar_arrive(full);
+      }
       return true;
     };
+    auto widen_k = [&](int item) -> bool {
+      if (kc > 0 && !mbar_wait_warp(kb_free, uint32_t((kc - 1) & 1), abort_flag)) return false;
+      if (!widen(item, sKb, 128, kb_full)) return false;
+      ++kc;
+      return true;
+    };
+    auto widen_v = [&](int item, int zero_from) -> bool {
+      if (vc > 0 && !mbar_wait_warp(vb_free, uint32_t((vc - 1) & 1), abort_flag)) return false;
+      if (!widen(item, sVb, zero_from, vb_full)) return false;
+      ++vc;
+      return true;
+    };
+
+    for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
+      const KvcItem I = kvc_item(prm, w, CAUSAL);
+      if (I.nkv == 0) continue;
+      // The query tile: loaded after the previous item's last S product.
+      if (!(ok = mbar_wait_warp(q_full, uint32_t(qi & 1), abort_flag))) break;
+      convert_q_tile(smem_u32(smem + C::kOffQ), t, prm.qbox);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(q_ready);
+      ++qi;
+      if (!(ok = widen_k(it))) break;
+      for (int jj = 0; jj < I.nkv && ok; ++jj) {
+        if (jj + 1 < I.nkv && !(ok = widen_k(it + 2 * (jj + 1)))) break;
+        // rows past the valid length become zeros
+        ok = widen_v(it + 2 * jj + 1, I.L - 128 * (I.j_lo + jj));
+      }
+      it += 2 * I.nkv;
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------ softmax (warps 0-3)
+    const int r = lane;                       // packed row (replicated in every lane quarter)
+    const uint32_t lane_base = uint32_t(warp * 32) << 16;
+    const uint32_t tO = tmem + lane_base + C::kColO;
+    const float c = prm.scale_log2;           // includes dk
+    int sc = 0, pvb = 0, oi = 0;
+    bool ok = true;
 
     for (int w = blockIdx.x; w < n_items && ok; w += gridDim.x) {
       const KvcItem I = kvc_item(prm, w, CAUSAL);
@@ -314,48 +413,12 @@ attn_kvcache_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       float m_ref = -INFINITY;
       float l = 0.f;
 
-      // K_0 of this item: the previous item's S products have all completed
-      // (its o_full was waited in its epilogue), so the K tile is free.
-      if (I.nkv > 0) {
-        // This item's query tile (bf16, four copies) -> f16 in place: thread t
-        // converts row t of both column blocks.
-        if (!(ok = mbar_wait_warp(q_full, uint32_t(oi & 1), abort_flag))) break;
-        if ((tid & 31) < prm.qbox) {
-#pragma unroll
-          for (int blk = 0; blk < C::kNumBlk; ++blk)
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch) {
-              const uint32_t a = smem_u32(smem + C::kOffQ) + blk * C::kBlockBytes + tid * 128 + ch * 16;
-              const uint4 v = ld_shared_v4(a);
-              const uint32_t in[4] = {v.x, v.y, v.z, v.w};
-              uint32_t o4[4];
-#pragma unroll
-              for (int k = 0; k < 4; ++k)
-                o4[k] = pack_f16x2(__uint_as_float(in[k] << 16), __uint_as_float(in[k] & 0xFFFF0000u));
-              st_shared_v4(a, o4[0], o4[1], o4[2], o4[3]);
-            }
-        }
-        fence_proxy_async_smem();
-        mbar_arrive(q_ready);
-        if (!(ok = widen(it, sKb, 128))) break;
-        mbar_arrive(kb_full);
-      }
       for (int jj = 0; jj < I.nkv; ++jj) {
         const int j = I.j_lo + jj;
         const int sb = (sc + jj) & 1;
         const uint32_t tS = tmem + lane_base + (sb ? C::kColS1 : C::kColS0);
         if (!(ok = mbar_wait_warp(&s_full[sb], uint32_t(((sc + jj) >> 1) & 1), abort_flag))) break;
         tc_fence_after();
-        // S_jj has completed: the K tile may take K_{jj+1}.
-        if (jj + 1 < I.nkv) {
-          if (!(ok = widen(it + 2 * (jj + 1), sKb, 128))) break;
-          mbar_arrive(kb_full);
-        }
-        // V_jj once PV_{jj-1} has completed (the previous item's last PV was
-        // waited on through o_full); rows past the valid length become zeros.
-        if (jj > 0 && !(ok = mbar_wait_warp(pv_done, uint32_t((pvb + jj - 1) & 1), abort_flag))) break;
-        if (!(ok = widen(it + 2 * jj + 1, sVb, I.L - 128 * j))) break;
-        mbar_arrive(vb_full);
 
         float s[32];
         {
@@ -400,7 +463,11 @@ attn_kvcache_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
         tmem_st16(tmem + lane_base + (sb ? C::kColP1 : C::kColP0) + 16 * warp, pk);
         l += (sump[0] + sump[1]) + (sump[2] + sump[3]);
         if (__any_sync(0xffffffffu, rescale)) {
-          // PV_{jj-1} has completed (waited above before widening V_jj).
+          // O may only be rescaled once PV_{jj-1} has completed.  PV_jj needs
+          // this tile's P, so pv_done is at most one phase ahead of this wait
+          // and the phases skipped when no rescale happens are never misread.
+          if (!(ok = mbar_wait_warp(pv_done, uint32_t((pvb + jj - 1) & 1), abort_flag))) break;
+          tc_fence_after();
           const float a = rescale ? alpha : 1.f;
 #pragma unroll 1
           for (int cc = 0; cc < D / 32; ++cc) {
@@ -447,7 +514,6 @@ attn_kvcache_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_c
       if (I.nkv > 0) {
         tc_fence_before();
         mbar_arrive(o_free);
-        it += 2 * I.nkv;
         sc += I.nkv;
         pvb += I.nkv - 1;
         ++oi;

@@ -55,6 +55,7 @@ KERNEL_SOURCES = {
     "bwd_dkdv": ("attn_bwd.cuh", "sm100.cuh"),
     "bwd_dq": ("attn_bwd.cuh", "sm100.cuh"),
     "kvcache": ("attn_kvcache.cuh", "sm100.cuh"),
+    "kvcache_fp8": ("attn_kvcache_fp8.cuh", "attn_kvcache.cuh", "attn_fwd_fp8.cuh", "sm100.cuh"),
     "fp8": ("attn_fwd_fp8.cuh", "sm100.cuh"),
 }
 
@@ -395,6 +396,7 @@ def run_ours(args, rank, world, local_rank):
             gbs = alg_bytes / (t_us * 1e-6) / 1e9
             kvcache["fp8_cache"] = {"us": round(t_us, 2), "alg_bytes": alg_bytes, "gb_s": round(gbs, 1),
                                     "frac": round(gbs / hbm, 4), "calls": n_d,
+                                    "traffic": recorded_traffic("kvcache_fp8"),
                                     "cache": "K, V in E4M3 with per-tensor scales (1 byte per element)"}
             del kc8, vc8, wsd
         if not args.no_cpu_baseline and rank == 0:

@@ -703,9 +703,10 @@ ATTN_EXPORT int attn_fwd_kvcache_fp8(const void* Q, const void* K8, const void* 
   prm.splits = int(splits);
   prm.qbox = qbox;
   prm.n_items = int(n_items);
-  // The widened tiles hold 2^-8 times the E4M3 values (see the kernel): the
-  // factor goes into the exp2 argument and into the final 1/l.
-  prm.scale_log2 = float(double(scale) * double(k_descale) * 256.0 * 1.4426950408889634);
+  // The scores come from the E4M3 key codes themselves (the kernel divides
+  // out its per-row query scaling); the widened value tiles hold 2^-8 times
+  // the E4M3 values, so that factor goes into the final 1/l.
+  prm.scale_log2 = float(double(scale) * double(k_descale) * 1.4426950408889634);
   const float v_scale = float(double(v_descale) * 256.0);
   if (!std::isfinite(prm.scale_log2) || !(prm.scale_log2 > 0.f) || !std::isfinite(v_scale))
     return ATTN_ERR_INVALID_ARG;

@@ -158,16 +158,17 @@ int attn_fwd_kvcache(const void* Q, const void* K, const void* V, void* O, float
 /*
  * attn_fwd_kvcache with the cache stored in FP8: K8, V8 are uint8 [B][H_kv][Nk][128]
  * E4M3 codes with per-tensor dequantisation factors k_descale, v_descale (finite,
- * > 0); the result is attn_fwd_kvcache's on K = k_descale * K8, V = v_descale * V8
- * (every E4M3 value times 2^-8 is exactly an f16 value, so the cache is widened
- * on chip without rounding; the query tile is converted to f16 on chip, which is
- * exact for bf16 values of magnitude 2^-14 .. 65504 -- larger |Q| elements are
- * outside this entry point's domain, smaller ones round to f16's subnormal
- * grid, an absolute error below 2^-25 -- and the arithmetic is otherwise that
- * of the bf16 path: fp32 scores and statistics, P rounded to f16).  Reading half
- * the bytes per cached row is the point: decode reads the whole cache every
- * step.  Q, O bf16 and LSE, kv_lens, causal alignment, num_splits as in
- * attn_fwd_kvcache.  Restrictions: d = 128 and (H / H_kv) * Nq <= 32 (decode
+ * > 0); the result is attn_fwd_kvcache's on K = k_descale * K8, V = v_descale * V8.
+ * Reading half the bytes per cached row is the point: decode reads the whole
+ * cache every step.  Arithmetic: the scores are formed on the E4M3 key codes
+ * directly, with each query row scaled by a power of two (largest element in
+ * [128, 256)) and written as the sum of two E4M3 terms -- exact for elements of
+ * at least 2^-10 of the row's largest magnitude, within 2^-10 (scaled units)
+ * below that -- with fp32 accumulation; the value codes are widened to f16 on
+ * chip without rounding and P is rounded to f16.  Statistics are fp32 as in
+ * the bf16 path, whose tolerances apply.  Q elements must be finite.  Q, O bf16
+ * and LSE, kv_lens, causal alignment, num_splits as in attn_fwd_kvcache.
+ * Restrictions: d = 128 and (H / H_kv) * Nq <= 32 (decode
  * shapes), else ATTN_ERR_UNSUPPORTED.  The workspace is always needed, sized by
  * attn_fwd_kvcache_workspace_bytes() with the same arguments.
  */

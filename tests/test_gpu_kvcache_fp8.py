@@ -1,10 +1,14 @@
 """GPU parity for decode against an FP8 (E4M3) key/value cache
 (attn_fwd_kvcache_fp8): the oracle's cache forward on the dequantised cache.
-Every E4M3 value is a bf16 value, so the cache is widened exactly and the
-tolerances are those of the bf16 path (O 1e-2 plus the output's half ulp,
-LSE 1e-3).  Covers decode and a few query rows per head, shared key/value
-heads, both masks, per-batch lengths with non-finite codes past the length,
-and several split counts."""
+The kernel forms the scores on the E4M3 key codes with each query row split
+into two E4M3 terms (exact for elements of at least 2^-10 of the row's
+largest magnitude, within 2^-10 of it in the row's scaled units below that),
+widens the value codes exactly and rounds P to f16, so the tolerances are
+those of the bf16 path (O 1e-2 plus the output's half ulp, LSE 1e-3).
+Covers decode and a few query rows per head, shared key/value heads, both
+masks, per-batch lengths with non-finite codes past the length, several
+split counts, and query rows whose elements span many binades (the split's
+inexact range)."""
 
 import math
 
@@ -23,10 +27,14 @@ DEV = "cuda:0"
 E4M3_MAX = 448.0
 
 
-def _run(B, H, Hk, Nq, Nk, causal, seed, lens=None, splits=0, poison=False):
+def _run(B, H, Hk, Nq, Nk, causal, seed, lens=None, splits=0, poison=False, q_spread=0):
     d = 128
     g = torch.Generator("cpu").manual_seed(seed)
-    q = torch.randn((B, H, Nq, d), generator=g).to(torch.bfloat16)
+    q = torch.randn((B, H, Nq, d), generator=g)
+    if q_spread:
+        # per-element factors 2^-q_spread .. 2^3: most of a row far below its largest element
+        q = q * torch.exp2(torch.randint(-q_spread, 4, q.shape, generator=g).float())
+    q = q.to(torch.bfloat16)
     k = torch.randn((B, Hk, Nk, d), generator=g)
     v = torch.randn((B, Hk, Nk, d), generator=g)
     kd, vd = float(k.abs().max()) / E4M3_MAX, float(v.abs().max()) / E4M3_MAX
@@ -77,3 +85,8 @@ def test_fp8_cache_few_rows(Nq):
 
 def test_fp8_cache_lengths_with_nan_past_the_length():
     _run(5, 4, 2, 3, 1000, True, seed=1400, lens=[1000, 517, 128, 1, 0], poison=True)
+
+
+@pytest.mark.parametrize("spread", [12, 24])
+def test_fp8_cache_query_rows_spanning_many_binades(spread):
+    _run(2, 8, 2, 1, 1500, True, seed=1500 + spread, q_spread=spread)

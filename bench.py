@@ -398,6 +398,20 @@ def run_ours(args, rank, world, local_rank):
                                     "frac": round(gbs / hbm, 4), "calls": n_d,
                                     "traffic": recorded_traffic("kvcache_fp8"),
                                     "cache": "K, V in E4M3 with per-tensor scales (1 byte per element)"}
+            if not args.no_cpu_baseline and rank == 0:
+                # the oracle (as it stands) on batch entry 0 of the same decode
+                import numpy as np
+                from oracle import attn_oracle as orc
+                codes = lambda t: t[0:1].view(torch.uint8).cpu().numpy().reshape(-1, w.N, w.d)
+                Q64 = qd[0:1].float().cpu().numpy().astype(np.float64).reshape(-1, 1, w.d)
+                K8h, V8h = codes(kc8), codes(vc8)
+                t = time.perf_counter()
+                orc.attn_fwd_kvcache_fp8(Q64, K8h, V8h, kd8, vd8, scale, causal, 1, w.H, hk)
+                dt = time.perf_counter() - t
+                b1 = hk * w.N * w.d * 2
+                kvcache["fp8_cache"]["cpu_oracle"] = {
+                    "value": round(b1 / dt / 1e9, 3), "unit": "GB/s", "seconds": round(dt, 3), "kind": "oracle",
+                    "sample": "batch entry 0 of the E4M3-cache decode, fp64 numpy"}
             del kc8, vc8, wsd
         if not args.no_cpu_baseline and rank == 0:
             # the oracle (as it stands) on batch entry 0 of the full-cache decode

@@ -532,6 +532,33 @@ size_t kvc_workspace(const KvcShape& sh, int64_t splits, int64_t d) {
   return size_t(parts) * size_t(sh.total_rows) * size_t(d + 1) * sizeof(float);
 }
 
+// The split-KV merge, launched as a programmatic dependent of the cache
+// kernel just before it on the stream: its grid is set up while the cache
+// kernel's last CTAs run, and each block waits (griddepcontrol.wait) until the
+// cache kernel has completed and its partials are visible.
+template <int D>
+int launch_merge(const attn::KvcParams& prm, int parts, cudaStream_t st) {
+  int64_t blocks = prm.total_rows;                            // one 256-thread block per row
+  if (blocks > kNumSMs * 8) blocks = kNumSMs * 8;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(unsigned(blocks));
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const float* part_o = prm.part_o;
+  const float* part_lse = prm.part_lse;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, attn::attn_kvcache_merge_kernel<D>, part_o, part_lse, prm.o,
+                                           prm.lse, (long long)prm.total_rows, parts);
+  if (e != cudaSuccess)
+    return fail(ATTN_ERR_LAUNCH, "split-KV merge launch: %s (%lld)", cudaGetErrorString(e), (long long)e);
+  return launch_status();
+}
+
 template <int D, bool CAUSAL, bool SPLIT, bool REPL>
 int launch_kvc(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const attn::KvcParams& prm,
                int grid, cudaStream_t st) {
@@ -541,11 +568,7 @@ int launch_kvc(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
   kern<<<grid, attn::KvcCfg<D>::kThreads, smem, st>>>(q, k, v, prm);
   int s = launch_status();
   if (s != ATTN_OK || !SPLIT) return s;
-  int64_t blocks = prm.total_rows;                            // one 256-thread block per row
-  if (blocks > kNumSMs * 8) blocks = kNumSMs * 8;
-  attn::attn_kvcache_merge_kernel<D><<<int(blocks), 256, 0, st>>>(prm.part_o, prm.part_lse, prm.o, prm.lse,
-                                                                   prm.total_rows, prm.splits * (REPL ? 4 : 1));
-  return launch_status();
+  return launch_merge<D>(prm, prm.splits * (REPL ? 4 : 1), st);
 }
 
 template <int D, bool CAUSAL>
@@ -644,11 +667,7 @@ int launch_kvc8(const CUtensorMap& q, const CUtensorMap& k8, const CUtensorMap& 
   kern<<<grid, attn::Kvc8Cfg::kThreads, smem, st>>>(q, k8, v8, prm, v_descale);
   int s = launch_status();
   if (s != ATTN_OK) return s;
-  int64_t blocks = prm.total_rows;
-  if (blocks > kNumSMs * 8) blocks = kNumSMs * 8;
-  attn::attn_kvcache_merge_kernel<128><<<int(blocks), 256, 0, st>>>(prm.part_o, prm.part_lse, prm.o, prm.lse,
-                                                                     prm.total_rows, prm.splits * 4);
-  return launch_status();
+  return launch_merge<128>(prm, prm.splits * 4, st);
 }
 
 }  // namespace

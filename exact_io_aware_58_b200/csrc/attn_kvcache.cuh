@@ -594,6 +594,9 @@ attn_kvcache_merge_kernel(const float* __restrict__ part_o, const float* __restr
   __shared__ float s_sum[8];
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // Launched as a programmatic dependent of the cache kernel: wait until it
+  // has completed and its partials are visible (a no-op otherwise).
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   for (long long row = blockIdx.x; row < total_rows; row += gridDim.x) {
     float mx = -INFINITY;
     for (int s = threadIdx.x; s < parts; s += 256) {

@@ -30,7 +30,7 @@ ATTN_ERR_LAUNCH = -5
 ATTN_ERR_TIMEOUT = -6
 ATTN_ERR_DEVICE = -7
 
-EXPORTED = ("attn_fwd", "attn_fwd_gqa", "attn_fwd_blocksparse", "attn_bwd", "attn_bwd_gqa", "attn_bwd_blocksparse",
+EXPORTED = ("attn_fwd", "attn_fwd_f32out", "attn_fwd_gqa", "attn_fwd_blocksparse", "attn_bwd", "attn_bwd_gqa", "attn_bwd_blocksparse",
             "attn_bwd_workspace_bytes", "attn_fwd_fp8", "attn_fwd_kvcache", "attn_fwd_kvcache_fp8", "attn_fwd_kvcache_splits",
             "attn_fwd_kvcache_workspace_bytes",
             "attn_bwd_preprocess", "attn_bwd_dkdv",
@@ -64,6 +64,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib = ctypes.CDLL(path)
     i64, vp, f32, i32 = ctypes.c_int64, ctypes.c_void_p, ctypes.c_float, ctypes.c_int
     lib.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, f32, vp]
+    lib.attn_fwd_f32out.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, f32, vp]
+    lib.attn_fwd_f32out.restype = i32
     lib.attn_fwd.restype = i32
     lib.attn_fwd_gqa.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i32, f32, vp]
     lib.attn_fwd_gqa.restype = i32
@@ -156,6 +158,21 @@ def attn_fwd(Q, K, V, O, LSE, causal: bool, scale: float, stream=None) -> None:
                                  float(scale), _stream_handle(stream))
     if st != ATTN_OK:
         raise AttnError(st, "attn_fwd")
+
+
+def attn_fwd_f32out(Q, K, V, O, O32, LSE, causal: bool, scale: float, stream=None) -> None:
+    """attn_fwd that also writes O32 (fp32, same shape as O): the normalised rows before their bf16 rounding."""
+    _check_bhnd("Q", Q)
+    for n, t in (("K", K), ("V", V), ("O", O)):
+        _check_bhnd(n, t, Q.shape)
+    if not O32.is_cuda or O32.dtype != torch.float32 or tuple(O32.shape) != tuple(Q.shape) or not O32.is_contiguous():
+        raise ValueError("O32 must be a contiguous CUDA fp32 tensor shaped like Q")
+    _check_lse(LSE, Q.shape)
+    B, H, N, d = Q.shape
+    st = load_library().attn_fwd_f32out(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(O32), _ptr(LSE), B, H, N, d,
+                                        int(bool(causal)), float(scale), _stream_handle(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd_f32out")
 
 
 def _check_kv(name: str, t: torch.Tensor, q_shape):

@@ -126,10 +126,10 @@ int set_smem(const void* kern, int bytes) {
               (long long)bytes);
 }
 
-template <int D, bool CAUSAL, bool SPARSE>
+template <int D, bool CAUSAL, bool SPARSE, bool O32 = false>
 int launch_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const CUtensorMap& o,
                const attn::FwdParams& prm, int grid, cudaStream_t st) {
-  auto kern = attn::attn_fwd_kernel<D, CAUSAL, SPARSE>;
+  auto kern = attn::attn_fwd_kernel<D, CAUSAL, SPARSE, O32>;
   constexpr int smem = attn::FwdCfg<D>::kSmemBytes;
   if (set_smem(reinterpret_cast<const void*>(kern), smem) != ATTN_OK) return ATTN_ERR_LAUNCH;
   kern<<<grid, attn::FwdCfg<D>::kThreads, smem, st>>>(q, k, v, o, prm);
@@ -188,13 +188,15 @@ extern "C" {
 namespace {
 
 int fwd_impl(const void* Q, const void* K, const void* V, void* O, float* LSE, const uint8_t* mask, int64_t B,
-             int64_t H, int64_t H_kv, int64_t N, int64_t d, int causal, float scale, void* stream) {
+             int64_t H, int64_t H_kv, int64_t N, int64_t d, int causal, float scale, void* stream,
+             float* O32 = nullptr) {
   int s = check_sizes(B, H, N, d);
   if (s != ATTN_OK) return s;
   if ((s = check_heads(H, H_kv)) != ATTN_OK) return s;
   if ((s = check_scale(scale)) != ATTN_OK) return s;
   if (!Q || !K || !V || !O || !LSE) return ATTN_ERR_INVALID_ARG;
-  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE))
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE) ||
+      (O32 && !aligned16(O32)))
     return ATTN_ERR_MISALIGNED;
   const int64_t bh = B * H, bhkv = B * H_kv;
   CUtensorMap mq, mk, mv, mo;
@@ -211,10 +213,16 @@ int fwd_impl(const void* Q, const void* K, const void* V, void* O, float* LSE, c
   prm.scale_log2 = scale * 1.4426950408889634f;
   prm.mask = mask;
   prm.nt = int((N + 127) / 128);
+  prm.o32 = O32;
   const bool sparse = mask != nullptr;
   const int64_t grid = bh * prm.n_mblk;
   if (grid > INT32_MAX) return ATTN_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (O32)
+    return d == 128 ? (causal ? launch_fwd<128, true, false, true>(mq, mk, mv, mo, prm, int(grid), st)
+                              : launch_fwd<128, false, false, true>(mq, mk, mv, mo, prm, int(grid), st))
+                    : (causal ? launch_fwd<64, true, false, true>(mq, mk, mv, mo, prm, int(grid), st)
+                              : launch_fwd<64, false, false, true>(mq, mk, mv, mo, prm, int(grid), st));
   return ATTN_DISPATCH(launch_fwd, mq, mk, mv, mo, prm, int(grid), st);
 }
 
@@ -225,6 +233,12 @@ extern "C" {
 ATTN_EXPORT int attn_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int64_t B, int64_t H,
                          int64_t N, int64_t d, int causal, float scale, void* stream) {
   return fwd_impl(Q, K, V, O, LSE, nullptr, B, H, H, N, d, causal, scale, stream);
+}
+
+ATTN_EXPORT int attn_fwd_f32out(const void* Q, const void* K, const void* V, void* O, float* O32, float* LSE,
+                                int64_t B, int64_t H, int64_t N, int64_t d, int causal, float scale, void* stream) {
+  if (!O32) return ATTN_ERR_INVALID_ARG;
+  return fwd_impl(Q, K, V, O, LSE, nullptr, B, H, H, N, d, causal, scale, stream, O32);
 }
 
 ATTN_EXPORT int attn_fwd_gqa(const void* Q, const void* K, const void* V, void* O, float* LSE, int64_t B, int64_t H,

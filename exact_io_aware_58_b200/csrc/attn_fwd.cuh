@@ -43,6 +43,7 @@ struct FwdParams {
   float scale_log2;    // scale * log2(e)
   const uint8_t* mask; // block-sparse only: [B*H][nt][nt], 1 = query tile attends key tile
   int nt;              // ceil(N / 128)
+  float* o32;          // O32 instances only: [B*H][N][D] fp32 copy of the normalised O
 };
 
 // Key tiles selected for the (up to) two 128-row query tiles of a CTA: bit t of
@@ -87,7 +88,9 @@ struct FwdCfg {
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;   // + slack for 1024-byte alignment
 };
 
-template <int D, bool CAUSAL, bool SPARSE>
+// O32: also write the normalised rows in fp32 to prm.o32 (a separate
+// instance, so the bf16-only instances are compiled without it).
+template <int D, bool CAUSAL, bool SPARSE, bool O32 = false>
 __global__ void __launch_bounds__(320, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -400,6 +403,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           const uint32_t w3 = pack_bf16x2(__uint_as_float(o[8 * ch + 6]) * inv_l, __uint_as_float(o[8 * ch + 7]) * inv_l);
           const uint32_t chunk = (cc & 1) * 4 + ch;
           st_shared_v4(smem_u32(stage) + blk * C::kBlockBytes + sw128_offset(r, chunk), w0, w1, w2, w3);
+        }
+        if (O32 && i < n) {
+          // the same normalised row in fp32, before the bf16 rounding
+          float4* dst = reinterpret_cast<float4*>(prm.o32 + (size_t(bh) * size_t(n) + size_t(i)) * D + cc * 32);
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            dst[k] = make_float4(__uint_as_float(o[4 * k]) * inv_l, __uint_as_float(o[4 * k + 1]) * inv_l,
+                                 __uint_as_float(o[4 * k + 2]) * inv_l, __uint_as_float(o[4 * k + 3]) * inv_l);
         }
       }
       if (i < n)

@@ -71,6 +71,16 @@ int attn_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE,
              void* stream);
 
 /*
+ * attn_fwd that also writes O32: the normalised output rows in fp32 ([B][H][N][d],
+ * the same values before their rounding to bf16), for checking the forward
+ * against a tolerance finer than the bf16 output's own rounding.  O32 must be
+ * non-null (else ATTN_ERR_INVALID_ARG) and 16-byte aligned; it costs one extra
+ * write of 4 bytes per output element.  Everything else as attn_fwd.
+ */
+int attn_fwd_f32out(const void* Q, const void* K, const void* V, void* O, float* O32, float* LSE,
+                    int64_t B, int64_t H, int64_t N, int64_t d, int causal, float scale, void* stream);
+
+/*
  * Forward with shared key/value heads (grouped-query / multi-query attention):
  * H query heads, H_kv key/value heads, H % H_kv == 0; query head h of batch b
  * attends with key/value head h / (H / H_kv) of batch b.  Head sharing changes

@@ -81,6 +81,14 @@ def test_fwd_argument_errors(lib):
         assert _fwd(lib, ptrs=p) == attn.ATTN_ERR_MISALIGNED
 
 
+def test_f32out_argument_errors(lib):
+    # the fp32 output is required; the forward's own checks apply to the rest
+    assert lib.attn_fwd_f32out(A, A, A, A, None, A, 1, 2, 128, 64, 0, 0.125, None) == attn.ATTN_ERR_INVALID_ARG
+    assert lib.attn_fwd_f32out(A, A, A, A, MIS, A, 1, 2, 128, 64, 0, 0.125, None) == attn.ATTN_ERR_MISALIGNED
+    assert lib.attn_fwd_f32out(A, A, A, A, A, A, 1, 2, 128, 96, 0, 0.125, None) == attn.ATTN_ERR_UNSUPPORTED
+    assert lib.attn_fwd_f32out(A, A, A, A, A, A, 1, 2, 0, 64, 0, 0.125, None) == attn.ATTN_ERR_INVALID_ARG
+
+
 def test_gqa_argument_errors(lib):
     p = [A] * 5
     # H must be a multiple of H_kv, and 1 <= H_kv <= H

@@ -6,9 +6,9 @@ library is missing the import of a compute entry point fails loudly; there is
 no fallback path.
 
 Raw entry points keep the C names and argument order (``attn_fwd``,
-``attn_bwd``, ``attn_bwd_workspace_bytes``, ``attn_check_status``,
-``attn_status_string``); ``forward`` / ``backward`` allocate the outputs with
-torch and call them.
+``attn_bwd``, ``attn_bwd_deterministic``, ``attn_bwd_workspace_bytes``,
+``attn_check_status``, ``attn_status_string``); ``forward`` / ``backward``
+allocate the outputs with torch and call them.
 """
 
 from __future__ import annotations
@@ -30,9 +30,10 @@ ATTN_ERR_LAUNCH = -5
 ATTN_ERR_TIMEOUT = -6
 ATTN_ERR_DEVICE = -7
 
-EXPORTED = ("attn_fwd", "attn_fwd_f32out", "attn_fwd_gqa", "attn_fwd_blocksparse", "attn_bwd", "attn_bwd_gqa", "attn_bwd_blocksparse",
-            "attn_bwd_workspace_bytes", "attn_fwd_fp8", "attn_fwd_kvcache", "attn_fwd_kvcache_fp8", "attn_fwd_kvcache_splits",
-            "attn_fwd_kvcache_workspace_bytes",
+EXPORTED = ("attn_fwd", "attn_fwd_f32out", "attn_fwd_gqa", "attn_fwd_blocksparse", "attn_bwd", "attn_bwd_gqa",
+            "attn_bwd_blocksparse", "attn_bwd_deterministic", "attn_bwd_workspace_bytes",
+            "attn_bwd_deterministic_workspace_bytes", "attn_fwd_fp8", "attn_fwd_kvcache", "attn_fwd_kvcache_fp8",
+            "attn_fwd_kvcache_splits", "attn_fwd_kvcache_workspace_bytes",
             "attn_bwd_preprocess", "attn_bwd_dkdv",
             "attn_bwd_dq", "attn_bwd_static_workspace", "attn_check_status", "attn_last_error",
             "attn_selftest_wait_timeout",
@@ -91,6 +92,11 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.attn_fwd_kvcache_workspace_bytes.restype = ctypes.c_size_t
     lib.attn_bwd_workspace_bytes.argtypes = [i64, i64, i64, i64]
     lib.attn_bwd_workspace_bytes.restype = ctypes.c_size_t
+    lib.attn_bwd_deterministic_workspace_bytes.argtypes = [i64, i64, i64, i64]
+    lib.attn_bwd_deterministic_workspace_bytes.restype = ctypes.c_size_t
+    lib.attn_bwd_deterministic.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i32, f32, vp,
+                                           ctypes.c_size_t, vp]
+    lib.attn_bwd_deterministic.restype = i32
     lib.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, f32, vp,
                              ctypes.c_size_t, vp]
     lib.attn_bwd.restype = i32
@@ -134,9 +140,18 @@ def _ptr(t) -> ctypes.c_void_p:
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _check_device(name: str, t: torch.Tensor):
+    # The library launches on the calling thread's current device (and takes
+    # its workspace and default stream from there): every tensor must live on it.
+    if t.is_cuda and t.device.index != torch.cuda.current_device():
+        raise ValueError(f"{name} is on {t.device}, but the current CUDA device is "
+                         f"cuda:{torch.cuda.current_device()}; call under torch.cuda.device({t.device})")
+
+
 def _check_bhnd(name: str, t: torch.Tensor, shape=None):
     if not t.is_cuda or t.dtype != torch.bfloat16 or t.dim() != 4 or not t.is_contiguous():
         raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor of shape (B, H, N, d)")
+    _check_device(name, t)
     if shape is not None and tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
 
@@ -145,6 +160,7 @@ def _check_lse(t: torch.Tensor, shape):
     B, H, N, _ = shape
     if not t.is_cuda or t.dtype != torch.float32 or tuple(t.shape) != (B, H, N) or not t.is_contiguous():
         raise ValueError("LSE must be a contiguous CUDA float32 tensor of shape (B, H, N)")
+    _check_device("LSE", t)
 
 
 def attn_fwd(Q, K, V, O, LSE, causal: bool, scale: float, stream=None) -> None:
@@ -179,6 +195,7 @@ def _check_kv(name: str, t: torch.Tensor, q_shape):
     B, H, N, d = q_shape
     if not t.is_cuda or t.dtype != torch.bfloat16 or t.dim() != 4 or not t.is_contiguous():
         raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor of shape (B, H_kv, N, d)")
+    _check_device(name, t)
     Hk = t.shape[1]
     if t.shape[0] != B or t.shape[2] != N or t.shape[3] != d or Hk < 1 or H % Hk != 0:
         raise ValueError(f"{name} has shape {tuple(t.shape)}; expected (B, H_kv, N, d) with H % H_kv == 0")
@@ -358,21 +375,45 @@ def attn_bwd_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
     return int(load_library().attn_bwd_workspace_bytes(B, H, N, d))
 
 
+def attn_bwd_deterministic_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    return int(load_library().attn_bwd_deterministic_workspace_bytes(B, H, N, d))
+
+
 def attn_bwd(Q, K, V, O, dO, LSE, dQ, dK, dV, causal: bool, scale: float, workspace, stream=None) -> None:
-    """dQ, dK, dV <- backward of attention; all tensors preallocated on the device."""
+    """dQ, dK, dV <- backward of attention (one pass over the key tiles; dQ
+    summed in an fp32 workspace accumulator); all tensors preallocated on the device."""
     _check_bhnd("Q", Q)
     for n, t in (("K", K), ("V", V), ("O", O), ("dO", dO), ("dQ", dQ), ("dK", dK), ("dV", dV)):
         _check_bhnd(n, t, Q.shape)
     _check_lse(LSE, Q.shape)
-    if not workspace.is_cuda or not workspace.is_contiguous():
-        raise ValueError("workspace must be a contiguous CUDA tensor")
     B, H, N, d = Q.shape
-    ws_bytes = workspace.numel() * workspace.element_size()
+    wp, wb = _ws(workspace)
     st = load_library().attn_bwd(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(dO), _ptr(LSE), _ptr(dQ), _ptr(dK),
-                                 _ptr(dV), B, H, N, d, int(bool(causal)), float(scale), _ptr(workspace), ws_bytes,
+                                 _ptr(dV), B, H, N, d, int(bool(causal)), float(scale), wp, wb,
                                  _stream_handle(stream))
     if st != ATTN_OK:
         raise AttnError(st, "attn_bwd")
+
+
+def attn_bwd_deterministic(Q, K, V, O, dO, LSE, dQ, dK, dV, causal: bool, scale: float, workspace,
+                           stream=None) -> None:
+    """The bitwise-reproducible backward (separate dK/dV and dQ kernels); K, V,
+    dK, dV may have H_kv heads (B, H_kv, N, d)."""
+    _check_bhnd("Q", Q)
+    for n, t in (("O", O), ("dO", dO), ("dQ", dQ)):
+        _check_bhnd(n, t, Q.shape)
+    Hk = _check_kv("K", K, Q.shape)
+    for n, t in (("V", V), ("dK", dK), ("dV", dV)):
+        if _check_kv(n, t, Q.shape) != Hk:
+            raise ValueError(f"{n} must have the same number of heads as K")
+    _check_lse(LSE, Q.shape)
+    B, H, N, d = Q.shape
+    wp, wb = _ws(workspace)
+    st = load_library().attn_bwd_deterministic(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(dO), _ptr(LSE), _ptr(dQ),
+                                               _ptr(dK), _ptr(dV), B, H, Hk, N, d, int(bool(causal)), float(scale),
+                                               wp, wb, _stream_handle(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_bwd_deterministic")
 
 
 def attn_bwd_static_workspace(Q, K, V, O, dO, LSE, dQ, dK, dV, causal: bool, scale: float, stream=None) -> None:
@@ -394,6 +435,7 @@ def attn_bwd_static_workspace(Q, K, V, O, dO, LSE, dQ, dK, dV, causal: bool, sca
 def _ws(workspace):
     if not workspace.is_cuda or not workspace.is_contiguous():
         raise ValueError("workspace must be a contiguous CUDA tensor")
+    _check_device("workspace", workspace)
     return _ptr(workspace), workspace.numel() * workspace.element_size()
 
 
@@ -466,18 +508,22 @@ def forward(Q, K, V, causal: bool, scale: float | None = None, stream=None):
     return O, LSE
 
 
-def alloc_workspace(B: int, H: int, N: int, d: int, device) -> torch.Tensor:
-    nbytes = attn_bwd_workspace_bytes(B, H, N, d)
+def alloc_workspace(B: int, H: int, N: int, d: int, device, deterministic: bool = False) -> torch.Tensor:
+    nbytes = (attn_bwd_deterministic_workspace_bytes if deterministic else attn_bwd_workspace_bytes)(B, H, N, d)
     return torch.empty((max(nbytes, 16) + 15) // 16 * 4, dtype=torch.float32, device=device)
 
 
-def backward(Q, K, V, O, LSE, dO, causal: bool, scale: float | None = None, workspace=None, stream=None):
+def backward(Q, K, V, O, LSE, dO, causal: bool, scale: float | None = None, workspace=None, stream=None,
+             deterministic: bool = False):
+    """dQ, dK, dV; ``deterministic`` selects the bitwise-reproducible two-kernel path."""
     B, H, N, d = Q.shape
     scale = default_scale(d) if scale is None else scale
     if workspace is None:
-        workspace = alloc_workspace(B, H, N, d, Q.device)
+        workspace = alloc_workspace(B, H, N, d, Q.device, deterministic)
     dQ, dK, dV = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
-    if K.shape[1] == H:
+    if deterministic:
+        attn_bwd_deterministic(Q, K, V, O, dO, LSE, dQ, dK, dV, causal, scale, workspace, stream)
+    elif K.shape[1] == H:
         attn_bwd(Q, K, V, O, dO, LSE, dQ, dK, dV, causal, scale, workspace, stream)
     else:
         attn_bwd_gqa(Q, K, V, O, dO, LSE, dQ, dK, dV, causal, scale, workspace, stream)

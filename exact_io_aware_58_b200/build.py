@@ -16,7 +16,7 @@ ROOT = os.path.dirname(HERE)
 INCLUDE = os.path.join(ROOT, "include")
 LIB_PATH = os.path.join(HERE, "libattn.so")
 SOURCES = ["attn_api.cu"]
-DEPENDS = ["attn_api.cu", "attn_fwd.cuh", "attn_fwd_fp8.cuh", "attn_bwd.cuh", "attn_kvcache.cuh", "attn_kvcache_fp8.cuh", "sm100.cuh"]
+DEPENDS = ["attn_api.cu", "attn_fwd.cuh", "attn_fwd_fp8.cuh", "attn_bwd.cuh", "attn_bwd_fused.cuh", "attn_kvcache.cuh", "attn_kvcache_fp8.cuh", "sm100.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

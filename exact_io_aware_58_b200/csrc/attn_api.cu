@@ -9,6 +9,7 @@
 #include <algorithm>
 #include <cmath>
 #include <cstdint>
+#include <cstdarg>
 #include <cstdio>
 #include <mutex>
 
@@ -17,6 +18,7 @@
 
 #include "../../include/attn.h"
 #include "attn_bwd.cuh"
+#include "attn_bwd_fused.cuh"
 #include "attn_fwd.cuh"
 #include "attn_fwd_fp8.cuh"
 #include "attn_kvcache.cuh"
@@ -27,8 +29,11 @@ namespace {
 // Detail of the most recent failure on this host thread (attn_last_error).
 thread_local char g_last_error[256] = "";
 
-int fail(int status, const char* fmt, const char* a = "", long long b = 0) {
-  std::snprintf(g_last_error, sizeof(g_last_error), fmt, a, b);
+__attribute__((format(printf, 2, 3))) int fail(int status, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  std::vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
   return status;
 }
 
@@ -55,7 +60,7 @@ EncodeTiledFn encode_fn() {
 bool make_map(CUtensorMap* m, const void* base, int64_t bh, int64_t n, int64_t d, int box_rows = 128) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) {
-    fail(ATTN_ERR_LAUNCH, "%sdriver entry point cuTensorMapEncodeTiled unavailable%lld", "", 0);
+    fail(ATTN_ERR_LAUNCH, "driver entry point cuTensorMapEncodeTiled unavailable");
     return false;
   }
   const cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(n), cuuint64_t(bh)};
@@ -66,7 +71,7 @@ bool make_map(CUtensorMap* m, const void* base, int64_t bh, int64_t n, int64_t d
                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
-    fail(ATTN_ERR_LAUNCH, "%scuTensorMapEncodeTiled returned CUresult %lld", "", (long long)r);
+    fail(ATTN_ERR_LAUNCH, "cuTensorMapEncodeTiled returned CUresult %lld", (long long)r);
     return false;
   }
   return true;
@@ -77,7 +82,7 @@ bool make_map(CUtensorMap* m, const void* base, int64_t bh, int64_t n, int64_t d
 bool make_map_u8(CUtensorMap* m, const void* base, int64_t bh, int64_t n, int64_t d) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) {
-    fail(ATTN_ERR_LAUNCH, "%sdriver entry point cuTensorMapEncodeTiled unavailable%lld", "", 0);
+    fail(ATTN_ERR_LAUNCH, "driver entry point cuTensorMapEncodeTiled unavailable");
     return false;
   }
   const cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(n), cuuint64_t(bh)};
@@ -88,7 +93,30 @@ bool make_map_u8(CUtensorMap* m, const void* base, int64_t bh, int64_t n, int64_
                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
-    fail(ATTN_ERR_LAUNCH, "%scuTensorMapEncodeTiled returned CUresult %lld", "", (long long)r);
+    fail(ATTN_ERR_LAUNCH, "cuTensorMapEncodeTiled returned CUresult %lld", (long long)r);
+    return false;
+  }
+  return true;
+}
+
+// 3-D map over the fp32 dQ accumulator [B*H][Npad][d] (rows past N are never
+// touched: the map's extent is N, so reduce rows past N are dropped); box = 32
+// fp32 columns (128 bytes) x 128 rows x 1 head, 128-byte swizzle.
+bool make_map_f32_acc(CUtensorMap* m, const void* base, int64_t bh, int64_t n, int64_t npad, int64_t d) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) {
+    fail(ATTN_ERR_LAUNCH, "driver entry point cuTensorMapEncodeTiled unavailable");
+    return false;
+  }
+  const cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(n), cuuint64_t(bh)};
+  const cuuint64_t strides[2] = {cuuint64_t(d * 4), cuuint64_t(npad * d * 4)};
+  const cuuint32_t box[3] = {32, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    fail(ATTN_ERR_LAUNCH, "cuTensorMapEncodeTiled (fp32 accumulator) returned CUresult %lld", (long long)r);
     return false;
   }
   return true;
@@ -158,13 +186,39 @@ int launch_dq(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, 
 
 template <int D>
 int launch_bwd_pre(const void* O, const void* dO, const float* lse, float* ws_lse2, float* ws_d, int n, int npad,
-                   int64_t rows_pad, cudaStream_t st) {
+                   int64_t rows_pad, cudaStream_t st, float* dq_acc = nullptr) {
   constexpr int rows_per_block = 256 / (D / 8);
   int64_t blocks = (rows_pad + rows_per_block - 1) / rows_per_block;
   if (blocks > 148 * 32) blocks = 148 * 32;
-  attn::attn_bwd_pre_kernel<D><<<int(blocks), 256, 0, st>>>(
-      static_cast<const __nv_bfloat16*>(O), static_cast<const __nv_bfloat16*>(dO), lse, ws_lse2, ws_d, n, npad,
-      static_cast<long long>(rows_pad));
+  const __nv_bfloat16* o = static_cast<const __nv_bfloat16*>(O);
+  const __nv_bfloat16* d_o = static_cast<const __nv_bfloat16*>(dO);
+  if (dq_acc)
+    attn::attn_bwd_pre_kernel<D, true><<<int(blocks), 256, 0, st>>>(o, d_o, lse, ws_lse2, ws_d, n, npad,
+                                                                    static_cast<long long>(rows_pad), dq_acc);
+  else
+    attn::attn_bwd_pre_kernel<D, false><<<int(blocks), 256, 0, st>>>(o, d_o, lse, ws_lse2, ws_d, n, npad,
+                                                                     static_cast<long long>(rows_pad));
+  return launch_status();
+}
+
+template <int D, bool CAUSAL, bool SPARSE>
+int launch_fused(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const CUtensorMap& dO,
+                 const CUtensorMap& dk, const CUtensorMap& dv, const CUtensorMap& dqacc, const attn::BwdParams& prm,
+                 int grid, cudaStream_t st) {
+  using C = attn::FusedCfg<D>;
+  auto kern = attn::attn_bwd_fused_kernel<D, CAUSAL, SPARSE>;
+  if (set_smem(reinterpret_cast<const void*>(kern), C::kSmemBytes) != ATTN_OK) return ATTN_ERR_LAUNCH;
+  kern<<<grid, C::kThreads, C::kSmemBytes, st>>>(q, k, v, dO, dk, dv, dqacc, prm);
+  return launch_status();
+}
+
+template <int D>
+int launch_dq_convert(const float* dq_acc, void* dQ, int n, int npad, int64_t rows, float scale, cudaStream_t st) {
+  constexpr int rows_per_block = 256 / (D / 8);
+  int64_t blocks = (rows + rows_per_block - 1) / rows_per_block;
+  if (blocks > 148 * 32) blocks = 148 * 32;
+  attn::attn_bwd_dq_convert_kernel<D><<<int(blocks), 256, 0, st>>>(dq_acc, static_cast<__nv_bfloat16*>(dQ), n, npad,
+                                                                    static_cast<long long>(rows), scale);
   return launch_status();
 }
 
@@ -253,9 +307,14 @@ ATTN_EXPORT int attn_fwd_blocksparse(const void* Q, const void* K, const void* V
   return fwd_impl(Q, K, V, O, LSE, block_mask, B, H, H_kv, N, d, causal, scale, stream);
 }
 
-ATTN_EXPORT size_t attn_bwd_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d) {
+ATTN_EXPORT size_t attn_bwd_deterministic_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d) {
   if (check_sizes(B, H, N, d) != ATTN_OK) return 0;
   return size_t(2) * sizeof(float) * size_t(B * H) * size_t(npad_of(N));
+}
+
+ATTN_EXPORT size_t attn_bwd_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d) {
+  if (check_sizes(B, H, N, d) != ATTN_OK) return 0;
+  return size_t(B * H) * size_t(npad_of(N)) * sizeof(float) * size_t(2 + d);
 }
 
 }  // extern "C"
@@ -274,7 +333,7 @@ int bwd_common_checks(int64_t B, int64_t H, int64_t N, int64_t d, const void* wo
   if (s != ATTN_OK) return s;
   if (!workspace) return ATTN_ERR_INVALID_ARG;
   if (!aligned16(workspace)) return ATTN_ERR_MISALIGNED;
-  if (workspace_bytes < attn_bwd_workspace_bytes(B, H, N, d)) return ATTN_ERR_WORKSPACE;
+  if (workspace_bytes < attn_bwd_deterministic_workspace_bytes(B, H, N, d)) return ATTN_ERR_WORKSPACE;
   out->bh = B * H;
   out->npad = npad_of(N);
   out->ws_lse2 = static_cast<float*>(const_cast<void*>(workspace));
@@ -375,12 +434,55 @@ int bwd_impl(const void* Q, const void* K, const void* V, const void* O, const v
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(dO) || !aligned16(LSE) ||
       !aligned16(dQ) || !aligned16(dK) || !aligned16(dV) || !aligned16(workspace))
     return ATTN_ERR_MISALIGNED;
-  if (workspace_bytes < attn_bwd_workspace_bytes(B, H, N, d)) return ATTN_ERR_WORKSPACE;
+  if (workspace_bytes < attn_bwd_deterministic_workspace_bytes(B, H, N, d)) return ATTN_ERR_WORKSPACE;
   s = attn_bwd_preprocess(O, dO, LSE, B, H, N, d, workspace, workspace_bytes, stream);
   if (s != ATTN_OK) return s;
   s = dkdv_impl(Q, K, V, dO, dK, dV, mask, B, H, H_kv, N, d, causal, scale, workspace, workspace_bytes, stream);
   if (s != ATTN_OK) return s;
   return dq_impl(Q, K, V, dO, dQ, mask, B, H, H_kv, N, d, causal, scale, workspace, workspace_bytes, stream);
+}
+
+// The fused backward: bwd_pre (also clearing the fp32 dQ accumulator), one
+// pass over the key tiles for dK, dV and the dQ partials, and the dQ
+// conversion.  Workspace: [B*H][Npad] LSE*log2(e), [B*H][Npad] D, then the
+// accumulator [B*H][Npad][d] fp32.
+int fused_impl(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
+               void* dQ, void* dK, void* dV, const uint8_t* mask, int64_t B, int64_t H, int64_t H_kv, int64_t N,
+               int64_t d, int causal, float scale, void* workspace, size_t workspace_bytes, void* stream) {
+  int s = check_sizes(B, H, N, d);
+  if (s != ATTN_OK) return s;
+  if ((s = check_heads(H, H_kv)) != ATTN_OK) return s;
+  if ((s = check_scale(scale)) != ATTN_OK) return s;
+  if (!Q || !K || !V || !O || !dO || !LSE || !dQ || !dK || !dV || !workspace) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(dO) || !aligned16(LSE) ||
+      !aligned16(dQ) || !aligned16(dK) || !aligned16(dV) || !aligned16(workspace))
+    return ATTN_ERR_MISALIGNED;
+  if (workspace_bytes < attn_bwd_workspace_bytes(B, H, N, d)) return ATTN_ERR_WORKSPACE;
+  BwdSetup su;
+  su.bh = B * H;
+  su.npad = npad_of(N);
+  su.ws_lse2 = static_cast<float*>(workspace);
+  su.ws_d = su.ws_lse2 + su.bh * su.npad;
+  float* dq_acc = su.ws_d + su.bh * su.npad;
+  const int64_t bhkv = B * H_kv;
+  CUtensorMap mq, mk, mv, mdo, mdk, mdv, macc;
+  if (!make_map(&mq, Q, su.bh, N, d) || !make_map(&mk, K, bhkv, N, d) || !make_map(&mv, V, bhkv, N, d) ||
+      !make_map(&mdo, dO, su.bh, N, d) || !make_map(&mdk, dK, bhkv, N, d) || !make_map(&mdv, dV, bhkv, N, d) ||
+      !make_map_f32_acc(&macc, dq_acc, su.bh, N, su.npad, d))
+    return ATTN_ERR_LAUNCH;
+  const attn::BwdParams prm = bwd_params(su, N, H, H_kv, scale, mask);
+  const bool sparse = mask != nullptr;
+  const int grid = int(bhkv * prm.n_tiles);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  s = (d == 128) ? launch_bwd_pre<128>(O, dO, LSE, su.ws_lse2, su.ws_d, int(N), int(su.npad), su.bh * su.npad, st,
+                                       dq_acc)
+                 : launch_bwd_pre<64>(O, dO, LSE, su.ws_lse2, su.ws_d, int(N), int(su.npad), su.bh * su.npad, st,
+                                      dq_acc);
+  if (s != ATTN_OK) return s;
+  s = ATTN_DISPATCH(launch_fused, mq, mk, mv, mdo, mdk, mdv, macc, prm, grid, st);
+  if (s != ATTN_OK) return s;
+  return (d == 128) ? launch_dq_convert<128>(dq_acc, dQ, int(N), int(su.npad), su.bh * N, scale, st)
+                    : launch_dq_convert<64>(dq_acc, dQ, int(N), int(su.npad), su.bh * N, scale, st);
 }
 
 }  // namespace
@@ -402,16 +504,24 @@ ATTN_EXPORT int attn_bwd_dq(const void* Q, const void* K, const void* V, const v
 ATTN_EXPORT int attn_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
                          void* dQ, void* dK, void* dV, int64_t B, int64_t H, int64_t N, int64_t d, int causal,
                          float scale, void* workspace, size_t workspace_bytes, void* stream) {
-  return bwd_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, nullptr, B, H, H, N, d, causal, scale, workspace, workspace_bytes,
-                  stream);
+  return fused_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, nullptr, B, H, H, N, d, causal, scale, workspace,
+                    workspace_bytes, stream);
+}
+
+ATTN_EXPORT int attn_bwd_deterministic(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                                       const float* LSE, void* dQ, void* dK, void* dV, int64_t B, int64_t H,
+                                       int64_t H_kv, int64_t N, int64_t d, int causal, float scale, void* workspace,
+                                       size_t workspace_bytes, void* stream) {
+  return bwd_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, nullptr, B, H, H_kv, N, d, causal, scale, workspace,
+                  workspace_bytes, stream);
 }
 
 ATTN_EXPORT int attn_bwd_gqa(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                              const float* LSE, void* dQ, void* dK, void* dV, int64_t B, int64_t H, int64_t H_kv,
                              int64_t N, int64_t d, int causal, float scale, void* workspace, size_t workspace_bytes,
                              void* stream) {
-  return bwd_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, nullptr, B, H, H_kv, N, d, causal, scale, workspace,
-                  workspace_bytes, stream);
+  return fused_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, nullptr, B, H, H_kv, N, d, causal, scale, workspace,
+                    workspace_bytes, stream);
 }
 
 ATTN_EXPORT int attn_bwd_blocksparse(const void* Q, const void* K, const void* V, const void* O, const void* dO,
@@ -419,8 +529,8 @@ ATTN_EXPORT int attn_bwd_blocksparse(const void* Q, const void* K, const void* V
                                      int64_t B, int64_t H, int64_t H_kv, int64_t N, int64_t d, int causal,
                                      float scale, void* workspace, size_t workspace_bytes, void* stream) {
   if (!block_mask) return ATTN_ERR_INVALID_ARG;
-  return bwd_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, block_mask, B, H, H_kv, N, d, causal, scale, workspace,
-                  workspace_bytes, stream);
+  return fused_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, block_mask, B, H, H_kv, N, d, causal, scale, workspace,
+                    workspace_bytes, stream);
 }
 
 }  // extern "C"
@@ -451,7 +561,7 @@ ATTN_EXPORT int attn_fwd_fp8(const void* Q8, const void* K8, const void* V8, voi
                              float q_descale, float k_descale, float v_descale, void* stream) {
   int s = check_sizes(B, H, N, d);
   if (s != ATTN_OK) return s;
-  if (d != 128) return fail(ATTN_ERR_UNSUPPORTED, "%sattn_fwd_fp8 supports d = 128 only (got %lld)", "", (long long)d);
+  if (d != 128) return fail(ATTN_ERR_UNSUPPORTED, "attn_fwd_fp8 supports d = 128 only (got %lld)", (long long)d);
   if ((s = check_heads(H, H_kv)) != ATTN_OK) return s;
   if ((s = check_scale(scale)) != ATTN_OK) return s;
   if (!positive_finite(q_descale) || !positive_finite(k_descale) || !positive_finite(v_descale))
@@ -697,10 +807,10 @@ ATTN_EXPORT int attn_fwd_kvcache_fp8(const void* Q, const void* K8, const void* 
   int s = kvc_check(B, H, H_kv, Nq, Nk, d, &sh);
   if (s != ATTN_OK) return s;
   if (d != 128)
-    return fail(ATTN_ERR_UNSUPPORTED, "%sattn_fwd_kvcache_fp8 supports d = 128 only (got %lld)", "", (long long)d);
+    return fail(ATTN_ERR_UNSUPPORTED, "attn_fwd_kvcache_fp8 supports d = 128 only (got %lld)", (long long)d);
   if (!kvc_replicated(sh))
     return fail(ATTN_ERR_UNSUPPORTED,
-                "%sattn_fwd_kvcache_fp8 takes at most 32 query rows per key/value head ((H / H_kv) * Nq = %lld)", "",
+                "attn_fwd_kvcache_fp8 takes at most 32 query rows per key/value head ((H / H_kv) * Nq = %lld)",
                 (long long)sh.rows);
   if ((s = check_scale(scale)) != ATTN_OK) return s;
   if (!(std::isfinite(k_descale) && k_descale > 0.f) || !(std::isfinite(v_descale) && v_descale > 0.f))
@@ -760,36 +870,25 @@ ATTN_EXPORT int attn_fwd_kvcache_fp8(const void* Q, const void* K8, const void* 
 // and code that runs where cudaMalloc is not allowed or would synchronise the
 // device.  For them the workspace lives in this file-scope device array.  It
 // exists on every GPU that loads the library, from module load until process
-// exit.  Its address is looked up once per device (cudaGetSymbolAddress with
-// that device current) and cached.
+// exit.  It runs the deterministic path (pre, dK/dV, dQ), whose workspace is
+// only the two per-row vectors.  The array's device address belongs to the
+// module instance of the current context, so it is looked up on every call
+// (cudaGetSymbolAddress with the calling thread's current device and context;
+// the lookup allocates nothing) rather than cached by device number, which
+// would go stale after cudaDeviceReset or under another context.
 // ---------------------------------------------------------------------------
 namespace {
 
 static __device__ __align__(256) unsigned char g_static_workspace[ATTN_STATIC_WORKSPACE_BYTES];
 
-constexpr int kMaxDevices = 64;
-
-void* static_workspace_for_current_device() {
-  static std::mutex mu;
-  static void* ptr[kMaxDevices] = {};
-  int dev = -1;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
-    fail(ATTN_ERR_DEVICE, "cudaGetDevice: %s (%lld)", cudaGetErrorString(e), (long long)dev);
+void* static_workspace_for_current_context() {
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_static_workspace);
+  if (e != cudaSuccess || p == nullptr) {
+    fail(ATTN_ERR_DEVICE, "cudaGetSymbolAddress(static workspace): %s (%lld)", cudaGetErrorString(e), (long long)e);
     return nullptr;
   }
-  std::lock_guard<std::mutex> lock(mu);
-  if (ptr[dev] == nullptr) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_static_workspace);
-    if (e != cudaSuccess || p == nullptr) {
-      fail(ATTN_ERR_DEVICE, "cudaGetSymbolAddress(static workspace): %s (%lld)", cudaGetErrorString(e),
-           (long long)e);
-      return nullptr;
-    }
-    ptr[dev] = p;
-  }
-  return ptr[dev];
+  return p;
 }
 
 }  // namespace
@@ -802,15 +901,15 @@ ATTN_EXPORT int attn_bwd_static_workspace(const void* Q, const void* K, const vo
                                           void* stream) {
   const int s = check_sizes(B, H, N, d);
   if (s != ATTN_OK) return s;
-  const size_t need = attn_bwd_workspace_bytes(B, H, N, d);
+  const size_t need = attn_bwd_deterministic_workspace_bytes(B, H, N, d);
   if (need > size_t(ATTN_STATIC_WORKSPACE_BYTES))
     return fail(ATTN_ERR_WORKSPACE,
-                "%sattn_bwd_static_workspace: these sizes need %lld workspace bytes, more than the "
+                "attn_bwd_static_workspace: these sizes need %lld workspace bytes, more than the "
                 "ATTN_STATIC_WORKSPACE_BYTES the library holds; use attn_bwd with a caller workspace",
-                "", (long long)need);
-  void* ws = static_workspace_for_current_device();
+                (long long)need);
+  void* ws = static_workspace_for_current_context();
   if (ws == nullptr) return ATTN_ERR_DEVICE;
-  return attn_bwd(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, d, causal, scale, ws,
+  return bwd_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, nullptr, B, H, H, N, d, causal, scale, ws,
                   size_t(ATTN_STATIC_WORKSPACE_BYTES), stream);
 }
 
@@ -863,7 +962,7 @@ ATTN_EXPORT int attn_check_status(void* stream) {
     const unsigned int zero = 0;
     if (cudaMemcpyToSymbol(attn::g_attn_status, &zero, sizeof(zero)) != cudaSuccess) return ATTN_ERR_DEVICE;
     if (v & attn::kStatusLayout)
-      return fail(ATTN_ERR_DEVICE, "%sa kernel found its shared memory window misaligned and did no work%lld", "", 0);
+      return fail(ATTN_ERR_DEVICE, "a kernel found its shared memory window misaligned and did no work");
     return ATTN_ERR_TIMEOUT;
   }
   return ATTN_OK;

@@ -30,13 +30,14 @@ constexpr float kLog2e = 1.4426950408889634f;
 // ---------------------------------------------------------------------------
 // bwd_pre: D_i = sum_k dO_ik O_ik, lse2_i = LSE_i * log2(e); padding rows
 // (i >= N, up to Npad) get D = 0 and lse2 = +inf so that recomputed
-// probabilities of padding queries are exactly 0.
+// probabilities of padding queries are exactly 0.  ZERO (fused backward
+// only): also clears row i < N of the fp32 dQ accumulator [B*H][Npad][D].
 // ---------------------------------------------------------------------------
-template <int D>
+template <int D, bool ZERO = false>
 __global__ void __launch_bounds__(256)
 attn_bwd_pre_kernel(const __nv_bfloat16* __restrict__ O, const __nv_bfloat16* __restrict__ dO,
                     const float* __restrict__ lse, float* __restrict__ ws_lse2, float* __restrict__ ws_d,
-                    int n, int npad, long long rows_pad) {
+                    int n, int npad, long long rows_pad, float* __restrict__ dq_acc = nullptr) {
   constexpr int kTpr = D / 8;                 // threads per row, 16 bytes each
   constexpr int kRowsPerBlock = 256 / kTpr;
   const int sub = threadIdx.x % kTpr;
@@ -57,6 +58,11 @@ attn_bwd_pre_kernel(const __nv_bfloat16* __restrict__ O, const __nv_bfloat16* __
         const float2 fb = __bfloat1622float2(pb[k]);
         acc = fmaf(fa.x, fb.x, acc);
         acc = fmaf(fa.y, fb.y, acc);
+      }
+      if (ZERO) {
+        float4* z = reinterpret_cast<float4*>(dq_acc + (size_t(bh) * size_t(npad) + size_t(i)) * D + sub * 8);
+        z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+        z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
       }
     }
 #pragma unroll

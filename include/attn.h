@@ -201,11 +201,20 @@ size_t attn_fwd_kvcache_workspace_bytes(int64_t B, int64_t H, int64_t H_kv, int6
                                         int64_t num_splits);
 
 /*
- * Bytes of caller-provided device workspace that attn_bwd needs for these
- * sizes (two fp32 per-row vectors per head, each padded to a multiple of 128
- * rows).  Returns 0 for sizes that attn_bwd would reject.
+ * Bytes of caller-provided device workspace that attn_bwd (and attn_bwd_gqa,
+ * attn_bwd_blocksparse) need for these sizes: two fp32 per-row vectors per
+ * head plus an fp32 dQ accumulator of d values per row, each padded to a
+ * multiple of 128 rows: B*H*Npad*(2 + d)*4 bytes, Npad = N rounded up to 128.
+ * Returns 0 for sizes that attn_bwd would reject.
  */
 size_t attn_bwd_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d);
+
+/*
+ * Bytes of workspace that attn_bwd_deterministic and the three split steps
+ * (attn_bwd_preprocess, attn_bwd_dkdv, attn_bwd_dq) need: the two per-row
+ * vectors only, B*H*Npad*2*4 bytes.  0 for rejected sizes.
+ */
+size_t attn_bwd_deterministic_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d);
 
 /*
  * Backward pass by recomputation ("Attention and KV Compression", section
@@ -213,13 +222,20 @@ size_t attn_bwd_workspace_bytes(int64_t B, int64_t H, int64_t N, int64_t d);
  * attention fits in memory", section "Training backward").
  * Inputs: Q, K, V, the forward's O and LSE, and the output gradient dO.
  * Outputs: dQ, dK, dV (bf16, BHND).  Three kernels run on `stream`:
- *   (1) per row, D_i = sum_k dO_ik O_ik and LSE_i * log2(e), into `workspace`;
- *   (2) per 128-key tile, dK and dV (score tiles recomputed, 4 MMAs per tile pair);
- *   (3) per 128-query tile, dQ (score tiles recomputed, 3 MMAs per tile pair).
+ *   (1) per row, D_i = sum_k dO_ik O_ik and LSE_i * log2(e) into `workspace`,
+ *       and the fp32 dQ accumulator cleared;
+ *   (2) per 128-key tile, one pass over the query tiles: the score tiles are
+ *       recomputed once and give dK, dV (summed in tensor memory) and, from
+ *       the same dS, each query tile's dQ contribution, which is added into
+ *       the fp32 accumulator (5 MMAs per tile pair);
+ *   (3) dQ = scale * accumulator, rounded to bf16.
+ * The additions into the accumulator happen in an order that varies from run
+ * to run, so dQ can differ between runs in its last bits (dK and dV do not);
+ * attn_bwd_deterministic gives bitwise-reproducible results at a higher cost.
  * `workspace` (device, 16-byte aligned) must hold attn_bwd_workspace_bytes()
  * bytes, else ATTN_ERR_WORKSPACE; its layout after the call is
- * [B*H][Npad] fp32 LSE*log2(e) (padding rows +inf) followed by
- * [B*H][Npad] fp32 D (padding rows 0), Npad = N rounded up to 128.
+ * [B*H][Npad] fp32 LSE*log2(e) (padding rows +inf), [B*H][Npad] fp32 D
+ * (padding rows 0), then [B*H][Npad][d] fp32 dQ / scale (rows >= N unused).
  * Outputs must not alias inputs or the workspace.
  */
 int attn_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
@@ -228,12 +244,29 @@ int attn_bwd(const void* Q, const void* K, const void* V, const void* O, const v
              void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * The same backward with bitwise-reproducible results: (1) the per-row vectors
+ * as in attn_bwd, (2) per 128-key tile, dK and dV (score tiles recomputed, 4
+ * MMAs per tile pair), (3) per 128-query tile, dQ (score tiles recomputed
+ * again, 3 MMAs per tile pair) -- no accumulation across CTAs, so no order
+ * dependence, at the price of recomputing S and dP twice.  Shared key/value
+ * heads as in attn_bwd_gqa (H_kv = H for multi-head attention).  `workspace`
+ * must hold attn_bwd_deterministic_workspace_bytes() bytes (layout: the two
+ * per-row vectors of attn_bwd).  It is exactly attn_bwd_preprocess,
+ * attn_bwd_dkdv and attn_bwd_dq in this order (for H_kv = H).
+ */
+int attn_bwd_deterministic(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                           const float* LSE, void* dQ, void* dK, void* dV,
+                           int64_t B, int64_t H, int64_t H_kv, int64_t N, int64_t d, int causal, float scale,
+                           void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Backward with shared key/value heads (see attn_fwd_gqa for the layout).
  * dQ: [B][H][N][d]; dK, dV: [B][H_kv][N][d], each the sum over the H / H_kv
- * query heads that share the key/value head (the dK/dV kernel loops over
- * those query heads, so the sum is formed in tensor memory without atomics).
- * The workspace is sized by attn_bwd_workspace_bytes(B, H, N, d) (query heads).
- * attn_bwd is this call with H_kv = H.
+ * query heads that share the key/value head (the per-key-tile kernel loops
+ * over those query heads, so the sum is formed in tensor memory without
+ * atomics).  Kernels and workspace as attn_bwd, sized by
+ * attn_bwd_workspace_bytes(B, H, N, d) (query heads).  attn_bwd is this call
+ * with H_kv = H.
  */
 int attn_bwd_gqa(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                  const float* LSE, void* dQ, void* dK, void* dV,
@@ -241,11 +274,11 @@ int attn_bwd_gqa(const void* Q, const void* K, const void* V, const void* O, con
                  void* workspace, size_t workspace_bytes, void* stream);
 
 /*
- * Backward of attn_fwd_blocksparse (same block_mask, same layouts as
- * attn_bwd_gqa).  The dQ kernel visits only the key tiles a query tile
- * selected; the dK/dV kernel visits only the (query head, query tile) pairs
- * that selected its key tile.  Rows with LSE = -inf contribute nothing; key
- * tiles that no query tile selected get dK = dV = 0.
+ * Backward of attn_fwd_blocksparse (same block_mask, same layouts and
+ * workspace as attn_bwd_gqa).  The per-key-tile kernel visits only the
+ * (query head, query tile) pairs that selected its key tile.  Rows with
+ * LSE = -inf contribute nothing; key tiles that no query tile selected get
+ * dK = dV = 0, and query tiles that selected no key tile get dQ = 0.
  */
 int attn_bwd_blocksparse(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                          const float* LSE, const uint8_t* block_mask, void* dQ, void* dK, void* dV,
@@ -253,10 +286,12 @@ int attn_bwd_blocksparse(const void* Q, const void* K, const void* V, const void
                          void* workspace, size_t workspace_bytes, void* stream);
 
 /*
- * The three steps of attn_bwd, callable one at a time (same arguments and
- * rules as attn_bwd; attn_bwd is exactly these three calls in this order on
- * one stream).  Useful to time the steps separately or to run dK/dV and dQ on
- * different streams once the preprocess step has completed.
+ * The three steps of attn_bwd_deterministic, callable one at a time (same
+ * arguments and rules; attn_bwd_deterministic with H_kv = H is exactly these
+ * three calls in this order on one stream; the workspace is sized by
+ * attn_bwd_deterministic_workspace_bytes()).  Useful to time the steps
+ * separately or to run dK/dV and dQ on different streams once the preprocess
+ * step has completed.
  *
  * attn_bwd_preprocess: per row, D_i = sum_k dO_ik O_ik and LSE_i*log2(e)
  *   into `workspace` (layout as for attn_bwd).  D is the row term of the
@@ -281,9 +316,9 @@ int attn_bwd_dq(const void* Q, const void* K, const void* V, const void* dO, voi
 
 /*
  * Backward without any caller-provided memory: same computation, arguments
- * and results as attn_bwd, but the workspace is a fixed array that the
- * library owns in device memory.  (The pages have no counterpart: this is a
- * deployment convenience, not part of the method.)
+ * and results as attn_bwd_deterministic (H_kv = H), but the workspace is a
+ * fixed array that the library owns in device memory.  (The pages have no
+ * counterpart: this is a deployment convenience, not part of the method.)
  *
  * Who needs it: callers that cannot allocate device memory where they run
  * the backward -- e.g. code inside a runtime whose memory is owned by another
@@ -294,15 +329,17 @@ int attn_bwd_dq(const void* Q, const void* K, const void* V, const void* dO, voi
  * Limits and behaviour:
  *  - The array is ATTN_STATIC_WORKSPACE_BYTES (32 MiB) on every GPU that
  *    loads the library, held from module load until process exit.  Sizes
- *    whose attn_bwd_workspace_bytes() exceed it are rejected with
- *    ATTN_ERR_WORKSPACE before anything is launched (attn_last_error() says
- *    how many bytes they need).  32 MiB covers B*H*ceil(N/128)*128 up to 2^22
- *    rows, e.g. B=8, H=32, N=16384.
- *  - The first call on a device looks the array's device address up (with
- *    that device current) and caches it; make that first call before any
- *    stream capture.  The device used is the calling thread's current device.
+ *    whose attn_bwd_deterministic_workspace_bytes() exceed it are rejected
+ *    with ATTN_ERR_WORKSPACE before anything is launched (attn_last_error()
+ *    says how many bytes they need).  32 MiB covers B*H*ceil(N/128)*128 up
+ *    to 2^22 rows, e.g. B=8, H=32, N=16384.
+ *  - The array belongs to the library's module in the calling thread's
+ *    current CUDA context (on its current device); every call looks its
+ *    device address up there (cudaGetSymbolAddress, which allocates
+ *    nothing).  The first call in a context loads the module if it is not
+ *    loaded yet; make that first call before any stream capture.
  *  - It calls no cudaMalloc, cudaFree or other allocating routine.
- *  - Every call on a device shares the one array, and the array keeps the
+ *  - Every call in a context shares the one array, and the array keeps the
  *    last call's contents.  Nothing in it needs to start at zero: the
  *    preprocess step writes every workspace element a call reads before the
  *    other kernels read it.  Calls whose GPU work overlaps (e.g. on two

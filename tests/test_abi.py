@@ -46,13 +46,21 @@ def test_status_strings(lib):
 
 
 def test_workspace_bytes(lib):
-    # two fp32 vectors per head, rows padded to a multiple of 128
-    assert attn.attn_bwd_workspace_bytes(1, 2, 256, 64) == 2 * 4 * 2 * 256
-    assert attn.attn_bwd_workspace_bytes(8, 32, 16384, 128) == 2 * 4 * 256 * 16384
-    assert attn.attn_bwd_workspace_bytes(1, 8, 100000, 128) == 2 * 4 * 8 * 100096
-    assert attn.attn_bwd_workspace_bytes(1, 1, 1, 64) == 2 * 4 * 128
-    assert attn.attn_bwd_workspace_bytes(1, 1, 1, 96) == 0       # unsupported d
-    assert attn.attn_bwd_workspace_bytes(0, 1, 1, 64) == 0
+    # deterministic path: two fp32 vectors per head, rows padded to a multiple of 128
+    det = attn.attn_bwd_deterministic_workspace_bytes
+    assert det(1, 2, 256, 64) == 2 * 4 * 2 * 256
+    assert det(8, 32, 16384, 128) == 2 * 4 * 256 * 16384
+    assert det(1, 8, 100000, 128) == 2 * 4 * 8 * 100096
+    assert det(1, 1, 1, 64) == 2 * 4 * 128
+    assert det(1, 1, 1, 96) == 0       # unsupported d
+    assert det(0, 1, 1, 64) == 0
+    # fused path: the same vectors plus a d-wide fp32 dQ accumulator per padded row
+    ws = attn.attn_bwd_workspace_bytes
+    assert ws(1, 2, 256, 64) == (2 + 64) * 4 * 2 * 256
+    assert ws(8, 32, 16384, 128) == (2 + 128) * 4 * 256 * 16384
+    assert ws(1, 8, 100000, 128) == (2 + 128) * 4 * 8 * 100096
+    assert ws(1, 1, 1, 96) == 0
+    assert ws(0, 1, 1, 64) == 0
 
 
 # Fake, never-dereferenced device addresses: argument checks happen before any
@@ -109,6 +117,8 @@ def test_bwd_argument_errors(lib):
         return lib.attn_bwd(*p, 1, 1, 128, d, 1, 0.125, ws_ptr, ws_bytes, None)
 
     assert bwd(ws_bytes=ws - 4) == attn.ATTN_ERR_WORKSPACE
+    # the deterministic path's smaller workspace is not enough for the fused path
+    assert bwd(ws_bytes=attn.attn_bwd_deterministic_workspace_bytes(1, 1, 128, 64)) == attn.ATTN_ERR_WORKSPACE
     assert bwd(ws_ptr=None) == attn.ATTN_ERR_INVALID_ARG
     assert bwd(ws_ptr=MIS) == attn.ATTN_ERR_MISALIGNED
     assert bwd(d=32) == attn.ATTN_ERR_UNSUPPORTED
@@ -116,6 +126,31 @@ def test_bwd_argument_errors(lib):
         p = [A] * 9
         p[k] = MIS
         assert bwd(ptrs=p) == attn.ATTN_ERR_MISALIGNED
+
+
+def test_bwd_deterministic_argument_errors(lib):
+    ws = attn.attn_bwd_deterministic_workspace_bytes(1, 4, 128, 64)
+
+    def bwd(ptrs=None, ws_ptr=A, ws_bytes=ws, d=64, hk=4):
+        p = ptrs or [A] * 9
+        return lib.attn_bwd_deterministic(*p, 1, 4, hk, 128, d, 1, 0.125, ws_ptr, ws_bytes, None)
+
+    assert bwd(ws_bytes=ws - 4) == attn.ATTN_ERR_WORKSPACE
+    assert bwd(ws_ptr=None) == attn.ATTN_ERR_INVALID_ARG
+    assert bwd(ws_ptr=MIS) == attn.ATTN_ERR_MISALIGNED
+    assert bwd(d=96) == attn.ATTN_ERR_UNSUPPORTED
+    assert bwd(hk=3) == attn.ATTN_ERR_INVALID_ARG
+    for k in range(9):
+        p = [A] * 9
+        p[k] = MIS
+        assert bwd(ptrs=p) == attn.ATTN_ERR_MISALIGNED
+
+
+def test_error_detail_has_no_stray_text(lib):
+    # a rejected fp8 call records a formatted detail string
+    p = [A] * 5
+    assert lib.attn_fwd_fp8(*p, 1, 1, 1, 128, 64, 0, 0.125, 1.0, 1.0, 1.0, None) == attn.ATTN_ERR_UNSUPPORTED
+    assert attn.attn_last_error() == "attn_fwd_fp8 supports d = 128 only (got 64)"
 
 
 def test_python_binding_validates_tensors():

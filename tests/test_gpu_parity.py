@@ -22,7 +22,7 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
 
 
-def _run(inp, causal, scale, with_bwd):
+def _run(inp, causal, scale, with_bwd, deterministic=False):
     q, k, v = (inp[n].to(DEV) for n in ("Q", "K", "V"))
     for n in list(inp):
         inp[n] = inp[n].cpu()        # the oracle reads host copies of the same bf16 values
@@ -31,8 +31,8 @@ def _run(inp, causal, scale, with_bwd):
     if with_bwd:
         do = inp["dO"].to(DEV)
         B, H, N, d = q.shape
-        ws = attn.alloc_workspace(B, H, N, d, q.device)
-        dq, dk, dv = attn.backward(q, k, v, o, lse, do, causal, scale, workspace=ws)
+        ws = attn.alloc_workspace(B, H, N, d, q.device, deterministic)
+        dq, dk, dv = attn.backward(q, k, v, o, lse, do, causal, scale, workspace=ws, deterministic=deterministic)
         out.update(dQ=dq, dK=dk, dV=dv, ws=ws)
     assert attn.attn_check_status() == attn.ATTN_OK
     return out
@@ -57,13 +57,14 @@ def _check_full(inp, out, causal, scale, with_bwd, heads=None):
 # Small shapes: several tiles and ragged tails, both head dims, both masks
 # ---------------------------------------------------------------------------
 
+@pytest.mark.parametrize("path", ["fused", "deterministic"])
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("N", [1, 7, 64, 127, 128, 129, 255, 256, 300, 513])
-def test_small_shapes_fwd_bwd(N, d, causal):
+def test_small_shapes_fwd_bwd(N, d, causal, path):
     inp = make_inputs(1, 2, N, d, seed=1000 + N + d)
     scale = 1.0 / math.sqrt(d)
-    out = _run(inp, causal, scale, True)
+    out = _run(inp, causal, scale, True, deterministic=(path == "deterministic"))
     _check_full(inp, out, causal, scale, True)
 
 
@@ -83,16 +84,25 @@ def test_workspace_vectors_bwd_pre():
     D_ref = np.sum(O_ref * dO, axis=-1)
     assert np.abs(Dv[:, :N] - D_ref).max() <= 2e-2 * np.abs(D_ref).max()
     assert (Dv[:, N:] == 0).all()
+    # the fused backward's fp32 dQ accumulator follows the vectors: dQ / scale
+    acc = out["ws"].view(-1)[2 * B * H * npad: 2 * B * H * npad + B * H * npad * d]
+    acc = acc.view(B * H, npad, d)[:, :N].cpu()
+    dQ_ref, _, _ = orc.attn_bwd(Q, K, V, dO, scale, True)
+    assert np.abs(acc.numpy().astype(np.float64) * scale - dQ_ref).max() <= 2e-2 * np.abs(dQ_ref).max()
+    # dQ is that sum times scale in fp32, rounded to nearest bf16
+    want = (acc * torch.tensor(scale, dtype=torch.float32)).to(torch.bfloat16)
+    assert torch.equal(out["dQ"].view(B * H, N, d).cpu(), want)
 
 
 # ---------------------------------------------------------------------------
 # The five workloads
 # ---------------------------------------------------------------------------
 
-def test_tiny_fwd_bwd():
+@pytest.mark.parametrize("path", ["fused", "deterministic"])
+def test_tiny_fwd_bwd(path):
     w = WORKLOADS["tiny"]
     inp = workload_inputs(w)
-    out = _run(inp, False, w.scale, True)
+    out = _run(inp, False, w.scale, True, deterministic=(path == "deterministic"))
     _check_full(inp, out, False, w.scale, True)
 
 
@@ -104,10 +114,11 @@ def test_fwd_outliers_full(causal):
     _check_full(inp, out, causal, w.scale, False)
 
 
-def test_train_d64():
+@pytest.mark.parametrize("path", ["fused", "deterministic"])
+def test_train_d64(path):
     w = WORKLOADS["train_d64"]
     inp = workload_inputs(w)
-    out = _run(inp, True, w.scale, True)
+    out = _run(inp, True, w.scale, True, deterministic=(path == "deterministic"))
     # forward on every head, backward on 6 seeded heads
     Q, K, V = (f64(inp[n]) for n in ("Q", "K", "V"))
     O_ref, L_ref = orc.attn_fwd(Q, K, V, w.scale, True)
@@ -231,13 +242,29 @@ def test_status_and_argument_errors_on_gpu():
 # ---------------------------------------------------------------------------
 
 def test_results_are_bitwise_reproducible():
-    # no atomics anywhere: the forward and both backward kernels reduce in a
-    # fixed order, so two runs on the same inputs give identical bits
+    # deterministic path: no cross-CTA accumulation anywhere, so the forward
+    # and both backward kernels reduce in a fixed order and two runs on the
+    # same inputs give identical bits
     inp = make_inputs(1, 4, 700, 128, seed=77)
-    a = _run(dict(inp), True, 1 / math.sqrt(128), True)
-    b = _run(dict(inp), True, 1 / math.sqrt(128), True)
+    a = _run(dict(inp), True, 1 / math.sqrt(128), True, deterministic=True)
+    b = _run(dict(inp), True, 1 / math.sqrt(128), True, deterministic=True)
     for name in ("O", "LSE", "dQ", "dK", "dV"):
         assert torch.equal(a[name], b[name]), name
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_fused_dk_dv_match_deterministic_bitwise(d, causal):
+    # dK and dV come from the same bf16 P^T / dS^T tiles and the same MMA
+    # sequence in both paths; only dQ is summed across CTAs in the fused one
+    inp = make_inputs(2, 3, 600, d, seed=78 + d)
+    scale = 1 / math.sqrt(d)
+    a = _run(dict(inp), causal, scale, True, deterministic=False)
+    b = _run(dict(inp), causal, scale, True, deterministic=True)
+    assert torch.equal(a["dK"], b["dK"]) and torch.equal(a["dV"], b["dV"])
+    # dQ: the same sums in another order, within a few bf16 ulps
+    diff = (a["dQ"].float() - b["dQ"].float()).abs().max().item()
+    assert diff <= 2 ** -6 * b["dQ"].float().abs().max().item()
 
 
 @pytest.mark.parametrize("case", range(8))

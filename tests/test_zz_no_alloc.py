@@ -1,8 +1,10 @@
 """attn_bwd_static_workspace: the backward for callers that cannot allocate
 device memory (the workspace is the library's fixed device array instead of a
-caller buffer).  Checked through the C ABI against attn_bwd with a caller
-workspace, on two calls in a row with different sizes, so that the second call
-runs over whatever the first left in the shared array.
+caller buffer).  Checked through the C ABI against attn_bwd_deterministic with
+a caller workspace -- the same kernels, so the results must be bit for bit
+equal -- and, independently, against the fp64 oracle, on two calls in a row
+with different sizes, so that the second call runs over whatever the first
+left in the shared array.
 
 This file is collected last on purpose: it must pass both on its own in a
 fresh process and after every other test.
@@ -16,6 +18,7 @@ import torch
 
 from exact_io_aware_58_b200 import attn
 from exact_io_aware_58_b200.inputs import make_inputs
+from oracle import attn_oracle as orc
 
 from ._parity import assert_grad, f64
 
@@ -34,8 +37,8 @@ def _case(B, H, N, d, causal, seed):
     q, k, v, do = (inp[n].to(DEV) for n in ("Q", "K", "V", "dO"))
     scale = 1.0 / math.sqrt(d)
     o, lse = attn.forward(q, k, v, causal, scale)
-    # existing entry point, caller-allocated workspace
-    ref = attn.backward(q, k, v, o, lse, do, causal, scale)
+    # existing deterministic entry point, caller-allocated workspace
+    ref = attn.backward(q, k, v, o, lse, do, causal, scale, deterministic=True)
     # the fixed-workspace entry point, called through the C ABI
     dq, dk, dv = (torch.full_like(q, float("nan")) for _ in range(3))
     stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
@@ -44,11 +47,14 @@ def _case(B, H, N, d, causal, seed):
     assert st == attn.ATTN_OK, attn.attn_last_error()
     assert attn.attn_check_status() == attn.ATTN_OK
     for name, got, want in zip(("dQ", "dK", "dV"), (dq, dk, dv), ref):
-        assert_grad(f64(got), f64(want), name)
+        assert torch.equal(got, want), name
+    Q, K, V, dO = (f64(inp[n]) for n in ("Q", "K", "V", "dO"))
+    for name, got, want in zip(("dQ", "dK", "dV"), (dq, dk, dv), orc.attn_bwd(Q, K, V, dO, scale, causal)):
+        assert_grad(f64(got), want, name)
 
 
 def test_static_workspace_matches_caller_workspace_twice():
-    _case(2, 4, 1000, 128, True, seed=21)     # first call on this device: address set-up
+    _case(2, 4, 1000, 128, True, seed=21)     # first call in this context: address look-up
     _case(1, 3, 300, 64, False, seed=22)      # second call: smaller sizes over the stale array
 
 
@@ -59,4 +65,4 @@ def test_static_workspace_rejects_sizes_beyond_its_capacity():
     st = lib.attn_bwd_static_workspace(*([fake] * 9), 1, 1, 2**22 + 1, 128, 1, 0.1, None)
     assert st == attn.ATTN_ERR_WORKSPACE
     assert "ATTN_STATIC_WORKSPACE_BYTES" in attn.attn_last_error()
-    assert attn.attn_bwd_workspace_bytes(8, 32, 16384, 128) <= attn.ATTN_STATIC_WORKSPACE_BYTES
+    assert attn.attn_bwd_deterministic_workspace_bytes(8, 32, 16384, 128) <= attn.ATTN_STATIC_WORKSPACE_BYTES

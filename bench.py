@@ -4,17 +4,25 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
 A step is one pass of the whole hot path over one batch: attn_fwd, then the
-backward (attn_bwd_preprocess, attn_bwd_dkdv, attn_bwd_dq), on the long-batch
-workload B=8, H=32, N=16384, d=128, causal, bf16 (the configuration whose
-target is forward >= 60 % and forward+backward >= 45 % of dense BF16 peak).
-Inputs are 1 GiB per tensor (larger than the 126 MB L2), so no L2 flush is
-needed between steps.
+backward as attn_bwd runs it (attn_bwd_fused_preprocess,
+attn_bwd_fused_dkdvdq, attn_bwd_fused_dq_convert), on the long-batch workload
+B=8, H=32, N=16384, d=128, causal, bf16 (the configuration whose target is
+forward >= 60 % and forward+backward >= 45 % of dense BF16 peak).  Inputs are
+1 GiB per tensor (larger than the 126 MB L2), so no L2 flush is needed
+between steps.
 
 Metric: attention TFLOP/s of forward+backward, counted as 4 N^2 d per head for
 the forward (halved under the causal mask) and 2.5x that for the backward.
-Multi-GPU (torchrun, one rank per GPU): every rank runs its own batch of the
-same workload (weak scaling, no collective on the data path); ``value`` is the
-FLOPs of all ranks over the slowest rank's time.
+The other four workloads (tiny fwd+bwd, the outlier-row forward with both
+masks, the d = 64 training shape, the 100K-token causal forward) are measured
+in the same run under the key ``configs``; the deterministic backward, shared
+key/value heads, block-sparse selection, decode against a cache and FP8 have
+keys of their own.
+
+Multi-GPU: ``--gpus N`` starts N rank processes on this node (one GPU each)
+unless it is already running under a launcher that set WORLD_SIZE; every rank
+runs its own batch of the same workload (weak scaling, no collective on the
+data path); ``value`` is the FLOPs of all ranks over the slowest rank's time.
 
 ``--impl reference`` times the fp64 CPU oracle on a bounded sample (the exact
 causal prefix sub-problem of one head: its first rows/keys), on rank 0 only.
@@ -52,6 +60,8 @@ def load_peaks():
 KERNEL_SOURCES = {
     "attn_fwd": ("attn_fwd.cuh", "sm100.cuh"),
     "bwd_pre": ("attn_bwd.cuh", "sm100.cuh"),
+    "bwd_fused": ("attn_bwd_fused.cuh", "attn_bwd.cuh", "sm100.cuh"),
+    "bwd_dq_convert": ("attn_bwd_fused.cuh", "attn_bwd.cuh", "sm100.cuh"),
     "bwd_dkdv": ("attn_bwd.cuh", "sm100.cuh"),
     "bwd_dq": ("attn_bwd.cuh", "sm100.cuh"),
     "kvcache": ("attn_kvcache.cuh", "sm100.cuh"),
@@ -143,7 +153,7 @@ def run_ours(args, rank, world, local_rank):
 
     from exact_io_aware_58_b200 import attn
     from exact_io_aware_58_b200.inputs import WORKLOADS, workload_inputs
-    from exact_io_aware_58_b200.multi import aggregate_tflops, max_over_ranks, rank_seed
+    from exact_io_aware_58_b200.multi import CudaClock, aggregate_tflops, max_over_ranks, rank_seed, run_timed
 
     w = WORKLOADS[WORKLOAD]
     if args.batch or args.heads or args.seq:
@@ -155,6 +165,8 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     attn.load_library()
     stream = torch.cuda.current_stream()
+    clock = CudaClock(stream)
+    barrier = dist.barrier if world > 1 else None
 
     inp = workload_inputs(w, seed=rank_seed(1234, rank), device=dev)
     q, k, v, do = inp["Q"], inp["K"], inp["V"], inp["dO"]
@@ -164,63 +176,38 @@ def run_ours(args, rank, world, local_rank):
     ws = attn.alloc_workspace(w.B, w.H, w.N, w.d, dev)
     scale = w.scale
 
-    def step(ev=None):
-        if ev is not None:
-            ev[0].record(stream)
+    # One step = the forward and the three kernels of attn_bwd, each bracketed
+    # by CUDA events on the launching stream.
+    def step(mark):
         attn.attn_fwd(q, k, v, o, lse, causal, scale, stream)
-        if ev is not None:
-            ev[1].record(stream)
-        attn.attn_bwd_preprocess(o, do, lse, ws, stream)
-        if ev is not None:
-            ev[2].record(stream)
-        attn.attn_bwd_dkdv(q, k, v, do, dk, dv, causal, scale, ws, stream)
-        if ev is not None:
-            ev[3].record(stream)
-        attn.attn_bwd_dq(q, k, v, do, dq, causal, scale, ws, stream)
-        if ev is not None:
-            ev[4].record(stream)
+        mark()
+        attn.attn_bwd_fused_preprocess(o, do, lse, ws, stream)
+        mark()
+        attn.attn_bwd_fused_dkdvdq(q, k, v, do, dk, dv, causal, scale, ws, stream)
+        mark()
+        attn.attn_bwd_fused_dq_convert(dq, scale, ws, stream)
 
-    for _ in range(args.warmup):
-        step()
-    st = attn.attn_check_status(stream)
-    if st != attn.ATTN_OK:
-        raise RuntimeError(f"device status after warm-up: {attn.attn_status_string(st)}")
+    sampler = []
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(args.steps)]
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    clocks = ClockSampler(local_rank)
-    time.sleep(0.3)
-    t0.record(stream)
-    for s in range(args.steps):
-        step(evs[s])
-    t1.record(stream)
-    torch.cuda.synchronize()
-    clk = clocks.stop()
-    if world > 1:
-        dist.barrier()
+    def start_clock_sampler():
+        sampler.append(ClockSampler(local_rank))
+        time.sleep(0.3)
+
+    total_ms, seg = run_timed(step, args.steps, args.warmup, clock, barrier, n_segments=4,
+                              on_timed_start=start_clock_sampler)
+    clk = sampler[0].stop()
     st = attn.attn_check_status(stream)
     if st != attn.ATTN_OK:
         raise RuntimeError(f"device status after timed region: {attn.attn_status_string(st)}")
 
-    total_ms = t0.elapsed_time(t1)
-    per_kernel = {"attn_fwd": 0.0, "bwd_pre": 0.0, "bwd_dkdv": 0.0, "bwd_dq": 0.0}
-    for e in evs:
-        per_kernel["attn_fwd"] += e[0].elapsed_time(e[1])
-        per_kernel["bwd_pre"] += e[1].elapsed_time(e[2])
-        per_kernel["bwd_dkdv"] += e[2].elapsed_time(e[3])
-        per_kernel["bwd_dq"] += e[3].elapsed_time(e[4])
-    per_kernel = {kname: t / args.steps for kname, t in per_kernel.items()}
-    t_fwd = per_kernel["attn_fwd"]
-    t_bwd = per_kernel["bwd_pre"] + per_kernel["bwd_dkdv"] + per_kernel["bwd_dq"]
-
+    names = ["attn_fwd", "bwd_pre", "bwd_fused", "bwd_dq_convert"]
     # max over ranks of the timed-region duration and of the per-kernel means
-    vals = max_over_ranks([total_ms, t_fwd, t_bwd] + list(per_kernel.values()), device=dev)
-    total_ms, t_fwd, t_bwd = vals[0], vals[1], vals[2]
-    per_kernel = dict(zip(per_kernel.keys(), vals[3:]))
+    vals = max_over_ranks([total_ms] + seg, device=dev)
+    total_ms = vals[0]
+    per_kernel = dict(zip(names, vals[1:]))
     ms_per_step = total_ms / args.steps
+    t_fwd = per_kernel["attn_fwd"]
+    t_bwd = per_kernel["bwd_pre"] + per_kernel["bwd_fused"] + per_kernel["bwd_dq_convert"]
 
     f_fwd = flops_fwd_per_rank(w)
     value = aggregate_tflops(3.5 * f_fwd, world, ms_per_step)
@@ -231,18 +218,44 @@ def run_ours(args, rank, world, local_rank):
     burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
     sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
 
-    # roofline of the dominant kernel: algorithmic FLOPs per launch (GEMMs on
-    # the causal half of the score matrix: fwd 2, dK/dV 4, dQ 3) over its
-    # CUDA-event mean duration.
-    alg = {"attn_fwd": f_fwd, "bwd_dkdv": 2.0 * f_fwd, "bwd_dq": 1.5 * f_fwd}
+    # Roofline of the dominant kernel: algorithmic FLOPs per launch (GEMMs on
+    # the causal half of the score matrix: forward 2; fused backward 5 = the
+    # 2.5x backward count) over its CUDA-event mean duration, against the
+    # measured burst peak (the sustained figure was measured at a lower SM
+    # clock than these kernels run at, so it would overstate the fraction; it
+    # is reported beside it).
+    alg = {"attn_fwd": f_fwd, "bwd_fused": 2.5 * f_fwd}
     dom = max(alg, key=lambda kname: per_kernel[kname])
     achieved = alg[dom] / (per_kernel[dom] * 1e-3) / 1e12
-    roofline = {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 1), "peak": sustained,
-                "peak_kind": f"bf16_tflops_sustained ({peaks_src})", "unit": "TFLOP/s",
-                "frac": round(achieved / sustained, 4), "frac_of_burst": round(achieved / burst, 4),
-                "traffic": recorded_traffic(dom)}
+    roofline = {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 1), "peak": burst,
+                "peak_kind": f"bf16_tflops burst ({peaks_src})", "unit": "TFLOP/s",
+                "frac": round(achieved / burst, 4), "frac_of_sustained": round(achieved / sustained, 4),
+                "frac_of_datasheet_2250": round(achieved / 2250.0, 4),
+                "alg_flops_per_launch": alg[dom], "traffic": recorded_traffic(dom)}
 
     peak_mem = torch.cuda.max_memory_allocated(dev)
+
+    # --------------------------------------- deterministic backward (3 kernels)
+    det = None
+    if not args.no_det:
+        wsd = attn.alloc_workspace(w.B, w.H, w.N, w.d, dev, deterministic=True)
+
+        def det_step(mark):
+            attn.attn_bwd_preprocess(o, do, lse, wsd, stream)
+            mark()
+            attn.attn_bwd_dkdv(q, k, v, do, dk, dv, causal, scale, wsd, stream)
+            mark()
+            attn.attn_bwd_dq(q, k, v, do, dq, causal, scale, wsd, stream)
+
+        n_d = max(3, min(args.steps, 5))
+        _, dseg = run_timed(det_step, n_d, args.warmup, clock, barrier, n_segments=3)
+        assert attn.attn_check_status(stream) == attn.ATTN_OK
+        dseg = max_over_ranks(dseg, device=dev)
+        det = {"kernel_ms": {"bwd_pre": round(dseg[0], 3), "bwd_dkdv": round(dseg[1], 3), "bwd_dq": round(dseg[2], 3)},
+               "bwd_tflops": round(aggregate_tflops(2.5 * f_fwd, world, sum(dseg)), 2),
+               "fwdbwd_tflops": round(aggregate_tflops(3.5 * f_fwd, world, t_fwd + sum(dseg)), 2),
+               "steps": n_d, "note": "bitwise-reproducible path (separate dK/dV and dQ kernels, 7 GEMMs per tile pair)"}
+        del wsd
 
     # ------------------------------------------------- shared key/value heads
     gqa = None
@@ -474,6 +487,11 @@ def run_ours(args, rank, world, local_rank):
                                  "sample": f"causal prefix of head (0,0): first {rows} rows, forward, fp64 numpy"}
         del qf, kf, vf
 
+    # ------------------------------------------- the other four workloads
+    configs = None
+    if not args.no_configs:
+        configs = measure_configs(args, rank, world, dev, stream, clock, barrier, burst, peaks_src)
+
     # ---------------------------------------------------------------- e2e
     # Through host buffers: every step copies its inputs Q, K, V, dO from
     # pinned host memory to the device and its results O, LSE, dQ, dK, dV back.
@@ -546,6 +564,7 @@ def run_ours(args, rank, world, local_rank):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline_sample(q[0, 0], k[0, 0], v[0, 0], do[0, 0], w, rows=args.cpu_rows)
 
+    assert world == args.gpus
     line = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -576,11 +595,13 @@ def run_ours(args, rank, world, local_rank):
         },
         "kernel_ms": {kname: round(t, 3) for kname, t in per_kernel.items()},
         "roofline": roofline,
+        "bwd_deterministic": det,
+        "configs": configs,
         "gqa": gqa,
         "block_sparse": sparse,
         "kvcache": kvcache,
         "fp8": fp8,
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": 4 * args.steps,      # attn_fwd + the three kernels of attn_bwd per timed step
         "clocks": clk,
         "e2e": e2e,
         "cpu_baseline": cpu,
@@ -588,6 +609,115 @@ def run_ours(args, rank, world, local_rank):
         "naive_score_bytes_per_layer": 2 * w.N * w.N * w.B * w.H,
     }
     return line
+
+
+def _oracle_threads():
+    threads = os.cpu_count()
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([int(i.get("num_threads", 1)) for i in threadpool_info()] + [1])
+    except Exception:
+        pass
+    return threads
+
+
+def measure_configs(args, rank, world, dev, stream, clock, barrier, burst, peaks_src):
+    """TFLOP/s, peak device memory and a bounded oracle sample for the tiny,
+    outlier-row, d = 64 training and 100K-token workloads (the long-batch one
+    is the main step).  Each timed step runs ``reps`` back-to-back calls so
+    that the short ones are not timed as host launch gaps."""
+    import numpy as np
+    import torch
+
+    from exact_io_aware_58_b200 import attn
+    from exact_io_aware_58_b200.inputs import WORKLOADS, sample_rows, workload_inputs
+    from exact_io_aware_58_b200.multi import aggregate_tflops, max_over_ranks, rank_seed, run_timed
+
+    plan = [("tiny", 100), ("fwd_outliers", 10), ("train_d64", 10), ("long_context", 1)]
+    out = {}
+    for name, reps in plan:
+        w = WORKLOADS[name]
+        torch.cuda.synchronize()
+        base = torch.cuda.memory_allocated(dev)
+        torch.cuda.reset_peak_memory_stats(dev)
+        inp = workload_inputs(w, seed=rank_seed(0, rank), device=dev)
+        q, k, v = inp["Q"], inp["K"], inp["V"]
+        do = inp.get("dO")
+        o = torch.empty_like(q)
+        lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+        with_bwd = do is not None
+        if with_bwd:
+            dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+            ws = attn.alloc_workspace(w.B, w.H, w.N, w.d, dev)
+        ent = {"shape": {"B": w.B, "H": w.H, "N": w.N, "d": w.d}, "note": w.note, "reps_per_step": reps}
+        for causal in w.causal:
+            key = "causal" if causal else "non_causal"
+
+            def step(mark):
+                for _ in range(reps):
+                    attn.attn_fwd(q, k, v, o, lse, causal, w.scale, stream)
+                if with_bwd:
+                    mark()
+                    for _ in range(reps):
+                        attn.attn_bwd(q, k, v, o, do, lse, dq, dk, dv, causal, w.scale, ws, stream)
+
+            n = max(3, min(args.steps, 10))
+            _, seg = run_timed(step, n, args.warmup, clock, barrier, n_segments=2 if with_bwd else 1)
+            assert attn.attn_check_status(stream) == attn.ATTN_OK
+            seg = [x / reps for x in max_over_ranks(seg, device=dev)]
+            f = w.flops_fwd(causal)
+            r = {"ms_fwd": round(seg[0], 5), "fwd_tflops": round(aggregate_tflops(f, world, seg[0]), 2),
+                 "fwd_of_burst": round(aggregate_tflops(f, world, seg[0]) / world / burst, 4)}
+            if with_bwd:
+                r.update({"ms_bwd": round(seg[1], 5),
+                          "fwdbwd_tflops": round(aggregate_tflops(3.5 * f, world, seg[0] + seg[1]), 2),
+                          "fwdbwd_of_burst": round(aggregate_tflops(3.5 * f, world, seg[0] + seg[1]) / world / burst,
+                                                   4)})
+            ent[key] = r
+        torch.cuda.synchronize()
+        ent["peak_mem_gib"] = round((torch.cuda.max_memory_allocated(dev) - base) / 2**30, 4)
+        ent["naive_score_bytes"] = 2 * w.N * w.N * w.B * w.H
+        ent["peaks"] = peaks_src
+
+        if rank == 0 and world >= 1 and not args.no_cpu_baseline:
+            # the oracle as it stands, on a bounded sample of the same inputs
+            from oracle import attn_oracle as orc
+            h64 = lambda t: t.float().cpu().numpy().astype(np.float64)
+            causal = w.causal[-1]
+            if name == "long_context":
+                rows = sample_rows(w.B, w.H, w.N, w.check_rows, 0).numpy()
+                bh, ii = rows // w.N, rows % w.N
+                secs, fl = 0.0, 0.0
+                for h in np.unique(bh):
+                    sel = ii[bh == h]
+                    qh, kh, vh = (h64(t.view(-1, w.N, w.d)[h]) for t in (q, k, v))
+                    t0 = time.perf_counter()
+                    orc.attn_fwd_rows(qh, kh, vh, w.scale, True, sel)
+                    secs += time.perf_counter() - t0
+                    fl += float(np.sum(4.0 * (sel + 1) * w.d))
+                sample = f"{len(rows)} sampled query rows (all heads), causal forward; full job x{w.N * w.H / len(rows):.0f}"
+                full = secs * w.N * w.H / len(rows)
+            else:
+                heads = 2 if name == "tiny" else 1
+                qh, kh, vh = (h64(t.view(-1, w.N, w.d)[:heads]) for t in (q, k, v))
+                t0 = time.perf_counter()
+                orc.attn_fwd(qh, kh, vh, w.scale, causal)
+                if with_bwd:
+                    orc.attn_bwd(qh, kh, vh, h64(do.view(-1, w.N, w.d)[:heads]), w.scale, causal)
+                secs = time.perf_counter() - t0
+                fl = (3.5 if with_bwd else 1.0) * w.flops_fwd(causal) * heads / (w.B * w.H)
+                sample = (f"{heads} of {w.B * w.H} heads, {'fwd+bwd' if with_bwd else 'fwd'}, "
+                          f"{'causal' if causal else 'non-causal'}")
+                full = secs * (w.B * w.H) / heads
+            ent["cpu_oracle"] = {"value": round(fl / secs / 1e12, 6), "unit": "TFLOP/s", "seconds": round(secs, 3),
+                                 "full_job_seconds_extrapolated": round(full, 1), "cores": _oracle_threads(),
+                                 "kind": "oracle", "sample": sample + ", fp64 numpy"}
+        out[name] = ent
+        del inp, q, k, v, o, lse, do
+        if with_bwd:
+            del dq, dk, dv, ws
+        torch.cuda.empty_cache()
+    return out
 
 
 def cpu_baseline_sample(q, k, v, do, w, rows):
@@ -603,12 +733,7 @@ def cpu_baseline_sample(q, k, v, do, w, rows):
         return t[:rows].float().cpu().numpy().astype(np.float64)[None]
 
     Q, K, V, dO = host(q), host(k), host(v), host(do)
-    threads = os.cpu_count()
-    try:
-        from threadpoolctl import threadpool_info
-        threads = max([int(i.get("num_threads", 1)) for i in threadpool_info()] + [1])
-    except Exception:
-        pass
+    threads = _oracle_threads()
     t = time.perf_counter()
     orc.attn_fwd(Q, K, V, w.scale, True)
     orc.attn_bwd(Q, K, V, dO, w.scale, True)
@@ -661,6 +786,28 @@ def run_reference(args):
     }
 
 
+def spawn_ranks(n: int) -> int:
+    """Run this script as ``n`` rank processes on this node, one GPU each, and
+    return the first non-zero exit code (0 if all succeed).  Rank 0 prints the
+    JSON line."""
+    import socket
+
+    import torch
+
+    from exact_io_aware_58_b200.multi import rank_envs
+
+    visible = torch.cuda.device_count()
+    if visible < n:
+        raise SystemExit(f"bench.py: --gpus {n} but only {visible} CUDA device(s) are visible")
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    procs = [subprocess.Popen([sys.executable, os.path.abspath(__file__), *sys.argv[1:]], env=env)
+             for env in rank_envs(n, port)]
+    rcs = [p.wait() for p in procs]
+    return next((rc for rc in rcs if rc != 0), 0)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -674,6 +821,8 @@ def main():
     ap.add_argument("--no-fp8", action="store_true", help="skip the FP8 forward measurement")
     ap.add_argument("--gqa-kv-heads", type=int, default=8)
     ap.add_argument("--no-sparse", action="store_true", help="skip the block-sparse measurement")
+    ap.add_argument("--no-det", action="store_true", help="skip the deterministic backward measurement")
+    ap.add_argument("--no-configs", action="store_true", help="skip the other four workloads")
     ap.add_argument("--sparse-window", type=int, default=16)
     ap.add_argument("--sparse-sink", type=int, default=2)
     ap.add_argument("--cpu-rows", type=int, default=16384)
@@ -685,14 +834,23 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
 
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
+    launched = "WORLD_SIZE" in os.environ
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
 
     if args.impl == "reference":
+        # host cores only: rank 0 prints the line, other ranks exit without work
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)
         return
+
+    if not launched and args.gpus > 1:
+        sys.exit(spawn_ranks(args.gpus))
+    if world != args.gpus:
+        raise SystemExit(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}; they must agree")
 
     import torch
     import torch.distributed as dist

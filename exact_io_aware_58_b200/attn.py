@@ -34,6 +34,7 @@ EXPORTED = ("attn_fwd", "attn_fwd_f32out", "attn_fwd_gqa", "attn_fwd_blocksparse
             "attn_bwd_blocksparse", "attn_bwd_deterministic", "attn_bwd_workspace_bytes",
             "attn_bwd_deterministic_workspace_bytes", "attn_fwd_fp8", "attn_fwd_kvcache", "attn_fwd_kvcache_fp8",
             "attn_fwd_kvcache_splits", "attn_fwd_kvcache_workspace_bytes",
+            "attn_bwd_fused_preprocess", "attn_bwd_fused_dkdvdq", "attn_bwd_fused_dq_convert",
             "attn_bwd_preprocess", "attn_bwd_dkdv",
             "attn_bwd_dq", "attn_bwd_static_workspace", "attn_check_status", "attn_last_error",
             "attn_selftest_wait_timeout",
@@ -97,6 +98,13 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.attn_bwd_deterministic.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i32, f32, vp,
                                            ctypes.c_size_t, vp]
     lib.attn_bwd_deterministic.restype = i32
+    lib.attn_bwd_fused_preprocess.argtypes = [vp, vp, vp, i64, i64, i64, i64, vp, ctypes.c_size_t, vp]
+    lib.attn_bwd_fused_preprocess.restype = i32
+    lib.attn_bwd_fused_dkdvdq.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, f32, vp,
+                                          ctypes.c_size_t, vp]
+    lib.attn_bwd_fused_dkdvdq.restype = i32
+    lib.attn_bwd_fused_dq_convert.argtypes = [vp, i64, i64, i64, i64, f32, vp, ctypes.c_size_t, vp]
+    lib.attn_bwd_fused_dq_convert.restype = i32
     lib.attn_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i32, f32, vp,
                              ctypes.c_size_t, vp]
     lib.attn_bwd.restype = i32
@@ -437,6 +445,40 @@ def _ws(workspace):
         raise ValueError("workspace must be a contiguous CUDA tensor")
     _check_device("workspace", workspace)
     return _ptr(workspace), workspace.numel() * workspace.element_size()
+
+
+def attn_bwd_fused_preprocess(O, dO, LSE, workspace, stream=None) -> None:
+    _check_bhnd("O", O)
+    _check_bhnd("dO", dO, O.shape)
+    _check_lse(LSE, O.shape)
+    B, H, N, d = O.shape
+    wp, wb = _ws(workspace)
+    st = load_library().attn_bwd_fused_preprocess(_ptr(O), _ptr(dO), _ptr(LSE), B, H, N, d, wp, wb,
+                                                  _stream_handle(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_bwd_fused_preprocess")
+
+
+def attn_bwd_fused_dkdvdq(Q, K, V, dO, dK, dV, causal: bool, scale: float, workspace, stream=None) -> None:
+    _check_bhnd("Q", Q)
+    for n, t in (("K", K), ("V", V), ("dO", dO), ("dK", dK), ("dV", dV)):
+        _check_bhnd(n, t, Q.shape)
+    B, H, N, d = Q.shape
+    wp, wb = _ws(workspace)
+    st = load_library().attn_bwd_fused_dkdvdq(_ptr(Q), _ptr(K), _ptr(V), _ptr(dO), _ptr(dK), _ptr(dV), B, H, N, d,
+                                              int(bool(causal)), float(scale), wp, wb, _stream_handle(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_bwd_fused_dkdvdq")
+
+
+def attn_bwd_fused_dq_convert(dQ, scale: float, workspace, stream=None) -> None:
+    _check_bhnd("dQ", dQ)
+    B, H, N, d = dQ.shape
+    wp, wb = _ws(workspace)
+    st = load_library().attn_bwd_fused_dq_convert(_ptr(dQ), B, H, N, d, float(scale), wp, wb,
+                                                  _stream_handle(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_bwd_fused_dq_convert")
 
 
 def attn_bwd_preprocess(O, dO, LSE, workspace, stream=None) -> None:

@@ -446,24 +446,48 @@ int bwd_impl(const void* Q, const void* K, const void* V, const void* O, const v
 // pass over the key tiles for dK, dV and the dQ partials, and the dQ
 // conversion.  Workspace: [B*H][Npad] LSE*log2(e), [B*H][Npad] D, then the
 // accumulator [B*H][Npad][d] fp32.
-int fused_impl(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
-               void* dQ, void* dK, void* dV, const uint8_t* mask, int64_t B, int64_t H, int64_t H_kv, int64_t N,
-               int64_t d, int causal, float scale, void* workspace, size_t workspace_bytes, void* stream) {
+int fused_setup(int64_t B, int64_t H, int64_t N, int64_t d, void* workspace, size_t workspace_bytes, BwdSetup* su,
+                float** dq_acc) {
   int s = check_sizes(B, H, N, d);
+  if (s != ATTN_OK) return s;
+  if (!workspace) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(workspace)) return ATTN_ERR_MISALIGNED;
+  if (workspace_bytes < attn_bwd_workspace_bytes(B, H, N, d)) return ATTN_ERR_WORKSPACE;
+  su->bh = B * H;
+  su->npad = npad_of(N);
+  su->ws_lse2 = static_cast<float*>(workspace);
+  su->ws_d = su->ws_lse2 + su->bh * su->npad;
+  *dq_acc = su->ws_d + su->bh * su->npad;
+  return ATTN_OK;
+}
+
+int fused_pre_impl(const void* O, const void* dO, const float* LSE, int64_t B, int64_t H, int64_t N, int64_t d,
+                   void* workspace, size_t workspace_bytes, void* stream) {
+  BwdSetup su;
+  float* dq_acc = nullptr;
+  int s = fused_setup(B, H, N, d, workspace, workspace_bytes, &su, &dq_acc);
+  if (s != ATTN_OK) return s;
+  if (!O || !dO || !LSE) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(O) || !aligned16(dO) || !aligned16(LSE)) return ATTN_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return (d == 128) ? launch_bwd_pre<128>(O, dO, LSE, su.ws_lse2, su.ws_d, int(N), int(su.npad), su.bh * su.npad, st,
+                                          dq_acc)
+                    : launch_bwd_pre<64>(O, dO, LSE, su.ws_lse2, su.ws_d, int(N), int(su.npad), su.bh * su.npad, st,
+                                         dq_acc);
+}
+
+int fused_main_impl(const void* Q, const void* K, const void* V, const void* dO, void* dK, void* dV,
+                    const uint8_t* mask, int64_t B, int64_t H, int64_t H_kv, int64_t N, int64_t d, int causal,
+                    float scale, void* workspace, size_t workspace_bytes, void* stream) {
+  BwdSetup su;
+  float* dq_acc = nullptr;
+  int s = fused_setup(B, H, N, d, workspace, workspace_bytes, &su, &dq_acc);
   if (s != ATTN_OK) return s;
   if ((s = check_heads(H, H_kv)) != ATTN_OK) return s;
   if ((s = check_scale(scale)) != ATTN_OK) return s;
-  if (!Q || !K || !V || !O || !dO || !LSE || !dQ || !dK || !dV || !workspace) return ATTN_ERR_INVALID_ARG;
-  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(dO) || !aligned16(LSE) ||
-      !aligned16(dQ) || !aligned16(dK) || !aligned16(dV) || !aligned16(workspace))
+  if (!Q || !K || !V || !dO || !dK || !dV) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(dO) || !aligned16(dK) || !aligned16(dV))
     return ATTN_ERR_MISALIGNED;
-  if (workspace_bytes < attn_bwd_workspace_bytes(B, H, N, d)) return ATTN_ERR_WORKSPACE;
-  BwdSetup su;
-  su.bh = B * H;
-  su.npad = npad_of(N);
-  su.ws_lse2 = static_cast<float*>(workspace);
-  su.ws_d = su.ws_lse2 + su.bh * su.npad;
-  float* dq_acc = su.ws_d + su.bh * su.npad;
   const int64_t bhkv = B * H_kv;
   CUtensorMap mq, mk, mv, mdo, mdk, mdv, macc;
   if (!make_map(&mq, Q, su.bh, N, d) || !make_map(&mk, K, bhkv, N, d) || !make_map(&mv, V, bhkv, N, d) ||
@@ -474,15 +498,41 @@ int fused_impl(const void* Q, const void* K, const void* V, const void* O, const
   const bool sparse = mask != nullptr;
   const int grid = int(bhkv * prm.n_tiles);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  s = (d == 128) ? launch_bwd_pre<128>(O, dO, LSE, su.ws_lse2, su.ws_d, int(N), int(su.npad), su.bh * su.npad, st,
-                                       dq_acc)
-                 : launch_bwd_pre<64>(O, dO, LSE, su.ws_lse2, su.ws_d, int(N), int(su.npad), su.bh * su.npad, st,
-                                      dq_acc);
+  return ATTN_DISPATCH(launch_fused, mq, mk, mv, mdo, mdk, mdv, macc, prm, grid, st);
+}
+
+int fused_convert_impl(void* dQ, int64_t B, int64_t H, int64_t N, int64_t d, float scale, void* workspace,
+                       size_t workspace_bytes, void* stream) {
+  BwdSetup su;
+  float* dq_acc = nullptr;
+  int s = fused_setup(B, H, N, d, workspace, workspace_bytes, &su, &dq_acc);
   if (s != ATTN_OK) return s;
-  s = ATTN_DISPATCH(launch_fused, mq, mk, mv, mdo, mdk, mdv, macc, prm, grid, st);
-  if (s != ATTN_OK) return s;
+  if ((s = check_scale(scale)) != ATTN_OK) return s;
+  if (!dQ) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(dQ)) return ATTN_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
   return (d == 128) ? launch_dq_convert<128>(dq_acc, dQ, int(N), int(su.npad), su.bh * N, scale, st)
                     : launch_dq_convert<64>(dq_acc, dQ, int(N), int(su.npad), su.bh * N, scale, st);
+}
+
+int fused_impl(const void* Q, const void* K, const void* V, const void* O, const void* dO, const float* LSE,
+               void* dQ, void* dK, void* dV, const uint8_t* mask, int64_t B, int64_t H, int64_t H_kv, int64_t N,
+               int64_t d, int causal, float scale, void* workspace, size_t workspace_bytes, void* stream) {
+  // every argument is checked before the first launch
+  int s = check_sizes(B, H, N, d);
+  if (s != ATTN_OK) return s;
+  if ((s = check_heads(H, H_kv)) != ATTN_OK) return s;
+  if ((s = check_scale(scale)) != ATTN_OK) return s;
+  if (!Q || !K || !V || !O || !dO || !LSE || !dQ || !dK || !dV || !workspace) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(dO) || !aligned16(LSE) ||
+      !aligned16(dQ) || !aligned16(dK) || !aligned16(dV) || !aligned16(workspace))
+    return ATTN_ERR_MISALIGNED;
+  if (workspace_bytes < attn_bwd_workspace_bytes(B, H, N, d)) return ATTN_ERR_WORKSPACE;
+  s = fused_pre_impl(O, dO, LSE, B, H, N, d, workspace, workspace_bytes, stream);
+  if (s != ATTN_OK) return s;
+  s = fused_main_impl(Q, K, V, dO, dK, dV, mask, B, H, H_kv, N, d, causal, scale, workspace, workspace_bytes, stream);
+  if (s != ATTN_OK) return s;
+  return fused_convert_impl(dQ, B, H, N, d, scale, workspace, workspace_bytes, stream);
 }
 
 }  // namespace
@@ -506,6 +556,24 @@ ATTN_EXPORT int attn_bwd(const void* Q, const void* K, const void* V, const void
                          float scale, void* workspace, size_t workspace_bytes, void* stream) {
   return fused_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, nullptr, B, H, H, N, d, causal, scale, workspace,
                     workspace_bytes, stream);
+}
+
+ATTN_EXPORT int attn_bwd_fused_preprocess(const void* O, const void* dO, const float* LSE, int64_t B, int64_t H,
+                                          int64_t N, int64_t d, void* workspace, size_t workspace_bytes,
+                                          void* stream) {
+  return fused_pre_impl(O, dO, LSE, B, H, N, d, workspace, workspace_bytes, stream);
+}
+
+ATTN_EXPORT int attn_bwd_fused_dkdvdq(const void* Q, const void* K, const void* V, const void* dO, void* dK,
+                                      void* dV, int64_t B, int64_t H, int64_t N, int64_t d, int causal, float scale,
+                                      void* workspace, size_t workspace_bytes, void* stream) {
+  return fused_main_impl(Q, K, V, dO, dK, dV, nullptr, B, H, H, N, d, causal, scale, workspace, workspace_bytes,
+                         stream);
+}
+
+ATTN_EXPORT int attn_bwd_fused_dq_convert(void* dQ, int64_t B, int64_t H, int64_t N, int64_t d, float scale,
+                                          void* workspace, size_t workspace_bytes, void* stream) {
+  return fused_convert_impl(dQ, B, H, N, d, scale, workspace, workspace_bytes, stream);
 }
 
 ATTN_EXPORT int attn_bwd_deterministic(const void* Q, const void* K, const void* V, const void* O, const void* dO,

@@ -53,30 +53,34 @@ struct FusedCfg {
   static constexpr int kWarpLoad = 9;
   static constexpr int kWarpDrain0 = 10;                    // warps 10..13: lane quarters 2, 3, 0, 1
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr bool kStageInDS = (D == 128);            // dQ partial staged through the dS tile
-  static constexpr int kQS = (D == 128) ? 2 : 4;            // Q_i ring (read by S^T and, last, by dK)
-  static constexpr int kOS = (D == 128) ? 2 : 3;            // dO_i ring
+  // Ring depths.  Q_i is read by S^T(i) (issued right after dV(i-1)) and,
+  // last, by dK(i); dO_i by dP^T(i) and, last, by dV(i).  dP^T(i+1) is only
+  // issued once dK(i), dQ(i) and the drain's TMEM read have happened, long
+  // after dV(i) frees the dO slot, so at D = 128 a single dO slot suffices and
+  // its 32 KB go to the dQ staging ring.
+  static constexpr int kQS = (D == 128) ? 2 : 4;
+  static constexpr int kOS = (D == 128) ? 1 : 3;
   static constexpr int kVS = 2;                             // (LSE2, D) vector ring
+  static constexpr int kStageBlocks = 2;                    // staging ring of [128][32] fp32 blocks
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kTileBytes;
   static constexpr int kOffQ = 2 * kTileBytes;
   static constexpr int kOffDO = kOffQ + kQS * kTileBytes;
   static constexpr int kOffDS = kOffDO + kOS * kTileBytes;  // dS^T, [128 keys][128 queries] bf16
   static constexpr int kDSBytes = 128 * 128 * 2;
-  static constexpr int kOffStage = kOffDS + kDSBytes;       // D = 64: [128 queries][64] fp32
-  static constexpr int kStageBytes = kStageInDS ? 0 : 128 * D * 4;
-  static constexpr int kOffVec = kOffStage + kStageBytes;
+  static constexpr int kOffStage = kOffDS + kDSBytes;
+  static constexpr int kOffVec = kOffStage + kStageBlocks * kBlockBytes;
   static constexpr int kOffBar = kOffVec + kVS * 2 * kVecBytes;
-  static constexpr int kNumBars = 2 * kQS + 2 * kOS + 2 * kVS + 11;
+  static constexpr int kNumBars = 2 * kQS + 2 * kOS + 2 * kVS + 10;
   static constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
-  static_assert(kStageInDS ? (128 * D * 4 == 2 * kDSBytes) : true, "D = 128 stages the dQ partial in two halves");
   // TMEM columns
   static constexpr uint32_t kColS = 0;
   static constexpr uint32_t kColDP = 128;
   static constexpr uint32_t kColDV = 256;
   static constexpr uint32_t kColDK = 256 + D;
-  static constexpr uint32_t kColDQ = (D == 128) ? kColDP : 256 + 2 * D;
+  static constexpr bool kDqInDP = (D == 128);               // dQ partial over the dP^T columns
+  static constexpr uint32_t kColDQ = kDqInDP ? kColDP : 256 + 2 * D;
   static_assert(kColDQ + D <= kTmemCols, "tensor memory budget");
 };
 
@@ -111,9 +115,8 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
   uint64_t* ds_full = p_full + 1;          // dS^T(i) in shared memory, dP^T(i) read (256 arrivals)
   uint64_t* dq_full = ds_full + 1;         // dQ partial (i) in TMEM
   uint64_t* dq_free = dq_full + 1;         // drain has read it out of TMEM (128 arrivals)
-  uint64_t* ds_read = dq_free + 1;         // dQ(i) and dK(i) MMAs done reading the dS tile
-  uint64_t* dsb_free = ds_read + 1;        // D = 128: staging through the dS tile finished
-  uint64_t* acc_full = dsb_free + 1;
+  uint64_t* ds_read = dq_free + 1;         // the dQ(i) MMA is done reading the dS tile
+  uint64_t* acc_full = ds_read + 1;
   uint64_t* drain = acc_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::kNumBars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + C::kNumBars) + 1;
@@ -159,7 +162,6 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     mbar_init(dq_full, 1);
     mbar_init(dq_free, 128);
     mbar_init(ds_read, 1);
-    mbar_init(dsb_free, 1);
     mbar_init(acc_full, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -241,7 +243,7 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     if (lane == 0) {
       constexpr uint32_t kIdescT = idesc_bf16(128, 128, false, false);   // S^T, dP^T (both K-major)
       constexpr uint32_t kIdescDV = idesc_bf16(128, D, false, true);     // A = P^T (TMEM), B = dO_i MN-major
-      constexpr uint32_t kIdescDK = idesc_bf16(128, D, false, true);     // A = dS^T K-major, B = Q_i MN-major
+      constexpr uint32_t kIdescDK = idesc_bf16(128, D, false, true);     // A = dS^T (TMEM), B = Q_i MN-major
       constexpr uint32_t kIdescDQ = idesc_bf16(128, D, true, true);      // A = dS MN-major, B = K_j MN-major
       const uint32_t sK = smem_u32(smem + C::kOffK);
       const uint32_t sV = smem_u32(smem + C::kOffV);
@@ -262,13 +264,11 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           mma_ts(tmem + C::kColDV, tmem + C::kColS + 64 * (kk >> 2) + (kk & 3) * 8,
                  smem_desc_sw128(o_tile(it) + kk * 2048, C::kBlockBytes, 1024), kIdescDV, (it > 0 || kk > 0) ? 1u : 0u);
       };
-      auto issue_dk = [&](int it) {   // dK += dS^T Q_i, K = 128 queries
+      auto issue_dk = [&](int it) {   // dK += dS^T Q_i, K = 128 queries; A = dS^T (bf16 over the dP^T columns)
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
-          const uint32_t off = (kk >> 2) * C::kBlockBytes + (kk & 3) * 32;
-          mma_ss(tmem + C::kColDK, smem_desc_sw128(sDS + off, 16, 1024),
+        for (int kk = 0; kk < 8; ++kk)
+          mma_ts(tmem + C::kColDK, tmem + C::kColDP + 64 * (kk >> 2) + (kk & 3) * 8,
                  smem_desc_sw128(q_tile(it) + kk * 2048, C::kBlockBytes, 1024), kIdescDK, (it > 0 || kk > 0) ? 1u : 0u);
-        }
       };
       auto issue_dq = [&]() {         // dQ_i partial = dS K_j, K = 128 keys
 #pragma unroll
@@ -301,16 +301,18 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         }
         if (!(ok = mbar_wait(ds_full, it & 1, abort_flag))) break;
         // D = 64: the dQ columns are free once the drain has read the previous partial
-        if (!C::kStageInDS && it > 0 && !(ok = mbar_wait(dq_free, (it - 1) & 1, abort_flag))) break;
+        if (!C::kDqInDP && it > 0 && !(ok = mbar_wait(dq_free, (it - 1) & 1, abort_flag))) break;
         tc_fence_after();
-        issue_dq();
-        mma_commit(dq_full);
+        // dK first: at D = 128 the dQ partial is written over the dP^T columns
+        // that hold dS^T, which the in-order MMA pipe has then finished reading
         issue_dk(it);
         mma_commit(&q_empty[it % QS]);        // Q_i read for the last time
+        issue_dq();
+        mma_commit(dq_full);
         mma_commit(ds_read);                  // the dS tile is no longer read
         if (more) {
           // D = 128: dP^T shares its columns with the dQ partial
-          if (C::kStageInDS && !(ok = mbar_wait(dq_free, it & 1, abort_flag))) break;
+          if (C::kDqInDP && !(ok = mbar_wait(dq_free, it & 1, abort_flag))) break;
           if (!(ok = wait_o(it + 1))) break;
           tc_fence_after();
           issue_t(C::kColDP, sV, o_tile(it + 1));
@@ -373,19 +375,23 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       mbar_arrive(p_full);
 
       if (!(ok = mbar_wait_warp(dp_full, it & 1, abort_flag))) break;
-      // the dS tile of the previous iteration is no longer needed (read by its
-      // MMAs, and at D = 128 by the drain's staging too)
-      if (it > 0 && !(ok = mbar_wait_warp(C::kStageInDS ? dsb_free : ds_read, (it - 1) & 1, abort_flag))) break;
+      // the dQ MMA of the previous iteration has read the dS tile
+      if (it > 0 && !(ok = mbar_wait_warp(ds_read, (it - 1) & 1, abort_flag))) break;
       tc_fence_after();
       const float4* d4 = reinterpret_cast<const float4*>(vec + 128 + 64 * g);
+      // dS^T for 32 query columns at a time: to shared memory (the dQ MMA's
+      // A operand) and, packed as bf16 pairs over the first 32 of this group's
+      // dP^T columns, to tensor memory (the dK MMA's A operand).  The packed
+      // columns of half h are [16h, 16h + 16): half 1 reads columns 32..63
+      // before nothing below column 32 is written again.
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t dpr[32];
         tmem_ld32(tB + 32 * h, dpr);
         tmem_ld_wait(dpr);
+        uint32_t pk[16];
 #pragma unroll
         for (int ch = 0; ch < 4; ++ch) {
-          uint32_t w[4];
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
             const int k = 32 * h + 8 * ch + 4 * u;            // query column inside the group
@@ -394,15 +400,17 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
             const float s1 = p[k + 1] * (__uint_as_float(dpr[8 * ch + 4 * u + 1]) - dv.y);
             const float s2 = p[k + 2] * (__uint_as_float(dpr[8 * ch + 4 * u + 2]) - dv.z);
             const float s3 = p[k + 3] * (__uint_as_float(dpr[8 * ch + 4 * u + 3]) - dv.w);
-            w[2 * u] = pack_bf16x2(s0, s1);
-            w[2 * u + 1] = pack_bf16x2(s2, s3);
+            pk[4 * ch + 2 * u] = pack_bf16x2(s0, s1);
+            pk[4 * ch + 2 * u + 1] = pack_bf16x2(s2, s3);
           }
-          st_shared_v4(sDSg + sw128_offset(r, 4 * h + ch), w[0], w[1], w[2], w[3]);
+          st_shared_v4(sDSg + sw128_offset(r, 4 * h + ch), pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
         }
+        tmem_st16(tB + 16 * h, pk);
       }
+      tmem_st_wait();
       mbar_arrive(&v_empty[it % VS]);   // this thread is done with the LSE/D vectors
-      tc_fence_before();                // dP^T has been read (its columns may be overwritten)
-      fence_proxy_async_smem();         // dS^T visible to the tensor core
+      tc_fence_before();                // dP^T read, dS^T written (tensor memory)
+      fence_proxy_async_smem();         // dS^T visible to the tensor core (shared memory)
       mbar_arrive(ds_full);
     }
     // epilogue: group 0 writes dV (staged in the V_j slot), group 1 writes dK (in the K_j slot)
@@ -426,13 +434,19 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     }
   } else {
     // ------------------------------------------------------------ dQ drain
-    // thread = query row r of the partial (TMEM lane); warp w reads lane quarter w % 4
+    // thread = query row r of the partial (TMEM lane); warp w reads lane quarter w % 4.
+    // The partial is read out of TMEM 64 columns at a time (so that, with the
+    // last read, its columns are released before any wait on the staging);
+    // each 32-column chunk is then staged as a [128][32] fp32 block in a ring
+    // of two and added into the accumulator by one TMA reduce.  A block is
+    // rewritten only after the reduce that used it two chunks before has read
+    // it, so the reduces stream out while the next chunks are staged and while
+    // the next tile pair is computed.
     const int qd = warp & 3;
     const int r = qd * 32 + lane;
     const uint32_t tQ = tmem + (uint32_t(qd * 32) << 16) + C::kColDQ;
     const bool leader = (warp == C::kWarpDrain0 && lane == 0);
-    const uint32_t stage = smem_u32(smem + (C::kStageInDS ? C::kOffDS : C::kOffStage));
-    uint8_t* stage_ptr = smem + (C::kStageInDS ? C::kOffDS : C::kOffStage);
+    uint8_t* stage = smem + C::kOffStage;
     // The four drain warps meet at named barriers inside the loop, so a failed
     // wait must not make one warp leave alone: the first barrier of every
     // iteration ANDs the warps' status and they all stop together.
@@ -442,65 +456,42 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       if (SPARSE) Lsel = sel_next(sel, Lsel, n_all);
       const int qrow = (i_start + L % n_q) * 128;
       const int bq = bq0 + L / n_q;
-      bool ok = mbar_wait_warp(dq_full, it & 1, abort_flag);
-      uint32_t a[32], b[32];
-      if (ok) {
-        tc_fence_after();
-        tmem_ld32(tQ + 0, a);
-        tmem_ld32(tQ + 32, b);
-        tmem_ld_wait(a);
-        reg_fence32(b);
-      }
-      if (C::kStageInDS) {
-        // the dQ and dK MMAs of this iteration must be done with the dS tile
-        if (ok) ok = mbar_wait_warp(ds_read, it & 1, abort_flag);
+      const bool ok = mbar_wait_warp(dq_full, it & 1, abort_flag);
+      if (ok) tc_fence_after();
+      bool go = true;
+#pragma unroll 1
+      for (int p = 0; p < D / 64 && go; ++p) {
+        uint32_t a[32], b[32];
         if (ok) {
-          stage_row32(stage, r, a);
-          stage_row32(stage + C::kBlockBytes, r, b);
-          tmem_ld32(tQ + 64, a);
-          tmem_ld32(tQ + 96, b);
+          tmem_ld32(tQ + 64 * p, a);
+          tmem_ld32(tQ + 64 * p + 32, b);
           tmem_ld_wait(a);
           reg_fence32(b);
-          tc_fence_before();
-          mbar_arrive(dq_free);               // the partial's TMEM columns are free
+          if (p == D / 64 - 1) {
+            tc_fence_before();
+            mbar_arrive(dq_free);             // the partial's TMEM columns are free
+          }
+        }
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {        // chunk 2p + h goes through staging block h
+          // block h was last read by the reduce issued two chunks ago
+          if (leader) bulk_wait_group_read1();
+          if (p == 0 && h == 0) {
+            if (!(go = named_barrier_and(3, 128, ok))) break;
+          } else {
+            named_barrier_sync(3, 128);
+          }
+          uint8_t* blk = stage + h * C::kBlockBytes;
+          stage_row32(smem_u32(blk), r, h ? b : a);
           fence_proxy_async_smem();
-        }
-        if (!named_barrier_and(3, 128, ok)) break;
-        if (leader) {
-          tma_reduce_add_3d(&tm_dqacc, stage_ptr, 0, qrow, bq);
-          tma_reduce_add_3d(&tm_dqacc, stage_ptr + C::kBlockBytes, 32, qrow, bq);
-          bulk_commit_group();
-          bulk_wait_group_read0();
-        }
-        named_barrier_sync(3, 128);
-        stage_row32(stage, r, a);
-        stage_row32(stage + C::kBlockBytes, r, b);
-        fence_proxy_async_smem();
-        named_barrier_sync(3, 128);
-        if (leader) {
-          tma_reduce_add_3d(&tm_dqacc, stage_ptr, 64, qrow, bq);
-          tma_reduce_add_3d(&tm_dqacc, stage_ptr + C::kBlockBytes, 96, qrow, bq);
-          bulk_commit_group();
-          bulk_wait_group_read0();
-          mbar_arrive(dsb_free);              // the dS tile may be written again
-        }
-      } else {
-        if (ok) {
-          tc_fence_before();
-          mbar_arrive(dq_free);
-        }
-        if (leader) bulk_wait_group_read0();  // the previous reduce has read the staging buffer
-        if (!named_barrier_and(3, 128, ok)) break;
-        stage_row32(stage, r, a);
-        stage_row32(stage + C::kBlockBytes, r, b);
-        fence_proxy_async_smem();
-        named_barrier_sync(3, 128);
-        if (leader) {
-          tma_reduce_add_3d(&tm_dqacc, stage_ptr, 0, qrow, bq);
-          tma_reduce_add_3d(&tm_dqacc, stage_ptr + C::kBlockBytes, 32, qrow, bq);
-          bulk_commit_group();
+          named_barrier_sync(3, 128);
+          if (leader) {
+            tma_reduce_add_3d(&tm_dqacc, blk, 64 * p + 32 * h, qrow, bq);
+            bulk_commit_group();
+          }
         }
       }
+      if (!go) break;
     }
     if (leader) bulk_wait_group0();   // every reduce has completed
   }

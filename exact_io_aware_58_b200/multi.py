@@ -6,10 +6,16 @@ Compression", section "The composability point": the kernel tiles over
 whatever heads exist).  So work is split across ranks by whole heads (or whole
 batches) with no collective on the data path; the only communication is the
 timing reduction (max over ranks) and, optionally, gathering results for a
-check.  One process per GPU, launched by torchrun.
+check.  One process per GPU.
+
+The benchmark's per-rank loop lives here (``run_timed``) with the clock and
+the barrier passed in, so the same code runs with CUDA events on a GPU and
+with a host clock in the multi-process CPU tests.
 """
 
 from __future__ import annotations
+
+import os
 
 import torch
 
@@ -43,3 +49,68 @@ def max_over_ranks(values, device=None, group=None) -> list[float]:
 def aggregate_tflops(flops_per_rank: float, world: int, ms_max: float) -> float:
     """Whole-job throughput: every rank's FLOPs over the slowest rank's time."""
     return flops_per_rank * world / (ms_max * 1e-3) / 1e12
+
+
+class CudaClock:
+    """Timestamps as CUDA events recorded on one stream (the stream the
+    kernels are launched on); ``sync`` waits for the device."""
+
+    def __init__(self, stream):
+        self.stream = stream
+
+    def mark(self):
+        e = torch.cuda.Event(enable_timing=True)
+        e.record(self.stream)
+        return e
+
+    @staticmethod
+    def elapsed_ms(a, b) -> float:
+        return a.elapsed_time(b)
+
+    @staticmethod
+    def sync():
+        torch.cuda.synchronize()
+
+
+def run_timed(step, steps: int, warmup: int, clock, barrier=None, n_segments: int = 1, on_timed_start=None):
+    """``warmup`` untimed calls of ``step(mark)``, then a barrier and a sync on
+    both sides of ``steps`` timed calls.  ``step`` calls ``mark()`` between its
+    kernels: ``n_segments`` segments need ``n_segments - 1`` inner marks (the
+    first and last are taken here).  Returns (total ms of the timed region,
+    [mean ms of each segment]) for this rank; reduce them with
+    ``max_over_ranks``."""
+    for _ in range(warmup):
+        step(lambda: None)
+    if barrier is not None:
+        barrier()
+    clock.sync()
+    if on_timed_start is not None:
+        on_timed_start()
+    marks = []
+    t0 = clock.mark()
+    for _ in range(steps):
+        m = [clock.mark()]
+        step(lambda: m.append(clock.mark()))
+        m.append(clock.mark())
+        if len(m) != n_segments + 1:
+            raise RuntimeError(f"step made {len(m) - 2} inner marks, expected {n_segments - 1}")
+        marks.append(m)
+    t1 = clock.mark()
+    clock.sync()
+    if barrier is not None:
+        barrier()
+    total = clock.elapsed_ms(t0, t1)
+    seg = [sum(clock.elapsed_ms(m[k], m[k + 1]) for m in marks) / steps for k in range(n_segments)]
+    return total, seg
+
+
+def rank_envs(n: int, port: int, base_env=None) -> list[dict]:
+    """Environment of each of ``n`` rank processes on this node (one GPU each):
+    the torch.distributed variables the benchmark reads."""
+    envs = []
+    for r in range(n):
+        e = dict(os.environ if base_env is None else base_env)
+        e.update({"RANK": str(r), "LOCAL_RANK": str(r), "WORLD_SIZE": str(n), "LOCAL_WORLD_SIZE": str(n),
+                  "MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port)})
+        envs.append(e)
+    return envs

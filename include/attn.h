@@ -244,6 +244,31 @@ int attn_bwd(const void* Q, const void* K, const void* V, const void* O, const v
              void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * The three steps of attn_bwd, callable one at a time (same arguments, rules
+ * and workspace as attn_bwd; attn_bwd is exactly these three calls in this
+ * order on one stream).  Useful to time the steps separately.
+ *
+ * attn_bwd_fused_preprocess: per row, D_i = sum_k dO_ik O_ik and
+ *   LSE_i*log2(e) into `workspace`, and the fp32 dQ accumulator set to zero.
+ * attn_bwd_fused_dkdvdq: one CTA per 128-key tile; writes dK and dV and adds
+ *   every query tile's dQ contribution (dS K_j, before the scale) into the
+ *   accumulator; reads the vectors ("Attention and KV Compression", section
+ *   "Recomputation in the backward pass": the score tiles are recomputed once).
+ * attn_bwd_fused_dq_convert: dQ = scale * accumulator, rounded to bf16.
+ */
+int attn_bwd_fused_preprocess(const void* O, const void* dO, const float* LSE,
+                              int64_t B, int64_t H, int64_t N, int64_t d,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+int attn_bwd_fused_dkdvdq(const void* Q, const void* K, const void* V, const void* dO,
+                          void* dK, void* dV,
+                          int64_t B, int64_t H, int64_t N, int64_t d, int causal, float scale,
+                          void* workspace, size_t workspace_bytes, void* stream);
+
+int attn_bwd_fused_dq_convert(void* dQ, int64_t B, int64_t H, int64_t N, int64_t d, float scale,
+                              void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * The same backward with bitwise-reproducible results: (1) the per-row vectors
  * as in attn_bwd, (2) per 128-key tile, dK and dV (score tiles recomputed, 4
  * MMAs per tile pair), (3) per 128-query tile, dQ (score tiles recomputed

@@ -63,3 +63,27 @@ def assert_grad(g: np.ndarray, g_ref: np.ndarray, what: str):
     mx = float(np.abs(g - g_ref).max())
     assert mx <= GRAD_REL * ref_max + GRAD_ABS_FLOOR, \
         f"{what}: max err {mx:.3e} > {GRAD_REL} * {ref_max:.3e} + {GRAD_ABS_FLOOR}"
+
+
+GUARD = 64 * 1024          # guard bytes on each side (a multiple of 16: views stay 16-byte aligned)
+PATTERN = 0xA5
+
+
+class Guarded:
+    """A CUDA tensor of ``shape``/``dtype`` (or of ``nbytes`` bytes, flat) with
+    GUARD bytes of PATTERN on both sides, to detect writes outside it."""
+
+    def __init__(self, shape, dtype, nbytes=None, device="cuda:0"):
+        elem = torch.empty((), dtype=dtype).element_size()
+        self.n = int(np.prod(shape)) if nbytes is None else nbytes // elem
+        self.g = GUARD // elem
+        self.buf = torch.empty(self.g + self.n + self.g, dtype=dtype, device=device)
+        self.buf.view(torch.uint8).fill_(PATTERN)
+        self.t = self.buf[self.g:self.g + self.n]
+        if nbytes is None:
+            self.t = self.t.view(shape)
+
+    def intact(self) -> bool:
+        raw = self.buf.view(torch.uint8)
+        gb = self.g * self.buf.element_size()
+        return bool((raw[:gb] == PATTERN).all()) and bool((raw[raw.numel() - gb:] == PATTERN).all())

@@ -15,7 +15,7 @@ from exact_io_aware_58_b200 import attn
 from exact_io_aware_58_b200.inputs import WORKLOADS, make_inputs, sample_rows, workload_inputs
 from oracle import attn_oracle as orc
 
-from ._parity import assert_grad, assert_lse, assert_o, f64
+from ._parity import Guarded, assert_grad, assert_lse, assert_o, f64
 
 pytestmark = pytest.mark.gpu
 
@@ -163,8 +163,9 @@ def test_long_context_sampled_no_quadratic_memory():
     inp = workload_inputs(w, device=DEV)
     q, k, v = (inp[n] for n in ("Q", "K", "V"))
     inp = {n: t.cpu() for n, t in inp.items()}
-    o = torch.empty_like(q)
-    lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=DEV)
+    # outputs inside guard regions: nothing may be written past the ragged last tile (N = 781.25 x 128)
+    og, lg = Guarded(q.shape, torch.bfloat16), Guarded((w.B, w.H, w.N), torch.float32)
+    o, lse = og.t, lg.t
     torch.cuda.synchronize()
     torch.cuda.reset_peak_memory_stats()
     base_alloc = torch.cuda.memory_allocated()
@@ -175,6 +176,7 @@ def test_long_context_sampled_no_quadratic_memory():
     # nothing is allocated by the call: no N x N buffer (20 GB per head if materialised)
     assert torch.cuda.max_memory_allocated() - base_alloc == 0
     assert free0 - free1 < 64 * 2**20
+    assert og.intact() and lg.intact()
     _check_sampled_rows(inp, {"O": o, "LSE": lse}, w, w.check_rows)
 
 

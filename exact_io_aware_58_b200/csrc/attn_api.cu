@@ -207,6 +207,17 @@ int launch_fused(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& 
                  int grid, cudaStream_t st) {
   using C = attn::FusedCfg<D>;
   auto kern = attn::attn_bwd_fused_kernel<D, CAUSAL, SPARSE>;
+  // The kernel moves registers between its warpgroups (setmaxnreg); the split
+  // only adds up if every thread was launched with exactly kRegsLaunch of them
+  // (otherwise the growing warpgroup would wait for registers that never come).
+  cudaFuncAttributes fa;
+  const cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess)
+    return fail(ATTN_ERR_LAUNCH, "cudaFuncGetAttributes(fused backward): %s (%lld)", cudaGetErrorString(e),
+                (long long)e);
+  if (fa.numRegs != int(C::kRegsLaunch))
+    return fail(ATTN_ERR_LAUNCH, "fused backward compiled to %d registers per thread, its warpgroup split needs %d",
+                fa.numRegs, int(C::kRegsLaunch));
   if (set_smem(reinterpret_cast<const void*>(kern), C::kSmemBytes) != ATTN_OK) return ATTN_ERR_LAUNCH;
   kern<<<grid, C::kThreads, C::kSmemBytes, st>>>(q, k, v, dO, dk, dv, dqacc, prm);
   return launch_status();

@@ -48,10 +48,19 @@ struct FusedCfg {
   static constexpr int kBlockBytes = 128 * 128;             // [128][64] bf16 or [128][32] fp32 column block
   static constexpr int kNumBlk = D / 64;
   static constexpr int kVecBytes = 512;                     // 128 fp32
-  static constexpr int kThreads = 448;
+  static constexpr int kThreads = 512;
   static constexpr int kWarpMma = 8;
-  static constexpr int kWarpLoad = 9;
-  static constexpr int kWarpDrain0 = 10;                    // warps 10..13: lane quarters 2, 3, 0, 1
+  static constexpr int kWarpLoad = 9;                       // warps 10, 11 only complete warpgroup 2
+  static constexpr int kWarpDrain0 = 12;                    // warps 12..15 (warpgroup 3): lane quarters 0..3
+  // Registers per thread: launched with kRegsLaunch for every warp; warpgroup
+  // 2 (MMA, TMA, two idle warps) gives back down to kRegsIssue and warpgroup 3
+  // (the drain) takes up to kRegsDrain, enough to hold a whole 128-column
+  // partial.  2 * 128 + 80 + 176 = 4 * 128: the per-SM-subpartition register
+  // file is used exactly (each holds one warp of every warpgroup).
+  static constexpr uint32_t kRegsLaunch = 128;
+  static constexpr uint32_t kRegsIssue = 80;
+  static constexpr uint32_t kRegsDrain = 176;
+  static_assert(2 * kRegsLaunch + kRegsIssue + kRegsDrain == 4 * kRegsLaunch, "register split");
   static constexpr uint32_t kTmemCols = 512;
   // Ring depths.  Q_i is read by S^T(i) (issued right after dV(i-1)) and,
   // last, by dK(i); dO_i by dP^T(i) and, last, by dV(i).  dP^T(i+1) is only
@@ -93,7 +102,7 @@ __device__ __forceinline__ void stage_row32(uint32_t block_u32, int r, const uin
 }
 
 template <int D, bool CAUSAL, bool SPARSE>
-__global__ void __launch_bounds__(448, 1)
+__global__ void __launch_bounds__(512, 1)
 attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                       const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
@@ -181,8 +190,10 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
-  if (warp == C::kWarpLoad) {
+  if (warp >= C::kWarpMma && warp < C::kWarpDrain0) {
+   // warpgroup 2: one TMA thread, one MMA thread, two idle warps
+   regs_dec<C::kRegsIssue>();
+   if (warp == C::kWarpLoad) {
     // ------------------------------------------------------------------ TMA
     if (lane == 0) {
       if (n_it > 0) {
@@ -324,6 +335,7 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       mbar_wait(drain, 0, abort_flag, false);
     }
     __syncwarp();
+   }
   } else if (warp < C::kWarpMma) {
     // -------------------------------------------------------------- compute
     // thread = key row r (TMEM lane), group g = query columns [64g, 64g+64)
@@ -434,14 +446,16 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     }
   } else {
     // ------------------------------------------------------------ dQ drain
+    regs_inc<C::kRegsDrain>();
     // thread = query row r of the partial (TMEM lane); warp w reads lane quarter w % 4.
-    // The partial is read out of TMEM 64 columns at a time (so that, with the
-    // last read, its columns are released before any wait on the staging);
-    // each 32-column chunk is then staged as a [128][32] fp32 block in a ring
-    // of two and added into the accumulator by one TMA reduce.  A block is
-    // rewritten only after the reduce that used it two chunks before has read
-    // it, so the reduces stream out while the next chunks are staged and while
-    // the next tile pair is computed.
+    // The whole partial is read out of TMEM at once (four loads, one wait), so
+    // its columns are released after a single round trip; then each 32-column
+    // chunk is staged as a [128][32] fp32 block in a ring of two and added
+    // into the accumulator by one TMA reduce.  A block is rewritten only after
+    // the reduce that used it two chunks before has read it, so the reduces
+    // stream out while the next chunks are staged and while the next tile
+    // pair is computed.
+    constexpr int NC = D / 32;                // 32-column chunks per partial
     const int qd = warp & 3;
     const int r = qd * 32 + lane;
     const uint32_t tQ = tmem + (uint32_t(qd * 32) << 16) + C::kColDQ;
@@ -457,38 +471,34 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       const int qrow = (i_start + L % n_q) * 128;
       const int bq = bq0 + L / n_q;
       const bool ok = mbar_wait_warp(dq_full, it & 1, abort_flag);
-      if (ok) tc_fence_after();
-      bool go = true;
-#pragma unroll 1
-      for (int p = 0; p < D / 64 && go; ++p) {
-        uint32_t a[32], b[32];
-        if (ok) {
-          tmem_ld32(tQ + 64 * p, a);
-          tmem_ld32(tQ + 64 * p + 32, b);
-          tmem_ld_wait(a);
-          reg_fence32(b);
-          if (p == D / 64 - 1) {
-            tc_fence_before();
-            mbar_arrive(dq_free);             // the partial's TMEM columns are free
-          }
-        }
+      uint32_t a[NC][32];
+      if (ok) {
+        tc_fence_after();
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {        // chunk 2p + h goes through staging block h
-          // block h was last read by the reduce issued two chunks ago
-          if (leader) bulk_wait_group_read1();
-          if (p == 0 && h == 0) {
-            if (!(go = named_barrier_and(3, 128, ok))) break;
-          } else {
-            named_barrier_sync(3, 128);
-          }
-          uint8_t* blk = stage + h * C::kBlockBytes;
-          stage_row32(smem_u32(blk), r, h ? b : a);
-          fence_proxy_async_smem();
+        for (int c = 0; c < NC; ++c) tmem_ld32(tQ + 32 * c, a[c]);
+        tmem_ld_wait(a[0]);
+#pragma unroll
+        for (int c = 1; c < NC; ++c) reg_fence32(a[c]);
+        tc_fence_before();
+        mbar_arrive(dq_free);                 // the partial's TMEM columns are free
+      }
+      bool go = true;
+#pragma unroll
+      for (int c = 0; c < NC; ++c) {          // chunk c goes through staging block c % 2
+        // the block was last read by the reduce issued two chunks ago
+        if (leader) bulk_wait_group_read1();
+        if (c == 0) {
+          if (!(go = named_barrier_and(3, 128, ok))) break;
+        } else {
           named_barrier_sync(3, 128);
-          if (leader) {
-            tma_reduce_add_3d(&tm_dqacc, blk, 64 * p + 32 * h, qrow, bq);
-            bulk_commit_group();
-          }
+        }
+        uint8_t* blk = stage + (c & 1) * C::kBlockBytes;
+        stage_row32(smem_u32(blk), r, a[c]);
+        fence_proxy_async_smem();
+        named_barrier_sync(3, 128);
+        if (leader) {
+          tma_reduce_add_3d(&tm_dqacc, blk, 32 * c, qrow, bq);
+          bulk_commit_group();
         }
       }
       if (!go) break;

@@ -100,6 +100,22 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, v
 }
 
 // ----------------------------------------------------------------------------
+// Register redistribution between warpgroups (all four warps of a warpgroup
+// execute the same instruction).  The block's registers are fixed at launch;
+// .dec returns registers to the block's pool and .inc takes them from it
+// (waiting until they are there), so the per-warpgroup counts must add up to
+// what the block was launched with -- the host checks the compiled count.
+// ----------------------------------------------------------------------------
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+// ----------------------------------------------------------------------------
 // Named barriers, fences
 // ----------------------------------------------------------------------------
 __device__ __forceinline__ void named_barrier_sync(uint32_t id, uint32_t nthreads) {

@@ -16,26 +16,29 @@
 // scales the sum and rounds it to bf16).
 //
 // CTA = one 128-key tile of one key/value head, looping over every (query
-// head of its group, query tile); 448 threads:
+// head of its group, query tile); 512 threads in four warpgroups:
 //   warps 0-7   compute: thread = key row (TMEM lane), group g = query columns
-//               [64g, 64g+64).  P^T is written back into TMEM as bf16 (A
-//               operand of dV); dS^T is written once to shared memory as a
-//               128B-swizzled [128 keys][128 queries] bf16 tile, which is
+//               [64g, 64g+64).  P^T is written back into TMEM as bf16 (the A
+//               operand of dV += P^T dO_i); dS^T is written once to shared
+//               memory as a 128B-swizzled [128 keys][128 queries] bf16 tile,
 //               the K-major A operand of dK += dS^T Q_i and, read the other
 //               way, the MN-major A operand of dQ_i = dS K_j.
-//   warp 8      MMA issuer (one thread).
+//   warp 8      MMA issuer (one thread); per query tile: dV, S^T of the next
+//               tile, dQ, dK, dP^T of the next tile.
 //   warp 9      TMA producer (resident K_j, V_j; rings of Q_i, dO_i, and the
-//               per-row LSE/D vectors).
-//   warps 10-13 dQ drain: thread = query row (TMEM lane); each reads the dQ_i
-//               partial out of TMEM, stages it as fp32 in shared memory and
-//               one thread adds the staged boxes into the accumulator with
-//               cp.reduce.async.bulk.tensor (this GPU's memory only).
+//               per-row LSE/D vectors).  Warps 8-11 run on fewer registers
+//               (setmaxnreg) so that warps 12-15 can have more.
+//   warps 12-15 dQ drain: thread = query row (TMEM lane); each reads its row
+//               of the dQ_i partial out of TMEM in one go (which frees the
+//               columns for the next dP^T), stages it as fp32 in shared
+//               memory, and one thread adds the staged boxes into the
+//               accumulator with cp.reduce.async.bulk.tensor (this GPU's
+//               memory only), while the next tile pair is computed.
 // Tensor memory (512 columns): S^T [0,128), dP^T [128,256), dV, dK (D each).
 // At D = 128 TMEM is full, so the dQ partial reuses the dP^T columns once the
-// compute warps have read dP^T, and the next dP^T waits for the drain; the
-// 227 KB of shared memory is full too (K, V, two Q and two dO slots, dS), so
-// the drain stages through the dS tile once both MMAs have read it.  At
-// D = 64 the dQ partial and its staging buffer have room of their own.
+// compute warps have read dP^T, and the next dP^T waits for the drain; dQ is
+// issued before dK so that this read-out overlaps dK.  At D = 64 the dQ
+// partial has columns of its own.
 #pragma once
 
 #include "attn_bwd.cuh"
@@ -254,7 +257,7 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     if (lane == 0) {
       constexpr uint32_t kIdescT = idesc_bf16(128, 128, false, false);   // S^T, dP^T (both K-major)
       constexpr uint32_t kIdescDV = idesc_bf16(128, D, false, true);     // A = P^T (TMEM), B = dO_i MN-major
-      constexpr uint32_t kIdescDK = idesc_bf16(128, D, false, true);     // A = dS^T (TMEM), B = Q_i MN-major
+      constexpr uint32_t kIdescDK = idesc_bf16(128, D, false, true);     // A = dS^T K-major, B = Q_i MN-major
       constexpr uint32_t kIdescDQ = idesc_bf16(128, D, true, true);      // A = dS MN-major, B = K_j MN-major
       const uint32_t sK = smem_u32(smem + C::kOffK);
       const uint32_t sV = smem_u32(smem + C::kOffV);
@@ -275,11 +278,13 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           mma_ts(tmem + C::kColDV, tmem + C::kColS + 64 * (kk >> 2) + (kk & 3) * 8,
                  smem_desc_sw128(o_tile(it) + kk * 2048, C::kBlockBytes, 1024), kIdescDV, (it > 0 || kk > 0) ? 1u : 0u);
       };
-      auto issue_dk = [&](int it) {   // dK += dS^T Q_i, K = 128 queries; A = dS^T (bf16 over the dP^T columns)
+      auto issue_dk = [&](int it) {   // dK += dS^T Q_i, K = 128 queries; A = dS^T K-major from the dS tile
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_ts(tmem + C::kColDK, tmem + C::kColDP + 64 * (kk >> 2) + (kk & 3) * 8,
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * C::kBlockBytes + (kk & 3) * 32;
+          mma_ss(tmem + C::kColDK, smem_desc_sw128(sDS + off, 16, 1024),
                  smem_desc_sw128(q_tile(it) + kk * 2048, C::kBlockBytes, 1024), kIdescDK, (it > 0 || kk > 0) ? 1u : 0u);
+        }
       };
       auto issue_dq = [&]() {         // dQ_i partial = dS K_j, K = 128 keys
 #pragma unroll
@@ -314,12 +319,11 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         // D = 64: the dQ columns are free once the drain has read the previous partial
         if (!C::kDqInDP && it > 0 && !(ok = mbar_wait(dq_free, (it - 1) & 1, abort_flag))) break;
         tc_fence_after();
-        // dK first: at D = 128 the dQ partial is written over the dP^T columns
-        // that hold dS^T, which the in-order MMA pipe has then finished reading
-        issue_dk(it);
-        mma_commit(&q_empty[it % QS]);        // Q_i read for the last time
+        // dQ first, so that the drain reads the partial out of TMEM while dK runs
         issue_dq();
         mma_commit(dq_full);
+        issue_dk(it);
+        mma_commit(&q_empty[it % QS]);        // Q_i read for the last time
         mma_commit(ds_read);                  // the dS tile is no longer read
         if (more) {
           // D = 128: dP^T shares its columns with the dQ partial
@@ -391,11 +395,8 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
       if (it > 0 && !(ok = mbar_wait_warp(ds_read, (it - 1) & 1, abort_flag))) break;
       tc_fence_after();
       const float4* d4 = reinterpret_cast<const float4*>(vec + 128 + 64 * g);
-      // dS^T for 32 query columns at a time: to shared memory (the dQ MMA's
-      // A operand) and, packed as bf16 pairs over the first 32 of this group's
-      // dP^T columns, to tensor memory (the dK MMA's A operand).  The packed
-      // columns of half h are [16h, 16h + 16): half 1 reads columns 32..63
-      // before nothing below column 32 is written again.
+      // dS^T for 32 query columns at a time into the shared-memory dS tile,
+      // the A operand of both dQ (read MN-major) and dK (read K-major).
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         uint32_t dpr[32];
@@ -417,11 +418,9 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
           }
           st_shared_v4(sDSg + sw128_offset(r, 4 * h + ch), pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
         }
-        tmem_st16(tB + 16 * h, pk);
       }
-      tmem_st_wait();
       mbar_arrive(&v_empty[it % VS]);   // this thread is done with the LSE/D vectors
-      tc_fence_before();                // dP^T read, dS^T written (tensor memory)
+      tc_fence_before();                // dP^T has been read (its columns may be overwritten)
       fence_proxy_async_smem();         // dS^T visible to the tensor core (shared memory)
       mbar_arrive(ds_full);
     }

@@ -356,6 +356,7 @@ attn::BwdParams bwd_params(const BwdSetup& su, int64_t N, int64_t H, int64_t H_k
                            const uint8_t* mask) {
   attn::BwdParams prm;
   prm.mask = mask;
+  prm.dq_acc = nullptr;
   prm.h = int(H);
   prm.h_kv = int(H_kv);
   prm.group = int(H / H_kv);
@@ -505,7 +506,8 @@ int fused_main_impl(const void* Q, const void* K, const void* V, const void* dO,
       !make_map(&mdo, dO, su.bh, N, d) || !make_map(&mdk, dK, bhkv, N, d) || !make_map(&mdv, dV, bhkv, N, d) ||
       !make_map_f32_acc(&macc, dq_acc, su.bh, N, su.npad, d))
     return ATTN_ERR_LAUNCH;
-  const attn::BwdParams prm = bwd_params(su, N, H, H_kv, scale, mask);
+  attn::BwdParams prm = bwd_params(su, N, H, H_kv, scale, mask);
+  prm.dq_acc = dq_acc;
   const bool sparse = mask != nullptr;
   const int grid = int(bhkv * prm.n_tiles);
   cudaStream_t st = static_cast<cudaStream_t>(stream);

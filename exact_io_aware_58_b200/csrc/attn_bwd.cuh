@@ -89,6 +89,7 @@ struct BwdParams {
   float scale;
   float scale_log2;
   const uint8_t* mask;    // block-sparse only: [B*H][nt][nt], 1 = query tile attends key tile
+  float* dq_acc;          // fused backward only: [B*H][npad][D] fp32 accumulator of dQ / scale
 };
 
 // Selection over a linear range [0, hi): sel(L) != 0 marks the visited items.

@@ -74,6 +74,10 @@ struct FusedCfg {
   static constexpr int kOS = (D == 128) ? 1 : 3;
   static constexpr int kVS = 2;                             // (LSE2, D) vector ring
   static constexpr int kStageBlocks = 2;                    // staging ring of [128][32] fp32 blocks
+  // 32-column chunks of each dQ partial added straight from registers with
+  // vector reductions instead of through the staging ring (measured: at
+  // D = 64 one of the two chunks that way is faster, at D = 128 none).
+  static constexpr int kRedChunks = (D == 64) ? 1 : 0;
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kTileBytes;
   static constexpr int kOffQ = 2 * kTileBytes;
@@ -464,6 +468,7 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
     // wait must not make one warp leave alone: the first barrier of every
     // iteration ANDs the warps' status and they all stop together.
     int Lsel = SPARSE ? sel_next(sel, -1, n_all) : 0;
+    uint32_t pos = 0;                         // chunks staged so far: position in the block ring
     for (int it = 0; it < n_it; ++it) {
       const int L = SPARSE ? Lsel : it;
       if (SPARSE) Lsel = sel_next(sel, Lsel, n_all);
@@ -481,9 +486,20 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         tc_fence_before();
         mbar_arrive(dq_free);                 // the partial's TMEM columns are free
       }
+      // the last kRed chunks go straight from registers with vector reductions
+      constexpr int kRed = C::kRedChunks;
+      static_assert(kRed < NC, "at least one chunk goes through the staging ring");
+      if (ok && qrow + r < prm.n) {
+        float* dst = prm.dq_acc + (size_t(bq) * size_t(prm.npad) + size_t(qrow + r)) * D;
+#pragma unroll
+        for (int c = NC - kRed; c < NC; ++c)
+#pragma unroll
+          for (int m = 0; m < 8; ++m)
+            red_add_v4(dst + 32 * c + 4 * m, a[c][4 * m], a[c][4 * m + 1], a[c][4 * m + 2], a[c][4 * m + 3]);
+      }
       bool go = true;
 #pragma unroll
-      for (int c = 0; c < NC; ++c) {          // chunk c goes through staging block c % 2
+      for (int c = 0; c < NC - kRed; ++c, ++pos) {   // chunk c goes through staging block pos % 2
         // the block was last read by the reduce issued two chunks ago
         if (leader) bulk_wait_group_read1();
         if (c == 0) {
@@ -491,7 +507,7 @@ attn_bwd_fused_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_con
         } else {
           named_barrier_sync(3, 128);
         }
-        uint8_t* blk = stage + (c & 1) * C::kBlockBytes;
+        uint8_t* blk = stage + (pos & 1) * C::kBlockBytes;
         stage_row32(smem_u32(blk), r, a[c]);
         fence_proxy_async_smem();
         named_barrier_sync(3, 128);

@@ -11,7 +11,11 @@
 #include <cstdint>
 #include <cstdarg>
 #include <cstdio>
+#include <map>
 #include <mutex>
+#include <queue>
+#include <tuple>
+#include <vector>
 
 #include <cuda.h>
 #include <cuda_runtime.h>
@@ -122,6 +126,8 @@ bool make_map_f32_acc(CUtensorMap* m, const void* base, int64_t bh, int64_t n, i
   return true;
 }
 
+constexpr int64_t kNumSMs = 148;   // B200: sizes the persistent grids and the automatic split count
+
 bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int check_sizes(int64_t B, int64_t H, int64_t N, int64_t d) {
@@ -155,12 +161,12 @@ int set_smem(const void* kern, int bytes) {
 }
 
 template <int D, bool CAUSAL, bool SPARSE, bool O32 = false>
-int launch_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const CUtensorMap& o,
-               const attn::FwdParams& prm, int grid, cudaStream_t st) {
+int launch_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const attn::FwdParams& prm,
+               int grid, cudaStream_t st) {
   auto kern = attn::attn_fwd_kernel<D, CAUSAL, SPARSE, O32>;
   constexpr int smem = attn::FwdCfg<D>::kSmemBytes;
   if (set_smem(reinterpret_cast<const void*>(kern), smem) != ATTN_OK) return ATTN_ERR_LAUNCH;
-  kern<<<grid, attn::FwdCfg<D>::kThreads, smem, st>>>(q, k, v, o, prm);
+  kern<<<grid, attn::FwdCfg<D>::kThreads, smem, st>>>(q, k, v, prm);
   return launch_status();
 }
 
@@ -252,6 +258,73 @@ extern "C" {
 
 namespace {
 
+// Grid size and dealing order of the persistent forward.  A causal item of
+// query block m visits min(nt, 2m + 2) key tiles, so items differ in cost; the
+// items are dealt in rounds of one per CTA, and the pair (grid size, plain or
+// snake order) that gives the smallest predicted makespan -- the largest sum
+// of item costs on one CTA, each item also charged a fixed 3 key tiles for its
+// set-up and output -- is chosen once per shape and cached, unless one CTA per
+// item (scheduled greedily by the hardware) is predicted to finish first.
+// Non-causal items all cost the same; block-sparse costs depend on the mask
+// (device data), so both use the plain order on every SM.
+struct FwdSched {
+  int grid;
+  int snake;
+};
+
+FwdSched fwd_schedule(int64_t bh, int64_t n_mblk, int64_t nt, bool causal, bool sparse) {
+  const int64_t items = bh * n_mblk;
+  if (items <= kNumSMs) return {int(items), 0};
+  if (!causal || sparse) return {int(kNumSMs), 0};
+  if (items > 65536) return {int(kNumSMs), 1};
+  static std::mutex mu;
+  static std::map<std::tuple<int64_t, int64_t, int64_t>, FwdSched> cache;
+  const auto key = std::make_tuple(bh, n_mblk, nt);
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto f = cache.find(key);
+    if (f != cache.end()) return f->second;
+  }
+  constexpr int64_t kFixed = 3;
+  // One CTA per item (grid = items): the hardware hands each SM the next item
+  // when it frees up (greedy, in item order), and each item also pays the
+  // set-up and drain that the persistent loop overlaps (about one key tile).
+  FwdSched best{int(items), 0};
+  int64_t best_cost = 0;
+  {
+    std::priority_queue<int64_t, std::vector<int64_t>, std::greater<int64_t>> sm;
+    for (int64_t c = 0; c < kNumSMs; ++c) sm.push(0);
+    for (int64_t i = 0; i < items; ++i) {
+      const int64_t m = n_mblk - 1 - i % n_mblk;
+      const int64_t t = sm.top() + std::min(nt, 2 * m + 2) + kFixed + 1;
+      sm.pop();
+      sm.push(t);
+      best_cost = std::max(best_cost, t);
+    }
+  }
+  std::vector<int64_t> load(size_t(kNumSMs), 0);
+  for (int64_t g = kNumSMs; g >= kNumSMs - 28; --g) {
+    for (int snake = 0; snake < 2; ++snake) {
+      std::fill(load.begin(), load.begin() + g, 0);
+      for (int64_t i = 0; i < items; ++i) {
+        const int64_t r = i / g;
+        int64_t c = i - r * g;
+        if (snake && (r & 1)) c = g - 1 - c;
+        const int64_t m = n_mblk - 1 - i % n_mblk;
+        load[size_t(c)] += std::min(nt, 2 * m + 2) + kFixed;
+      }
+      const int64_t cost = *std::max_element(load.begin(), load.begin() + g);
+      if (cost < best_cost) {
+        best_cost = cost;
+        best = {int(g), snake};
+      }
+    }
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  cache[key] = best;
+  return best;
+}
+
 int fwd_impl(const void* Q, const void* K, const void* V, void* O, float* LSE, const uint8_t* mask, int64_t B,
              int64_t H, int64_t H_kv, int64_t N, int64_t d, int causal, float scale, void* stream,
              float* O32 = nullptr) {
@@ -264,11 +337,11 @@ int fwd_impl(const void* Q, const void* K, const void* V, void* O, float* LSE, c
       (O32 && !aligned16(O32)))
     return ATTN_ERR_MISALIGNED;
   const int64_t bh = B * H, bhkv = B * H_kv;
-  CUtensorMap mq, mk, mv, mo;
-  if (!make_map(&mq, Q, bh, N, d) || !make_map(&mk, K, bhkv, N, d) || !make_map(&mv, V, bhkv, N, d) ||
-      !make_map(&mo, O, bh, N, d))
+  CUtensorMap mq, mk, mv;
+  if (!make_map(&mq, Q, bh, N, d) || !make_map(&mk, K, bhkv, N, d) || !make_map(&mv, V, bhkv, N, d))
     return ATTN_ERR_LAUNCH;
   attn::FwdParams prm;
+  prm.o = static_cast<__nv_bfloat16*>(O);
   prm.lse = LSE;
   prm.n = int(N);
   prm.n_mblk = int((N + 255) / 256);
@@ -280,15 +353,19 @@ int fwd_impl(const void* Q, const void* K, const void* V, void* O, float* LSE, c
   prm.nt = int((N + 127) / 128);
   prm.o32 = O32;
   const bool sparse = mask != nullptr;
-  const int64_t grid = bh * prm.n_mblk;
-  if (grid > INT32_MAX) return ATTN_ERR_INVALID_ARG;
+  const int64_t items = bh * prm.n_mblk;
+  if (items > INT32_MAX) return ATTN_ERR_INVALID_ARG;
+  prm.n_items = int(items);
+  const FwdSched sched = fwd_schedule(bh, prm.n_mblk, prm.nt, causal != 0, sparse);
+  prm.snake = sched.snake;
+  const int grid = sched.grid;   // persistent: at most one CTA per SM
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (O32)
-    return d == 128 ? (causal ? launch_fwd<128, true, false, true>(mq, mk, mv, mo, prm, int(grid), st)
-                              : launch_fwd<128, false, false, true>(mq, mk, mv, mo, prm, int(grid), st))
-                    : (causal ? launch_fwd<64, true, false, true>(mq, mk, mv, mo, prm, int(grid), st)
-                              : launch_fwd<64, false, false, true>(mq, mk, mv, mo, prm, int(grid), st));
-  return ATTN_DISPATCH(launch_fwd, mq, mk, mv, mo, prm, int(grid), st);
+    return d == 128 ? (causal ? launch_fwd<128, true, false, true>(mq, mk, mv, prm, grid, st)
+                              : launch_fwd<128, false, false, true>(mq, mk, mv, prm, grid, st))
+                    : (causal ? launch_fwd<64, true, false, true>(mq, mk, mv, prm, grid, st)
+                              : launch_fwd<64, false, false, true>(mq, mk, mv, prm, grid, st));
+  return ATTN_DISPATCH(launch_fwd, mq, mk, mv, prm, grid, st);
 }
 
 }  // namespace
@@ -678,7 +755,6 @@ ATTN_EXPORT int attn_fwd_fp8(const void* Q8, const void* K8, const void* V8, voi
 // ---------------------------------------------------------------------------
 namespace {
 
-constexpr int64_t kNumSMs = 148;   // B200: sizes the persistent grid and the automatic split count
 constexpr int64_t kMaxSplits = 256;
 static_assert(kMaxSplits * 4 <= attn::kKvcMaxParts, "the merge kernel holds every partial's LSE in shared memory");
 

@@ -8,15 +8,26 @@
 // kept, the partial output is rescaled by exp(m_old - m_new) when the max
 // grows, and only O and one statistic per row (LSE) are written out.
 //
-// B200 mapping (one CTA = two 128-row query tiles of one head, 320 threads):
-//   warp 9      TMA producer: Q0, Q1 once, then K_j / V_j 128-row tiles into a
-//               ring of shared-memory slots (128-byte swizzle).
+// B200 mapping: a persistent grid of at most one CTA per SM (320 threads).  A
+// work item is two 128-row query tiles of one head; items are ordered
+// heads-major, heaviest causal blocks first within a head (so that a head's
+// K/V stays in L2 while its items run), and dealt out in rounds of one item
+// per CTA (every other round in reverse when that balances better).  All
+// roles walk the same item sequence and their barrier phases run on across
+// items, so the next item's Q load and first QK^T products overlap the
+// current item's last softmax and its output stores.
+//   warp 9      TMA producer: per item Q0, Q1, then K_j / V_j 128-row tiles
+//               into a ring of shared-memory slots (128-byte swizzle) that
+//               runs on across items.
 //   warp 8      MMA issuer (one thread): S_t = Q_t K_j^T and O_t += P_t V_j as
 //               tcgen05.mma with fp32 accumulators in tensor memory (TMEM).
 //   warps 0-3   softmax for query tile 0, warps 4-7 for tile 1: each thread owns
 //               one query row (= one TMEM lane), so the row max and sum need no
 //               shuffles.  P is rounded to bf16 and written back into TMEM over
 //               the upper half of S, where the PV MMA reads it as its A operand.
+//               At the end of an item each thread writes its normalised O row
+//               (and LSE) straight to global memory, so that the Q slots are
+//               free for the next item as soon as its last QK^T is done.
 // The issue order PV_t(j-1), S_t(j) lets the tensor core run one tile's GEMMs
 // while the other tile's softmax runs (ping-pong between the two tiles).
 //
@@ -34,6 +45,7 @@ constexpr float kRescaleLog2 = 8.0f;
 constexpr float kLn2 = 0.6931471805599453f;
 
 struct FwdParams {
+  __nv_bfloat16* o;    // [B*H][N][D] output
   float* lse;          // [B*H][N] natural-log LSE
   int n;               // sequence length N
   int n_mblk;          // number of 256-row query blocks per head
@@ -44,7 +56,17 @@ struct FwdParams {
   const uint8_t* mask; // block-sparse only: [B*H][nt][nt], 1 = query tile attends key tile
   int nt;              // ceil(N / 128)
   float* o32;          // O32 instances only: [B*H][N][D] fp32 copy of the normalised O
+  int n_items;         // B*H*n_mblk work items
+  int snake;           // 1: odd rounds of grid-size items are dealt to the CTAs in reverse
 };
+
+// The items of round r (items [r*G, r*G + G), G = grid size) go one per CTA;
+// with `snake`, odd rounds go in reverse CTA order, which pairs heavy causal
+// blocks with light ones (the host picks the order and G that balance best).
+__device__ __forceinline__ int fwd_round_item(int r, int G, int snake) {
+  const int pos = (snake && (r & 1)) ? G - 1 - int(blockIdx.x) : int(blockIdx.x);
+  return r * G + pos;
+}
 
 // Key tiles selected for the (up to) two 128-row query tiles of a CTA: bit t of
 // flags(j) says query tile t attends key tile j.  Every role scans the same
@@ -83,55 +105,71 @@ struct FwdCfg {
   static constexpr int kOffQ = 0;
   static constexpr int kOffKV = 2 * kTileBytes;
   static constexpr int kOffBar = kOffKV + kSlots * kTileBytes;
-  static constexpr int kNumBars = 2 + 2 * kSlots + 2 + 2 + 2 + 1;
+  static constexpr int kNumBars = 2 + 2 * kSlots + 2 + 2 + 2 + 2 + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;   // + slack for 1024-byte alignment
 };
+
+// Work item -> (query head, first query row, key tiles that may be visible,
+// selection, key tiles visited).  Every role evaluates the same function.
+struct FwdItem {
+  int bh, bkv, m0, kv_hi, nkv;
+  TileSelect sel;
+};
+
+template <bool CAUSAL, bool SPARSE>
+__device__ __forceinline__ FwdItem fwd_item(const FwdParams& prm, int item) {
+  FwdItem w;
+  w.bh = item / prm.n_mblk;
+  w.bkv = (w.bh / prm.h) * prm.h_kv + (w.bh % prm.h) / prm.group;
+  const int m_blk = prm.n_mblk - 1 - (item % prm.n_mblk);   // heaviest causal blocks of a head first
+  w.m0 = m_blk * 256;
+  const int n_kv_total = (prm.n + 127) >> 7;
+  w.kv_hi = CAUSAL ? min(n_kv_total, (w.m0 >> 7) + 2) : n_kv_total;
+  w.sel = TileSelect{nullptr, nullptr};
+  if (SPARSE) {
+    const int qt0 = w.m0 >> 7;
+    w.sel.r0 = prm.mask + (size_t(w.bh) * prm.nt + qt0) * prm.nt;
+    w.sel.r1 = (qt0 + 1 < prm.nt) ? w.sel.r0 + prm.nt : nullptr;
+  }
+  w.nkv = SPARSE ? w.sel.count(w.kv_hi) : w.kv_hi;
+  return w;
+}
 
 // O32: also write the normalised rows in fp32 to prm.o32 (a separate
 // instance, so the bf16-only instances are compiled without it).
 template <int D, bool CAUSAL, bool SPARSE, bool O32 = false>
 __global__ void __launch_bounds__(320, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                const FwdParams prm) {
+                const __grid_constant__ CUtensorMap tm_v, const FwdParams prm) {
   using C = FwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBar);
-  uint64_t* q_full = bars;
-  uint64_t* kv_full = q_full + 2;
+  uint64_t* q_full = bars;                  // Q0, Q1 of the current item landed
+  uint64_t* q_empty = q_full + 1;           // the item's last QK^T products are done: Q slots free
+  uint64_t* kv_full = q_empty + 1;
   uint64_t* kv_empty = kv_full + C::kSlots;
-  uint64_t* s_full = kv_empty + C::kSlots;
-  uint64_t* p_full = s_full + 2;
-  uint64_t* o_full = p_full + 2;
-  uint64_t* drain = o_full + 2;
+  uint64_t* s_full = kv_empty + C::kSlots;  // [2] S_t in TMEM
+  uint64_t* p_full = s_full + 2;            // [2] P_t written back (128 arrivals)
+  uint64_t* o_full = p_full + 2;            // [2] the item's O_t complete
+  uint64_t* o_free = o_full + 2;            // [2] O_t read out by the epilogue (128 arrivals)
+  uint64_t* drain = o_free + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int n = prm.n;
-  const int bh = blockIdx.x / prm.n_mblk;                                      // query head
-  const int bkv = (bh / prm.h) * prm.h_kv + (bh % prm.h) / prm.group;          // its key/value head
-  const int m_blk = prm.n_mblk - 1 - (blockIdx.x % prm.n_mblk);   // heaviest causal blocks first
-  const int m0 = m_blk * 256;
-  const int n_kv_total = (n + 127) >> 7;
-  const int kv_hi = CAUSAL ? min(n_kv_total, (m0 >> 7) + 2) : n_kv_total;   // key tiles [0, kv_hi) may be visible
-  TileSelect sel{nullptr, nullptr};
-  if (SPARSE) {
-    const int qt0 = m0 >> 7;
-    sel.r0 = prm.mask + (size_t(bh) * prm.nt + qt0) * prm.nt;
-    sel.r1 = (qt0 + 1 < prm.nt) ? sel.r0 + prm.nt : nullptr;
-  }
-  const int nkv = SPARSE ? sel.count(kv_hi) : kv_hi;   // key tiles this CTA visits
 
   if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     for (int t = 0; t < 2; ++t) {
-      mbar_init(&q_full[t], 1);
       mbar_init(&s_full[t], 1);
       mbar_init(&p_full[t], 128);
       mbar_init(&o_full[t], 1);
+      mbar_init(&o_free[t], 128);
     }
     for (int s = 0; s < C::kSlots; ++s) {
       mbar_init(&kv_full[s], 1);
@@ -149,7 +187,6 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     tma_prefetch_desc(&tm_q);
     tma_prefetch_desc(&tm_k);
     tma_prefetch_desc(&tm_v);
-    tma_prefetch_desc(&tm_o);
   }
   tc_fence_before();
   __syncthreads();
@@ -159,36 +196,39 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   if (warp == C::kWarpLoad) {
     // ------------------------------------------------------------------ TMA
     if (lane == 0) {
-      // A CTA that visits no key tile (block-sparse) loads nothing: its Q slots
-      // are the staging area of the zero output it writes.
-      for (int t = 0; t < 2 && nkv > 0; ++t) {
-        mbar_arrive_expect_tx(&q_full[t], C::kTileBytes);
-        for (int b = 0; b < C::kNumBlk; ++b)
-          tma_load_3d(&tm_q, &q_full[t], smem + C::kOffQ + t * C::kTileBytes + b * C::kBlockBytes,
-                      b * 64, m0 + 128 * t, bh);
-      }
-      int issued = 0;
+      int issued = 0;    // K/V tiles loaded (ring position)
+      int qn = 0;        // items whose Q was loaded
       bool ok = true;
-      int jsel = SPARSE ? sel.next(-1, kv_hi) : 0;
-      for (int it = 0; it < 2 * nkv; ++it) {
-        const int slot = it % C::kSlots;
-        const int use = it / C::kSlots;
-        if (use > 0 && !mbar_wait(&kv_empty[slot], (use - 1) & 1, abort_flag)) { ok = false; break; }
-        const CUtensorMap* tm = (it & 1) ? &tm_v : &tm_k;
-        const int j = SPARSE ? jsel : (it >> 1);
-        if (SPARSE && (it & 1)) jsel = sel.next(jsel, kv_hi);
-        mbar_arrive_expect_tx(&kv_full[slot], C::kTileBytes);
-        for (int b = 0; b < C::kNumBlk; ++b)
-          tma_load_3d(tm, &kv_full[slot], smem + C::kOffKV + slot * C::kTileBytes + b * C::kBlockBytes,
-                      b * 64, 128 * j, bkv);
-        ++issued;
+      for (int rr = 0, item = fwd_round_item(0, gridDim.x, prm.snake); rr * int(gridDim.x) < prm.n_items && ok;
+           item = fwd_round_item(++rr, gridDim.x, prm.snake)) {
+        if (item >= prm.n_items) continue;
+        const FwdItem w = fwd_item<CAUSAL, SPARSE>(prm, item);
+        if (w.nkv == 0) continue;   // block-sparse: nothing selected, nothing loaded
+        // the previous item's last QK^T products must be done with the Q slots
+        if (qn > 0 && !(ok = mbar_wait(q_empty, (qn - 1) & 1, abort_flag))) break;
+        mbar_arrive_expect_tx(q_full, 2 * C::kTileBytes);
+        for (int t = 0; t < 2; ++t)
+          for (int b = 0; b < C::kNumBlk; ++b)
+            tma_load_3d(&tm_q, q_full, smem + C::kOffQ + t * C::kTileBytes + b * C::kBlockBytes, b * 64,
+                        w.m0 + 128 * t, w.bh);
+        ++qn;
+        int jsel = SPARSE ? w.sel.next(-1, w.kv_hi) : 0;
+        for (int kk = 0; kk < 2 * w.nkv; ++kk) {
+          const int slot = issued % C::kSlots;
+          const int use = issued / C::kSlots;
+          if (use > 0 && !(ok = mbar_wait(&kv_empty[slot], (use - 1) & 1, abort_flag))) break;
+          const CUtensorMap* tm = (kk & 1) ? &tm_v : &tm_k;
+          const int j = SPARSE ? jsel : (kk >> 1);
+          if (SPARSE && (kk & 1)) jsel = w.sel.next(jsel, w.kv_hi);
+          mbar_arrive_expect_tx(&kv_full[slot], C::kTileBytes);
+          for (int b = 0; b < C::kNumBlk; ++b)
+            tma_load_3d(tm, &kv_full[slot], smem + C::kOffKV + slot * C::kTileBytes + b * C::kBlockBytes,
+                        b * 64, 128 * j, w.bkv);
+          ++issued;
+        }
       }
-      (void)ok;
       // No copy may still be landing in shared memory when the CTA leaves.
-      if (nkv > 0) {
-        mbar_wait(&q_full[0], 0, abort_flag, false);
-        mbar_wait(&q_full[1], 0, abort_flag, false);
-      }
+      if (qn > 0) mbar_wait(q_full, (qn - 1) & 1, abort_flag, false);
       for (int it = max(0, issued - C::kSlots); it < issued; ++it)
         mbar_wait(&kv_full[it % C::kSlots], (it / C::kSlots) & 1, abort_flag, false);
     }
@@ -200,7 +240,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       constexpr uint32_t kIdescPV = idesc_bf16(128, D, false, true);
       const uint32_t sQ = smem_u32(smem + C::kOffQ);
       const uint32_t sKV = smem_u32(smem + C::kOffKV);
-      int it = 0;
+      int it = 0;        // K/V tiles consumed (ring position)
       auto wait_kv = [&](int& slot) -> bool {
         slot = it % C::kSlots;
         const bool r = mbar_wait(&kv_full[slot], (it / C::kSlots) & 1, abort_flag);
@@ -228,43 +268,58 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                  (acc || kk > 0) ? 1u : 0u);
       };
 
-      bool ok = nkv > 0 && mbar_wait(&q_full[0], 0, abort_flag) && mbar_wait(&q_full[1], 0, abort_flag);
-      if (ok) {
+      bool ok = true;
+      int qn = 0;        // items processed
+      int pc = 0;        // key tiles processed over all items (S/P barrier phases)
+      for (int rr = 0, item = fwd_round_item(0, gridDim.x, prm.snake); rr * int(gridDim.x) < prm.n_items && ok;
+           item = fwd_round_item(++rr, gridDim.x, prm.snake)) {
+        if (item >= prm.n_items) continue;
+        const int nkv = fwd_item<CAUSAL, SPARSE>(prm, item).nkv;
+        if (nkv == 0) continue;
+        // PV of key tile jl (of this item) for query tile t; the item's first
+        // PV overwrites O_t, which the previous item's epilogue must have read.
+        auto pv = [&](int t, int jl, int vslot) -> bool {
+          if (!mbar_wait(&p_full[t], (pc + jl) & 1, abort_flag)) return false;
+          if (jl == 0 && qn > 0 && !mbar_wait(&o_free[t], (qn - 1) & 1, abort_flag)) return false;
+          tc_fence_after();
+          issue_pv(t, vslot, jl > 0);
+          return true;
+        };
         int ks;
-        ok = wait_kv(ks);
-        if (ok) {
-          tc_fence_after();
-          issue_s(0, ks);
-          mma_commit(&s_full[0]);
-          issue_s(1, ks);
-          mma_commit(&s_full[1]);
-          mma_commit(&kv_empty[ks]);
-        }
-      }
-      for (int j = 1; j < nkv && ok; ++j) {
-        int vs, ks;
-        if (!(ok = wait_kv(vs))) break;
+        if (!(ok = mbar_wait(q_full, qn & 1, abort_flag))) break;
         if (!(ok = wait_kv(ks))) break;
-        for (int t = 0; t < 2; ++t) {
-          if (!(ok = mbar_wait(&p_full[t], (j - 1) & 1, abort_flag))) break;
-          tc_fence_after();
-          issue_pv(t, vs, j - 1 > 0);
-          if (t == 1) mma_commit(&kv_empty[vs]);
-          issue_s(t, ks);
-          mma_commit(&s_full[t]);
+        tc_fence_after();
+        issue_s(0, ks);
+        mma_commit(&s_full[0]);
+        issue_s(1, ks);
+        mma_commit(&s_full[1]);
+        mma_commit(&kv_empty[ks]);
+        if (nkv == 1) mma_commit(q_empty);
+        for (int j = 1; j < nkv && ok; ++j) {
+          int vs;
+          if (!(ok = wait_kv(vs))) break;
+          if (!(ok = wait_kv(ks))) break;
+          for (int t = 0; t < 2; ++t) {
+            if (!(ok = pv(t, j - 1, vs))) break;
+            if (t == 1) mma_commit(&kv_empty[vs]);
+            issue_s(t, ks);
+            mma_commit(&s_full[t]);
+          }
+          if (!ok) break;
+          mma_commit(&kv_empty[ks]);
+          if (j == nkv - 1) mma_commit(q_empty);   // the item's last QK^T: Q slots free
         }
-        if (ok) mma_commit(&kv_empty[ks]);
-      }
-      if (ok) {
+        if (!ok) break;
         int vs;
-        ok = wait_kv(vs);
+        if (!(ok = wait_kv(vs))) break;
         for (int t = 0; t < 2 && ok; ++t) {
-          if (!(ok = mbar_wait(&p_full[t], (nkv - 1) & 1, abort_flag))) break;
-          tc_fence_after();
-          issue_pv(t, vs, nkv - 1 > 0);
+          if (!(ok = pv(t, nkv - 1, vs))) break;
           mma_commit(&o_full[t]);
         }
-        if (ok) mma_commit(&kv_empty[vs]);
+        if (!ok) break;
+        mma_commit(&kv_empty[vs]);
+        pc += nkv;
+        ++qn;
       }
       // Every MMA issued so far must finish before tensor memory is released.
       mma_commit(drain);
@@ -276,153 +331,163 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int t = warp >> 2;
     const int qw = warp & 3;
     const int r = qw * 32 + lane;           // row inside the tile = TMEM lane
-    const int i = m0 + 128 * t + r;         // global query row
     const uint32_t lane_base = uint32_t(qw * 32) << 16;
     const uint32_t tS = tmem + lane_base + (t ? C::kColS1 : C::kColS0);
     const uint32_t tP = tS + C::kColPOff;
     const uint32_t tO = tmem + lane_base + (t ? C::kColO1 : C::kColO0);
     const float c = prm.scale_log2;
-    float m_ref = -INFINITY;
-    float l = 0.f;
     bool ok = true;
-
-    int jsel = SPARSE ? sel.next(-1, kv_hi) : 0;
-    for (int jj = 0; jj < nkv; ++jj) {
-      // jj counts visited tiles (barrier phases); j is the key tile itself
-      const int j = SPARSE ? jsel : jj;
-      const bool tile_on = SPARSE ? ((sel.flags(j) >> t) & 1u) != 0 : true;
-      if (SPARSE) jsel = sel.next(jsel, kv_hi);
-      if (!(ok = mbar_wait_warp(&s_full[t], jj & 1, abort_flag))) break;
-      tc_fence_after();
-      float s[128];
-      {
-        uint32_t a[32], b[32], e[32], f[32];
-        tmem_ld32(tS + 0, a);
-        tmem_ld32(tS + 32, b);
-        tmem_ld32(tS + 64, e);
-        tmem_ld32(tS + 96, f);
-        tmem_ld_wait(a);
-        reg_fence32(b);
-        reg_fence32(e);
-        reg_fence32(f);
+    int qn = 0, pc = 0;
+    for (int rr = 0, item = fwd_round_item(0, gridDim.x, prm.snake); rr * int(gridDim.x) < prm.n_items && ok;
+           item = fwd_round_item(++rr, gridDim.x, prm.snake)) {
+        if (item >= prm.n_items) continue;
+      const FwdItem w = fwd_item<CAUSAL, SPARSE>(prm, item);
+      const int m0 = w.m0;
+      const int i = m0 + 128 * t + r;         // global query row
+      const size_t row = size_t(w.bh) * size_t(n) + size_t(i);
+      if (w.nkv == 0) {
+        // block-sparse: a block that selected nothing: O = 0, LSE = -inf
+        if (i < n) {
+          uint4* dst = reinterpret_cast<uint4*>(prm.o + row * D);
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          s[k] = __uint_as_float(a[k]);
-          s[32 + k] = __uint_as_float(b[k]);
-          s[64 + k] = __uint_as_float(e[k]);
-          s[96 + k] = __uint_as_float(f[k]);
+          for (int k = 0; k < D / 8; ++k) dst[k] = make_uint4(0u, 0u, 0u, 0u);
+          if (O32) {
+            float4* d32 = reinterpret_cast<float4*>(prm.o32 + row * D);
+#pragma unroll
+            for (int k = 0; k < D / 4; ++k) d32[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+          prm.lse[row] = -INFINITY;
         }
+        continue;
       }
-      const bool need_mask = !tile_on || (CAUSAL && (128 * j + 127 > m0 + 128 * t)) || (128 * j + 128 > n);
-      if (need_mask) {
-        int limit = tile_on ? n - 1 - 128 * j : -1;     // a tile this query tile did not select: all masked
-        if (CAUSAL) limit = min(limit, i - 128 * j);
+      float m_ref = -INFINITY;
+      float l = 0.f;
+      int jsel = SPARSE ? w.sel.next(-1, w.kv_hi) : 0;
+      for (int jj = 0; jj < w.nkv; ++jj) {
+        // jj counts visited tiles (barrier phases); j is the key tile itself
+        const int j = SPARSE ? jsel : jj;
+        const bool tile_on = SPARSE ? ((w.sel.flags(j) >> t) & 1u) != 0 : true;
+        if (SPARSE) jsel = w.sel.next(jsel, w.kv_hi);
+        if (!(ok = mbar_wait_warp(&s_full[t], (pc + jj) & 1, abort_flag))) break;
+        tc_fence_after();
+        float s[128];
+        {
+          uint32_t a[32], b[32], e[32], f[32];
+          tmem_ld32(tS + 0, a);
+          tmem_ld32(tS + 32, b);
+          tmem_ld32(tS + 64, e);
+          tmem_ld32(tS + 96, f);
+          tmem_ld_wait(a);
+          reg_fence32(b);
+          reg_fence32(e);
+          reg_fence32(f);
 #pragma unroll
-        for (int k = 0; k < 128; ++k)
-          if (k > limit) s[k] = -INFINITY;
-      }
-      // Row max as 8 independent chains (a single 127-long dependency chain
-      // would leave the issue slots idle for its whole latency).
-      float mxp[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) mxp[u] = s[u];
-#pragma unroll
-      for (int k = 8; k < 128; k += 8)
-#pragma unroll
-        for (int u = 0; u < 8; ++u) mxp[u] = fmaxf(mxp[u], s[k + u]);
-      const float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
-                             fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
-      const float m_tile = mx * c;
-      float alpha = 1.f;
-      bool rescale = false;
-      if (m_tile > m_ref + kRescaleLog2) {
-        alpha = ex2(m_ref - m_tile);      // 0 when m_ref is still -inf
-        m_ref = m_tile;
-        rescale = (jj > 0);
-      }
-      l *= alpha;
-      const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
-      // P in 32-key chunks (16 packed columns each): a chunk's registers are
-      // free again as soon as it is stored, which keeps the loop spill-free.
-      float sump[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const float p0 = ex2(fmaf(s[32 * q + 2 * k], c, neg_m));
-          const float p1 = ex2(fmaf(s[32 * q + 2 * k + 1], c, neg_m));
-          sump[k & 3] += p0 + p1;
-          pk[k] = pack_bf16x2(p0, p1);
+          for (int k = 0; k < 32; ++k) {
+            s[k] = __uint_as_float(a[k]);
+            s[32 + k] = __uint_as_float(b[k]);
+            s[64 + k] = __uint_as_float(e[k]);
+            s[96 + k] = __uint_as_float(f[k]);
+          }
         }
-        tmem_st16(tP + 16 * q, pk);
-      }
-      l += (sump[0] + sump[1]) + (sump[2] + sump[3]);
-      if (__any_sync(0xffffffffu, rescale)) {
-        // O_t holds the sum through key tile j-1 (its last PV completed before S_t(j)).
-        const float a = rescale ? alpha : 1.f;
+        const bool need_mask = !tile_on || (CAUSAL && (128 * j + 127 > m0 + 128 * t)) || (128 * j + 128 > n);
+        if (need_mask) {
+          int limit = tile_on ? n - 1 - 128 * j : -1;     // a tile this query tile did not select: all masked
+          if (CAUSAL) limit = min(limit, i - 128 * j);
+#pragma unroll
+          for (int k = 0; k < 128; ++k)
+            if (k > limit) s[k] = -INFINITY;
+        }
+        // Row max as 8 independent chains (a single 127-long dependency chain
+        // would leave the issue slots idle for its whole latency).
+        float mxp[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) mxp[u] = s[u];
+#pragma unroll
+        for (int k = 8; k < 128; k += 8)
+#pragma unroll
+          for (int u = 0; u < 8; ++u) mxp[u] = fmaxf(mxp[u], s[k + u]);
+        const float mx = fmaxf(fmaxf(fmaxf(mxp[0], mxp[1]), fmaxf(mxp[2], mxp[3])),
+                               fmaxf(fmaxf(mxp[4], mxp[5]), fmaxf(mxp[6], mxp[7])));
+        const float m_tile = mx * c;
+        float alpha = 1.f;
+        bool rescale = false;
+        if (m_tile > m_ref + kRescaleLog2) {
+          alpha = ex2(m_ref - m_tile);      // 0 when m_ref is still -inf
+          m_ref = m_tile;
+          rescale = (jj > 0);
+        }
+        l *= alpha;
+        const float neg_m = (m_ref == -INFINITY) ? 0.f : -m_ref;
+        // P in 32-key chunks (16 packed columns each): a chunk's registers are
+        // free again as soon as it is stored, which keeps the loop spill-free.
+        float sump[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            const float p0 = ex2(fmaf(s[32 * q + 2 * k], c, neg_m));
+            const float p1 = ex2(fmaf(s[32 * q + 2 * k + 1], c, neg_m));
+            sump[k & 3] += p0 + p1;
+            pk[k] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(tP + 16 * q, pk);
+        }
+        l += (sump[0] + sump[1]) + (sump[2] + sump[3]);
+        if (__any_sync(0xffffffffu, rescale)) {
+          // O_t holds the sum through key tile j-1 (its last PV completed before S_t(j)).
+          const float a = rescale ? alpha : 1.f;
 #pragma unroll 1
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t o[32];
-          tmem_ld32(tO + cc * 32, o);
-          tmem_ld_wait(o);
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t o[32];
+            tmem_ld32(tO + cc * 32, o);
+            tmem_ld_wait(o);
 #pragma unroll
-          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * a);
-          tmem_st32(tO + cc * 32, o);
+            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * a);
+            tmem_st32(tO + cc * 32, o);
+          }
         }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&p_full[t]);
       }
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&p_full[t]);
-    }
+      if (!ok) break;
 
-    // ------------------------------------------------------------ epilogue
-    const bool any_tile = !SPARSE || nkv > 0;   // dense: every CTA visits at least one key tile
-    if (ok && any_tile) ok = mbar_wait_warp(&o_full[t], 0, abort_flag);
-    uint8_t* stage = smem + C::kOffQ + t * C::kTileBytes;   // Q_t is no longer read
-    if (ok) {
+      // ---------------------------------------------------------- epilogue
+      if (!(ok = mbar_wait_warp(&o_full[t], qn & 1, abort_flag))) break;
       tc_fence_after();
       // l == 0 only for rows that see no key at all (block-sparse): O = 0, LSE = -inf.
       const float inv_l = (SPARSE && !(l > 0.f)) ? 0.f : 1.f / l;
 #pragma unroll 1
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t o[32];
-        if (any_tile) {
-          tmem_ld32(tO + cc * 32, o);
-          tmem_ld_wait(o);
-        } else {
-#pragma unroll
-          for (int k = 0; k < 32; ++k) o[k] = 0u;
+        tmem_ld32(tO + cc * 32, o);
+        tmem_ld_wait(o);
+        if (cc == D / 32 - 1) {
+          tc_fence_before();
+          mbar_arrive(&o_free[t]);            // O_t has been read: the next item may overwrite it
         }
-        const uint32_t blk = cc >> 1;
+        if (i < n) {
+          uint4* dst = reinterpret_cast<uint4*>(prm.o + row * D + cc * 32);
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          const uint32_t w0 = pack_bf16x2(__uint_as_float(o[8 * ch + 0]) * inv_l, __uint_as_float(o[8 * ch + 1]) * inv_l);
-          const uint32_t w1 = pack_bf16x2(__uint_as_float(o[8 * ch + 2]) * inv_l, __uint_as_float(o[8 * ch + 3]) * inv_l);
-          const uint32_t w2 = pack_bf16x2(__uint_as_float(o[8 * ch + 4]) * inv_l, __uint_as_float(o[8 * ch + 5]) * inv_l);
-          const uint32_t w3 = pack_bf16x2(__uint_as_float(o[8 * ch + 6]) * inv_l, __uint_as_float(o[8 * ch + 7]) * inv_l);
-          const uint32_t chunk = (cc & 1) * 4 + ch;
-          st_shared_v4(smem_u32(stage) + blk * C::kBlockBytes + sw128_offset(r, chunk), w0, w1, w2, w3);
-        }
-        if (O32 && i < n) {
-          // the same normalised row in fp32, before the bf16 rounding
-          float4* dst = reinterpret_cast<float4*>(prm.o32 + (size_t(bh) * size_t(n) + size_t(i)) * D + cc * 32);
+          for (int ch = 0; ch < 4; ++ch)
+            dst[ch] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * ch + 0]) * inv_l, __uint_as_float(o[8 * ch + 1]) * inv_l),
+                                 pack_bf16x2(__uint_as_float(o[8 * ch + 2]) * inv_l, __uint_as_float(o[8 * ch + 3]) * inv_l),
+                                 pack_bf16x2(__uint_as_float(o[8 * ch + 4]) * inv_l, __uint_as_float(o[8 * ch + 5]) * inv_l),
+                                 pack_bf16x2(__uint_as_float(o[8 * ch + 6]) * inv_l, __uint_as_float(o[8 * ch + 7]) * inv_l));
+          if (O32) {
+            // the same normalised row in fp32, before the bf16 rounding
+            float4* d32 = reinterpret_cast<float4*>(prm.o32 + row * D + cc * 32);
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
-            dst[k] = make_float4(__uint_as_float(o[4 * k]) * inv_l, __uint_as_float(o[4 * k + 1]) * inv_l,
-                                 __uint_as_float(o[4 * k + 2]) * inv_l, __uint_as_float(o[4 * k + 3]) * inv_l);
+            for (int k = 0; k < 8; ++k)
+              d32[k] = make_float4(__uint_as_float(o[4 * k]) * inv_l, __uint_as_float(o[4 * k + 1]) * inv_l,
+                                   __uint_as_float(o[4 * k + 2]) * inv_l, __uint_as_float(o[4 * k + 3]) * inv_l);
+          }
         }
       }
-      if (i < n)
-        prm.lse[size_t(bh) * size_t(n) + size_t(i)] = (SPARSE && !(l > 0.f)) ? -INFINITY : (m_ref + __log2f(l)) * kLn2;
-    }
-    fence_proxy_async_smem();
-    named_barrier_sync(1 + t, 128);
-    // A store never starts past the last row (rows past N inside a box are dropped by TMA).
-    if (qw == 0 && lane == 0 && *abort_flag == 0 && m0 + 128 * t < n) {
-      for (int b = 0; b < C::kNumBlk; ++b) tma_store_3d(&tm_o, stage + b * C::kBlockBytes, b * 64, m0 + 128 * t, bh);
-      bulk_commit_group();
-      bulk_wait_group_read0();
+      if (i < n) prm.lse[row] = (SPARSE && !(l > 0.f)) ? -INFINITY : (m_ref + __log2f(l)) * kLn2;
+      pc += w.nkv;
+      ++qn;
     }
   }
 

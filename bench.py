@@ -16,8 +16,8 @@ the forward (halved under the causal mask) and 2.5x that for the backward.
 The other four workloads (tiny fwd+bwd, the outlier-row forward with both
 masks, the d = 64 training shape, the 100K-token causal forward) are measured
 in the same run under the key ``configs``; the deterministic backward, shared
-key/value heads, block-sparse selection, decode against a cache and FP8 have
-keys of their own.
+key/value heads, block-sparse selection, packed variable-length prefill,
+decode against a cache and FP8 have keys of their own.
 
 Multi-GPU: ``--gpus N`` starts N rank processes on this node (one GPU each)
 unless it is already running under a launcher that set WORLD_SIZE; every rank
@@ -333,6 +333,37 @@ def run_ours(args, rank, world, local_rank):
                   "fwdbwd_tflops": round(aggregate_tflops(3.5 * f_sparse, world, sf + sb), 2), "steps": n_s}
         del mask
 
+    # ------------------------------------- packed variable-length prefill
+    # 16 sequences of lengths drawn uniformly in [N/16, N] in one packed
+    # (total, H, d) buffer (cu_seqlens), causal, the long-batch heads and
+    # head dim; FLOPs counted per sequence (4 L^2 d per head, halved causal).
+    varlen = None
+    if not args.no_varlen:
+        gen = torch.Generator("cpu").manual_seed(rank_seed(77, rank))
+        lens = torch.randint(w.N // 16, w.N + 1, (16,), generator=gen).tolist()
+        cu = torch.tensor([0] + list(torch.cumsum(torch.tensor(lens), 0).tolist()), dtype=torch.int32)
+        total = int(cu[-1])
+        gv = torch.Generator(dev).manual_seed(rank_seed(78, rank))
+        qv, kv_, vv = (torch.randn((total, w.H, w.d), generator=gv, device=dev).mul_(w.std).to(torch.bfloat16)
+                       for _ in range(3))
+        ov = torch.empty_like(qv)
+        lv = torch.empty((w.H, total), dtype=torch.float32, device=dev)
+        cud = cu.to(dev)
+        f_var = sum(4.0 * L * L * w.d * w.H / 2 for L in lens)
+
+        def var_step(mark):
+            attn.attn_fwd_varlen(qv, kv_, vv, ov, lv, cud, causal, scale, stream)
+
+        n_v = max(3, min(args.steps, 5))
+        _, vseg = run_timed(var_step, n_v, args.warmup, clock, barrier, n_segments=1)
+        assert attn.attn_check_status(stream) == attn.ATTN_OK
+        tv = max_over_ranks(vseg, device=dev)[0]
+        varlen = {"workload": f"16 packed sequences, lengths uniform in [N/16, N] (total {total} tokens), "
+                              f"H={w.H}, d={w.d}, causal", "ms_fwd": round(tv, 3),
+                  "fwd_tflops": round(aggregate_tflops(f_var, world, tv), 2),
+                  "fwd_of_burst": round(aggregate_tflops(f_var, world, tv) / world / burst, 4), "steps": n_v}
+        del qv, kv_, vv, ov, lv
+
     # ------------------------------------------- decode against a KV cache
     # One new query row per head of the same batch against a cache of N rows
     # held in H_kv shared key/value heads: HBM-bound (each cache byte is used
@@ -599,6 +630,7 @@ def run_ours(args, rank, world, local_rank):
         "configs": configs,
         "gqa": gqa,
         "block_sparse": sparse,
+        "varlen": varlen,
         "kvcache": kvcache,
         "fp8": fp8,
         "gpu_launches": 4 * args.steps,      # attn_fwd + the three kernels of attn_bwd per timed step
@@ -822,6 +854,7 @@ def main():
     ap.add_argument("--gqa-kv-heads", type=int, default=8)
     ap.add_argument("--no-sparse", action="store_true", help="skip the block-sparse measurement")
     ap.add_argument("--no-det", action="store_true", help="skip the deterministic backward measurement")
+    ap.add_argument("--no-varlen", action="store_true", help="skip the packed variable-length prefill measurement")
     ap.add_argument("--no-configs", action="store_true", help="skip the other four workloads")
     ap.add_argument("--sparse-window", type=int, default=16)
     ap.add_argument("--sparse-sink", type=int, default=2)

@@ -30,7 +30,8 @@ ATTN_ERR_LAUNCH = -5
 ATTN_ERR_TIMEOUT = -6
 ATTN_ERR_DEVICE = -7
 
-EXPORTED = ("attn_fwd", "attn_fwd_f32out", "attn_fwd_gqa", "attn_fwd_blocksparse", "attn_bwd", "attn_bwd_gqa",
+EXPORTED = ("attn_fwd", "attn_fwd_f32out", "attn_fwd_gqa", "attn_fwd_blocksparse", "attn_fwd_varlen", "attn_bwd",
+            "attn_bwd_gqa",
             "attn_bwd_blocksparse", "attn_bwd_deterministic", "attn_bwd_workspace_bytes",
             "attn_bwd_deterministic_workspace_bytes", "attn_fwd_fp8", "attn_fwd_kvcache", "attn_fwd_kvcache_fp8",
             "attn_fwd_kvcache_splits", "attn_fwd_kvcache_workspace_bytes",
@@ -76,6 +77,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.attn_bwd_gqa.restype = i32
     lib.attn_fwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i32, f32, vp]
     lib.attn_fwd_blocksparse.restype = i32
+    lib.attn_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i32, f32, vp]
+    lib.attn_fwd_varlen.restype = i32
     lib.attn_bwd_blocksparse.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i32, f32,
                                          vp, ctypes.c_size_t, vp]
     lib.attn_bwd_blocksparse.restype = i32
@@ -265,6 +268,32 @@ def attn_fwd_blocksparse(Q, K, V, O, LSE, block_mask, causal: bool, scale: float
                                              Hk, N, d, int(bool(causal)), float(scale), _stream_handle(stream))
     if st != ATTN_OK:
         raise AttnError(st, "attn_fwd_blocksparse")
+
+
+def attn_fwd_varlen(Q, K, V, O, LSE, cu_seqlens, causal: bool, scale: float, stream=None) -> None:
+    """Packed sequences: Q, O (total, H, d), K, V (total, H_kv, d) bf16, LSE (H, total) fp32,
+    cu_seqlens int32 (n_seqs + 1,) token offsets, all on the current CUDA device."""
+    for name, t in (("Q", Q), ("K", K), ("V", V), ("O", O)):
+        if not t.is_cuda or t.dtype != torch.bfloat16 or t.dim() != 3 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor of shape (total, heads, d)")
+        _check_device(name, t)
+    total, H, d = Q.shape
+    if tuple(O.shape) != tuple(Q.shape):
+        raise ValueError("O must have Q's shape")
+    if K.shape != V.shape or K.shape[0] != total or K.shape[2] != d or K.shape[1] < 1 or H % K.shape[1] != 0:
+        raise ValueError(f"K, V have shapes {tuple(K.shape)}, {tuple(V.shape)}; expected (total, H_kv, d)")
+    if not LSE.is_cuda or LSE.dtype != torch.float32 or tuple(LSE.shape) != (H, total) or not LSE.is_contiguous():
+        raise ValueError("LSE must be a contiguous CUDA float32 tensor of shape (H, total)")
+    _check_device("LSE", LSE)
+    if not cu_seqlens.is_cuda or cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1 \
+            or cu_seqlens.numel() < 2 or not cu_seqlens.is_contiguous():
+        raise ValueError("cu_seqlens must be a contiguous CUDA int32 tensor of shape (n_seqs + 1,)")
+    _check_device("cu_seqlens", cu_seqlens)
+    st = load_library().attn_fwd_varlen(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), _ptr(LSE), _ptr(cu_seqlens),
+                                        cu_seqlens.numel() - 1, total, H, K.shape[1], d, int(bool(causal)),
+                                        float(scale), _stream_handle(stream))
+    if st != ATTN_OK:
+        raise AttnError(st, "attn_fwd_varlen")
 
 
 def attn_bwd_blocksparse(Q, K, V, O, dO, LSE, block_mask, dQ, dK, dV, causal: bool, scale: float, workspace,

@@ -128,6 +128,29 @@ bool make_map_f32_acc(CUtensorMap* m, const void* base, int64_t bh, int64_t n, i
 
 constexpr int64_t kNumSMs = 148;   // B200: sizes the persistent grids and the automatic split count
 
+// 3-D map over a packed [total][H][d] bf16 tensor (coordinates x, head,
+// token); box = 64 columns x 1 head x 128 tokens, 128-byte swizzle: the same
+// shared-memory tile as make_map's.  Tokens past `total` read as zeros.
+bool make_map_packed(CUtensorMap* m, const void* base, int64_t total, int64_t h, int64_t d) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) {
+    fail(ATTN_ERR_LAUNCH, "driver entry point cuTensorMapEncodeTiled unavailable");
+    return false;
+  }
+  const cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(h), cuuint64_t(total)};
+  const cuuint64_t strides[2] = {cuuint64_t(d * 2), cuuint64_t(h * d * 2)};
+  const cuuint32_t box[3] = {64, 1, 128};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    fail(ATTN_ERR_LAUNCH, "cuTensorMapEncodeTiled (packed) returned CUresult %lld", (long long)r);
+    return false;
+  }
+  return true;
+}
+
 bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int check_sizes(int64_t B, int64_t H, int64_t N, int64_t d) {
@@ -160,10 +183,10 @@ int set_smem(const void* kern, int bytes) {
               (long long)bytes);
 }
 
-template <int D, bool CAUSAL, bool SPARSE, bool O32 = false>
+template <int D, bool CAUSAL, bool SPARSE, bool O32 = false, bool VARLEN = false>
 int launch_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const attn::FwdParams& prm,
                int grid, cudaStream_t st) {
-  auto kern = attn::attn_fwd_kernel<D, CAUSAL, SPARSE, O32>;
+  auto kern = attn::attn_fwd_kernel<D, CAUSAL, SPARSE, O32, VARLEN>;
   constexpr int smem = attn::FwdCfg<D>::kSmemBytes;
   if (set_smem(reinterpret_cast<const void*>(kern), smem) != ATTN_OK) return ATTN_ERR_LAUNCH;
   kern<<<grid, attn::FwdCfg<D>::kThreads, smem, st>>>(q, k, v, prm);
@@ -340,7 +363,7 @@ int fwd_impl(const void* Q, const void* K, const void* V, void* O, float* LSE, c
   CUtensorMap mq, mk, mv;
   if (!make_map(&mq, Q, bh, N, d) || !make_map(&mk, K, bhkv, N, d) || !make_map(&mv, V, bhkv, N, d))
     return ATTN_ERR_LAUNCH;
-  attn::FwdParams prm;
+  attn::FwdParams prm = {};
   prm.o = static_cast<__nv_bfloat16*>(O);
   prm.lse = LSE;
   prm.n = int(N);
@@ -375,6 +398,45 @@ extern "C" {
 ATTN_EXPORT int attn_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int64_t B, int64_t H,
                          int64_t N, int64_t d, int causal, float scale, void* stream) {
   return fwd_impl(Q, K, V, O, LSE, nullptr, B, H, H, N, d, causal, scale, stream);
+}
+
+ATTN_EXPORT int attn_fwd_varlen(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                                const int32_t* cu_seqlens, int64_t n_seqs, int64_t total, int64_t H, int64_t H_kv,
+                                int64_t d, int causal, float scale, void* stream) {
+  if (n_seqs < 1 || total < 1 || H < 1) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  int s = check_heads(H, H_kv);
+  if (s != ATTN_OK) return s;
+  if ((s = check_scale(scale)) != ATTN_OK) return s;
+  // item counts (heads x 256-row blocks per sequence) and row indices must fit in 31 bits
+  if (n_seqs > INT32_MAX - 1 || total > INT32_MAX - 256 || H * ((total + 255) / 256 + n_seqs) > INT32_MAX)
+    return ATTN_ERR_INVALID_ARG;
+  if (!Q || !K || !V || !O || !LSE || !cu_seqlens) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE))
+    return ATTN_ERR_MISALIGNED;
+  if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return ATTN_ERR_MISALIGNED;
+  CUtensorMap mq, mk, mv;
+  if (!make_map_packed(&mq, Q, total, H, d) || !make_map_packed(&mk, K, total, H_kv, d) ||
+      !make_map_packed(&mv, V, total, H_kv, d))
+    return ATTN_ERR_LAUNCH;
+  attn::FwdParams prm = {};
+  prm.o = static_cast<__nv_bfloat16*>(O);
+  prm.lse = LSE;
+  prm.h = int(H);
+  prm.h_kv = int(H_kv);
+  prm.group = int(H / H_kv);
+  prm.scale_log2 = scale * 1.4426950408889634f;
+  prm.cu_seqlens = cu_seqlens;
+  prm.n_seqs = int(n_seqs);
+  prm.total = int(total);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the item count depends on the lengths (device data): a CTA per SM, plain dealing
+  const int grid = int(kNumSMs);
+  if (d == 128)
+    return causal ? launch_fwd<128, true, false, false, true>(mq, mk, mv, prm, grid, st)
+                  : launch_fwd<128, false, false, false, true>(mq, mk, mv, prm, grid, st);
+  return causal ? launch_fwd<64, true, false, false, true>(mq, mk, mv, prm, grid, st)
+                : launch_fwd<64, false, false, false, true>(mq, mk, mv, prm, grid, st);
 }
 
 ATTN_EXPORT int attn_fwd_f32out(const void* Q, const void* K, const void* V, void* O, float* O32, float* LSE,

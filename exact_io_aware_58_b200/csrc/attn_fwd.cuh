@@ -56,8 +56,11 @@ struct FwdParams {
   const uint8_t* mask; // block-sparse only: [B*H][nt][nt], 1 = query tile attends key tile
   int nt;              // ceil(N / 128)
   float* o32;          // O32 instances only: [B*H][N][D] fp32 copy of the normalised O
-  int n_items;         // B*H*n_mblk work items
+  int n_items;         // B*H*n_mblk work items (packed-sequence instances count their own)
   int snake;           // 1: odd rounds of grid-size items are dealt to the CTAs in reverse
+  const int* cu_seqlens;   // packed sequences only: [n_seqs + 1] token offsets (device)
+  int n_seqs;              // packed sequences only: number of sequences
+  int total;               // packed sequences only: total tokens (rows of Q, K, V, O)
 };
 
 // The items of round r (items [r*G, r*G + G), G = grid size) go one per CTA;
@@ -111,20 +114,71 @@ struct FwdCfg {
 };
 
 // Work item -> (query head, first query row, key tiles that may be visible,
-// selection, key tiles visited).  Every role evaluates the same function.
+// selection, key tiles visited, where its rows live).  Every role evaluates
+// the same function on the same increasing item sequence.
 struct FwdItem {
   int bh, bkv, m0, kv_hi, nkv;
+  int n;                // rows of this item's sequence (N, or the packed sequence's length)
+  int head, head_kv;    // query / key-value head (packed sequences)
+  int tok0;             // first token of the sequence in the packed tensors (0 otherwise)
   TileSelect sel;
 };
 
-template <bool CAUSAL, bool SPARSE>
-__device__ __forceinline__ FwdItem fwd_item(const FwdParams& prm, int item) {
+// Packed sequences: sequence s holds tokens [cu[s], cu[s+1]); its items are
+// its heads times its 256-row blocks, heaviest causal blocks first.  The
+// cursor only moves forward, because each role asks for increasing items.
+struct SeqCursor {
+  int s = 0;       // current sequence
+  int base = 0;    // items of the sequences before it
+};
+
+// First token and length of sequence s, clamped to [0, total] (offsets past
+// the tensors, or decreasing ones, give empty sequences: nothing is read or
+// written outside the tensors whatever cu_seqlens holds).
+__device__ __forceinline__ int seq_start(const FwdParams& prm, int s) {
+  return min(max(prm.cu_seqlens[s], 0), prm.total);
+}
+__device__ __forceinline__ int seq_len(const FwdParams& prm, int s) {
+  return max(min(max(prm.cu_seqlens[s + 1], 0), prm.total) - seq_start(prm, s), 0);
+}
+__device__ __forceinline__ int seq_blocks(const FwdParams& prm, int s) { return (seq_len(prm, s) + 255) >> 8; }
+
+__device__ __forceinline__ int packed_items(const FwdParams& prm) {
+  int total = 0;
+  for (int s = 0; s < prm.n_seqs; ++s) total += prm.h * seq_blocks(prm, s);
+  return total;
+}
+
+template <bool CAUSAL, bool SPARSE, bool VARLEN>
+__device__ __forceinline__ FwdItem fwd_item(const FwdParams& prm, int item, SeqCursor& cur) {
   FwdItem w;
-  w.bh = item / prm.n_mblk;
-  w.bkv = (w.bh / prm.h) * prm.h_kv + (w.bh % prm.h) / prm.group;
-  const int m_blk = prm.n_mblk - 1 - (item % prm.n_mblk);   // heaviest causal blocks of a head first
+  int m_blk, n_mblk;
+  if (VARLEN) {
+    while (cur.s + 1 < prm.n_seqs && item >= cur.base + prm.h * seq_blocks(prm, cur.s)) {
+      cur.base += prm.h * seq_blocks(prm, cur.s);
+      ++cur.s;
+    }
+    n_mblk = max(seq_blocks(prm, cur.s), 1);
+    const int local = item - cur.base;
+    w.head = local / n_mblk;
+    w.head_kv = w.head / prm.group;
+    w.tok0 = seq_start(prm, cur.s);
+    w.n = seq_len(prm, cur.s);
+    w.bh = w.head;
+    w.bkv = w.head_kv;
+    m_blk = n_mblk - 1 - local % n_mblk;
+  } else {
+    n_mblk = prm.n_mblk;
+    w.bh = item / n_mblk;
+    w.bkv = (w.bh / prm.h) * prm.h_kv + (w.bh % prm.h) / prm.group;
+    w.head = w.bh;
+    w.head_kv = w.bkv;
+    w.tok0 = 0;
+    w.n = prm.n;
+    m_blk = n_mblk - 1 - (item % n_mblk);   // heaviest causal blocks of a head first
+  }
   w.m0 = m_blk * 256;
-  const int n_kv_total = (prm.n + 127) >> 7;
+  const int n_kv_total = (w.n + 127) >> 7;
   w.kv_hi = CAUSAL ? min(n_kv_total, (w.m0 >> 7) + 2) : n_kv_total;
   w.sel = TileSelect{nullptr, nullptr};
   if (SPARSE) {
@@ -136,9 +190,23 @@ __device__ __forceinline__ FwdItem fwd_item(const FwdParams& prm, int item) {
   return w;
 }
 
+// TMA coordinates of rows [r0, r0 + 128) of a head: BHND tensors are mapped
+// as [B*H][N][d] (coordinates x, row, head); packed ones as [total][H][d]
+// (coordinates x, head, token).
+template <bool VARLEN>
+__device__ __forceinline__ void load_rows(const CUtensorMap* map, uint64_t* bar, void* dst, int x, int head,
+                                          int tok0, int r0) {
+  if (VARLEN)
+    tma_load_3d(map, bar, dst, x, head, tok0 + r0);
+  else
+    tma_load_3d(map, bar, dst, x, r0, head);
+}
+
 // O32: also write the normalised rows in fp32 to prm.o32 (a separate
 // instance, so the bf16-only instances are compiled without it).
-template <int D, bool CAUSAL, bool SPARSE, bool O32 = false>
+// VARLEN: packed sequences of different lengths ([total][H][d] tensors, one
+// causal/non-causal attention per sequence; dense, bf16 output only).
+template <int D, bool CAUSAL, bool SPARSE, bool O32 = false, bool VARLEN = false>
 __global__ void __launch_bounds__(320, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const FwdParams prm) {
@@ -160,7 +228,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int n = prm.n;
+  const int n_items = VARLEN ? packed_items(prm) : prm.n_items;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -199,18 +267,19 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       int issued = 0;    // K/V tiles loaded (ring position)
       int qn = 0;        // items whose Q was loaded
       bool ok = true;
-      for (int rr = 0, item = fwd_round_item(0, gridDim.x, prm.snake); rr * int(gridDim.x) < prm.n_items && ok;
+      SeqCursor cur;
+      for (int rr = 0, item = fwd_round_item(0, gridDim.x, prm.snake); rr * int(gridDim.x) < n_items && ok;
            item = fwd_round_item(++rr, gridDim.x, prm.snake)) {
-        if (item >= prm.n_items) continue;
-        const FwdItem w = fwd_item<CAUSAL, SPARSE>(prm, item);
+        if (item >= n_items) continue;
+        const FwdItem w = fwd_item<CAUSAL, SPARSE, VARLEN>(prm, item, cur);
         if (w.nkv == 0) continue;   // block-sparse: nothing selected, nothing loaded
         // the previous item's last QK^T products must be done with the Q slots
         if (qn > 0 && !(ok = mbar_wait(q_empty, (qn - 1) & 1, abort_flag))) break;
         mbar_arrive_expect_tx(q_full, 2 * C::kTileBytes);
         for (int t = 0; t < 2; ++t)
           for (int b = 0; b < C::kNumBlk; ++b)
-            tma_load_3d(&tm_q, q_full, smem + C::kOffQ + t * C::kTileBytes + b * C::kBlockBytes, b * 64,
-                        w.m0 + 128 * t, w.bh);
+            load_rows<VARLEN>(&tm_q, q_full, smem + C::kOffQ + t * C::kTileBytes + b * C::kBlockBytes, b * 64,
+                              w.bh, w.tok0, w.m0 + 128 * t);
         ++qn;
         int jsel = SPARSE ? w.sel.next(-1, w.kv_hi) : 0;
         for (int kk = 0; kk < 2 * w.nkv; ++kk) {
@@ -222,8 +291,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           if (SPARSE && (kk & 1)) jsel = w.sel.next(jsel, w.kv_hi);
           mbar_arrive_expect_tx(&kv_full[slot], C::kTileBytes);
           for (int b = 0; b < C::kNumBlk; ++b)
-            tma_load_3d(tm, &kv_full[slot], smem + C::kOffKV + slot * C::kTileBytes + b * C::kBlockBytes,
-                        b * 64, 128 * j, w.bkv);
+            load_rows<VARLEN>(tm, &kv_full[slot], smem + C::kOffKV + slot * C::kTileBytes + b * C::kBlockBytes,
+                              b * 64, w.bkv, w.tok0, 128 * j);
           ++issued;
         }
       }
@@ -271,10 +340,11 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       bool ok = true;
       int qn = 0;        // items processed
       int pc = 0;        // key tiles processed over all items (S/P barrier phases)
-      for (int rr = 0, item = fwd_round_item(0, gridDim.x, prm.snake); rr * int(gridDim.x) < prm.n_items && ok;
+      SeqCursor cur;
+      for (int rr = 0, item = fwd_round_item(0, gridDim.x, prm.snake); rr * int(gridDim.x) < n_items && ok;
            item = fwd_round_item(++rr, gridDim.x, prm.snake)) {
-        if (item >= prm.n_items) continue;
-        const int nkv = fwd_item<CAUSAL, SPARSE>(prm, item).nkv;
+        if (item >= n_items) continue;
+        const int nkv = fwd_item<CAUSAL, SPARSE, VARLEN>(prm, item, cur).nkv;
         if (nkv == 0) continue;
         // PV of key tile jl (of this item) for query tile t; the item's first
         // PV overwrites O_t, which the previous item's epilogue must have read.
@@ -338,25 +408,33 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const float c = prm.scale_log2;
     bool ok = true;
     int qn = 0, pc = 0;
-    for (int rr = 0, item = fwd_round_item(0, gridDim.x, prm.snake); rr * int(gridDim.x) < prm.n_items && ok;
+    SeqCursor cur;
+    for (int rr = 0, item = fwd_round_item(0, gridDim.x, prm.snake); rr * int(gridDim.x) < n_items && ok;
            item = fwd_round_item(++rr, gridDim.x, prm.snake)) {
-        if (item >= prm.n_items) continue;
-      const FwdItem w = fwd_item<CAUSAL, SPARSE>(prm, item);
+        if (item >= n_items) continue;
+      const FwdItem w = fwd_item<CAUSAL, SPARSE, VARLEN>(prm, item, cur);
       const int m0 = w.m0;
-      const int i = m0 + 128 * t + r;         // global query row
-      const size_t row = size_t(w.bh) * size_t(n) + size_t(i);
+      const int n = VARLEN ? w.n : prm.n;
+      const int i = m0 + 128 * t + r;         // query row within its sequence
+      // where row i lives: LSE index and (computed where it is used) O element offset
+      const size_t l_off = VARLEN ? size_t(w.head) * size_t(prm.total) + size_t(w.tok0 + i)
+                                  : size_t(w.bh) * size_t(n) + size_t(i);
+      auto o_offset = [&]() -> size_t {
+        return VARLEN ? (size_t(w.tok0 + i) * size_t(prm.h) + size_t(w.head)) * D : l_off * D;
+      };
       if (w.nkv == 0) {
         // block-sparse: a block that selected nothing: O = 0, LSE = -inf
         if (i < n) {
-          uint4* dst = reinterpret_cast<uint4*>(prm.o + row * D);
+          const size_t o_off = o_offset();
+          uint4* dst = reinterpret_cast<uint4*>(prm.o + o_off);
 #pragma unroll
           for (int k = 0; k < D / 8; ++k) dst[k] = make_uint4(0u, 0u, 0u, 0u);
           if (O32) {
-            float4* d32 = reinterpret_cast<float4*>(prm.o32 + row * D);
+            float4* d32 = reinterpret_cast<float4*>(prm.o32 + o_off);
 #pragma unroll
             for (int k = 0; k < D / 4; ++k) d32[k] = make_float4(0.f, 0.f, 0.f, 0.f);
           }
-          prm.lse[row] = -INFINITY;
+          prm.lse[l_off] = -INFINITY;
         }
         continue;
       }
@@ -458,6 +536,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       tc_fence_after();
       // l == 0 only for rows that see no key at all (block-sparse): O = 0, LSE = -inf.
       const float inv_l = (SPARSE && !(l > 0.f)) ? 0.f : 1.f / l;
+      const size_t o_off = o_offset();
 #pragma unroll 1
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t o[32];
@@ -468,7 +547,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           mbar_arrive(&o_free[t]);            // O_t has been read: the next item may overwrite it
         }
         if (i < n) {
-          uint4* dst = reinterpret_cast<uint4*>(prm.o + row * D + cc * 32);
+          uint4* dst = reinterpret_cast<uint4*>(prm.o + o_off + cc * 32);
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch)
             dst[ch] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * ch + 0]) * inv_l, __uint_as_float(o[8 * ch + 1]) * inv_l),
@@ -477,7 +556,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                                  pack_bf16x2(__uint_as_float(o[8 * ch + 6]) * inv_l, __uint_as_float(o[8 * ch + 7]) * inv_l));
           if (O32) {
             // the same normalised row in fp32, before the bf16 rounding
-            float4* d32 = reinterpret_cast<float4*>(prm.o32 + row * D + cc * 32);
+            float4* d32 = reinterpret_cast<float4*>(prm.o32 + o_off + cc * 32);
 #pragma unroll
             for (int k = 0; k < 8; ++k)
               d32[k] = make_float4(__uint_as_float(o[4 * k]) * inv_l, __uint_as_float(o[4 * k + 1]) * inv_l,
@@ -485,7 +564,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           }
         }
       }
-      if (i < n) prm.lse[row] = (SPARSE && !(l > 0.f)) ? -INFINITY : (m_ref + __log2f(l)) * kLn2;
+      if (i < n) prm.lse[l_off] = (SPARSE && !(l > 0.f)) ? -INFINITY : (m_ref + __log2f(l)) * kLn2;
       pc += w.nkv;
       ++qn;
     }

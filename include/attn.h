@@ -94,6 +94,29 @@ int attn_fwd_gqa(const void* Q, const void* K, const void* V, void* O, float* LS
                  void* stream);
 
 /*
+ * Forward over packed sequences of different lengths (prefill of many
+ * sequences in one call: "FlashAttention -- how 100K-token attention fits in
+ * memory", section "Arithmetic intensity"; the tiling and online softmax are
+ * those of attn_fwd).  Sequence s holds tokens [cu_seqlens[s], cu_seqlens[s+1])
+ * of the packed tensors and attends only to its own tokens (causal: token i of
+ * a sequence sees its tokens 0..i).
+ *   Q, O        bf16 [total][H][d]      (token-major, row stride H*d)
+ *   K, V        bf16 [total][H_kv][d]   query head h reads key/value head h / (H / H_kv)
+ *   LSE         fp32 [H][total]         natural-log row log-sum-exp
+ *   cu_seqlens  int32 [n_seqs + 1] DEVICE array, non-decreasing, cu_seqlens[0] = 0,
+ *               cu_seqlens[n_seqs] = total (4-byte aligned).  Offsets are clamped
+ *               to [0, total] on the device, so nothing outside the tensors is read
+ *               or written whatever the array holds; tokens outside every sequence
+ *               get no output.  Empty sequences are allowed.
+ * d must be 64 or 128 (else ATTN_ERR_UNSUPPORTED); n_seqs, total >= 1.  The
+ * result for each sequence equals attn_fwd_gqa on that sequence alone, bit for
+ * bit.  Other rules as attn_fwd.
+ */
+int attn_fwd_varlen(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                    const int32_t* cu_seqlens, int64_t n_seqs, int64_t total, int64_t H, int64_t H_kv,
+                    int64_t d, int causal, float scale, void* stream);
+
+/*
  * Forward restricted to selected blocks ("Attention and KV Compression",
  * section "The composability point": sparse selection changes which blocks
  * are attended, and the kernel runs on the selected blocks).

@@ -59,6 +59,7 @@ __all__ = [
     "e4m3_decode",
     "attn_fwd_fp8",
     "attn_fwd_kvcache_fp8",
+    "attn_fwd_varlen",
 ]
 
 
@@ -351,3 +352,32 @@ def attn_fwd_kvcache_fp8(Q, K8, V8, k_descale: float, v_descale: float, scale: f
     K = float(k_descale) * e4m3_decode(K8)
     V = float(v_descale) * e4m3_decode(V8)
     return attn_fwd_kvcache(Q, K, V, scale, causal, B, H, H_kv, kv_lens=kv_lens)
+
+
+# ---------------------------------------------------------------------------
+# Packed variable-length sequences ("FlashAttention -- how 100K-token
+# attention fits in memory", section "Arithmetic intensity": prefill of many
+# sequences at once).  Sequence s holds tokens [cu[s], cu[s+1]) of the packed
+# (total, H, d) tensors and attends only to its own tokens; each sequence is
+# the plain attention above.
+# ---------------------------------------------------------------------------
+
+def attn_fwd_varlen(Q, K, V, cu_seqlens, scale: float, causal: bool, H: int, H_kv: int):
+    """Q (total, H, d), K, V (total, H_kv, d), cu_seqlens (n_seqs + 1,) ->
+    O (total, H, d), LSE (H, total).  Query head h reads key/value head
+    h // (H // H_kv)."""
+    Q, K, V = (np.asarray(x, dtype=np.float64) for x in (Q, K, V))
+    total, _, d = Q.shape
+    O = np.zeros((total, H, d))
+    LSE = np.zeros((H, total))
+    cu = [int(c) for c in cu_seqlens]
+    for a, b in zip(cu[:-1], cu[1:]):
+        if b <= a:
+            continue
+        q = Q[a:b].transpose(1, 0, 2)                      # (H, len, d)
+        k = K[a:b].transpose(1, 0, 2)
+        v = V[a:b].transpose(1, 0, 2)
+        o, lse = attn_fwd_gqa(q, k, v, scale, causal, 1, H, H_kv)
+        O[a:b] = o.transpose(1, 0, 2)
+        LSE[:, a:b] = lse
+    return O, LSE

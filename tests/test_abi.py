@@ -247,3 +247,22 @@ def test_kvcache_fp8_argument_errors(lib):
         q = [A] * 5
         q[k] = MIS
         assert call(ptrs=q) == attn.ATTN_ERR_MISALIGNED
+
+
+def test_varlen_argument_errors(lib):
+    p = [A] * 5
+
+    def call(ptrs=None, cu=A, n_seqs=2, total=300, H=4, Hk=2, d=128, scale=0.1):
+        return lib.attn_fwd_varlen(*(ptrs or p), cu, n_seqs, total, H, Hk, d, 1, scale, None)
+
+    assert call(n_seqs=0) == attn.ATTN_ERR_INVALID_ARG
+    assert call(total=0) == attn.ATTN_ERR_INVALID_ARG
+    assert call(d=96) == attn.ATTN_ERR_UNSUPPORTED
+    assert call(Hk=3) == attn.ATTN_ERR_INVALID_ARG
+    assert call(scale=0.0) == attn.ATTN_ERR_INVALID_ARG
+    assert call(cu=None) == attn.ATTN_ERR_INVALID_ARG
+    assert call(cu=ctypes.c_void_p(0x100002)) == attn.ATTN_ERR_MISALIGNED
+    for k in range(5):
+        q = [A] * 5
+        q[k] = MIS
+        assert call(ptrs=q) == attn.ATTN_ERR_MISALIGNED

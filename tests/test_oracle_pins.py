@@ -717,3 +717,72 @@ def test_kvcache_fp8_is_kvcache_on_the_dequantised_cache():
     O2, L2 = orc.attn_fwd_kvcache(q, Kd, Vd, 0.7, True, B, H, Hk, kv_lens=[9, 4])
     np.testing.assert_allclose(O, O2, rtol=1e-14)
     np.testing.assert_allclose(L, L2, rtol=1e-14)
+
+
+# ---------------------------------------------------------------------------
+# Packed variable-length sequences
+# ---------------------------------------------------------------------------
+
+def _block_diagonal_reference(Q, K, V, cu, scale, causal, H, H_kv):
+    """Brute force over all packed tokens at once: one (total x total) score
+    matrix per head, every pair of tokens from different sequences masked
+    (and later tokens of the same sequence too, if causal), then a plain
+    softmax -- a formulation independent of the per-sequence split."""
+    total = Q.shape[0]
+    seq = np.zeros(total, dtype=np.int64)
+    pos = np.zeros(total, dtype=np.int64)
+    for s, (a, b) in enumerate(zip(cu[:-1], cu[1:])):
+        seq[a:b] = s
+        pos[a:b] = np.arange(b - a)
+    O = np.zeros_like(Q, dtype=np.float64)
+    LSE = np.zeros((H, total))
+    for h in range(H):
+        kh = h // (H // H_kv)
+        S = scale * Q[:, h, :] @ K[:, kh, :].T
+        allowed = seq[:, None] == seq[None, :]
+        if causal:
+            allowed &= pos[None, :] <= pos[:, None]
+        S = np.where(allowed, S, -np.inf)
+        m = S.max(axis=1, keepdims=True)
+        e = np.exp(S - m)
+        z = e.sum(axis=1, keepdims=True)
+        O[:, h, :] = (e / z) @ V[:, kh, :]
+        LSE[h] = (m + np.log(z))[:, 0]
+    return O, LSE
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_matches_block_diagonal_brute_force(causal):
+    rng = np.random.default_rng(31)
+    lens = [3, 1, 0, 7, 5]
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    total, H, Hk, d = int(cu[-1]), 4, 2, 6
+    Q, K, V = (rng.standard_normal((total, h, d)) for h in (H, Hk, Hk))
+    O, L = orc.attn_fwd_varlen(Q, K, V, cu, 0.4, causal, H, Hk)
+    O_ref, L_ref = _block_diagonal_reference(Q, K, V, cu, 0.4, causal, H, Hk)
+    np.testing.assert_allclose(O, O_ref, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(L, L_ref, rtol=1e-12, atol=1e-12)
+
+
+def test_varlen_sequences_are_independent():
+    rng = np.random.default_rng(32)
+    cu = np.array([0, 4, 9, 12])
+    Q, K, V = (rng.standard_normal((12, 2, 5)) for _ in range(3))
+    O, L = orc.attn_fwd_varlen(Q, K, V, cu, 0.3, True, 2, 2)
+    K2, V2 = K.copy(), V.copy()
+    K2[4:9] += 10.0                      # change only the middle sequence's keys and values
+    V2[4:9] *= -3.0
+    O2, L2 = orc.attn_fwd_varlen(Q, K2, V2, cu, 0.3, True, 2, 2)
+    same = np.r_[0:4, 9:12]
+    np.testing.assert_array_equal(O[same], O2[same])
+    np.testing.assert_array_equal(L[:, same], L2[:, same])
+    assert not np.allclose(O[4:9], O2[4:9])
+
+
+def test_varlen_single_sequence_is_plain_attention():
+    rng = np.random.default_rng(33)
+    Q, K, V = (rng.standard_normal((11, 3, 4)) for _ in range(3))
+    O, L = orc.attn_fwd_varlen(Q, K, V, [0, 11], 0.5, True, 3, 3)
+    O_ref, L_ref = orc.attn_fwd(Q.transpose(1, 0, 2), K.transpose(1, 0, 2), V.transpose(1, 0, 2), 0.5, True)
+    np.testing.assert_allclose(O, O_ref.transpose(1, 0, 2), rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(L, L_ref, rtol=1e-13, atol=1e-13)

@@ -84,6 +84,13 @@ def test_fp8_forward_shared_heads_statistics(causal):
     _case(2, 4, 2, 1024, causal, seed=950 + causal, stats=True)
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_fp8_forward_many_items_per_cta(causal):
+    # 2 x 40 query heads on 8 key/value heads, 3 row blocks each: 240 CTAs,
+    # more than one wave on the SMs, with a ragged last block (513 rows)
+    _case(2, 40, 8, 513, causal, seed=960 + causal, stats=True)
+
+
 def test_fp8_forward_peaked_rows():
     # queries scaled up so rows put most of their weight on a few keys (the
     # lazy rescale fires and P spans the whole E4M3 range)

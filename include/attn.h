@@ -384,8 +384,9 @@ int attn_bwd_dq(const void* Q, const void* K, const void* V, const void* dO, voi
  *  - The array belongs to the library's module in the calling thread's
  *    current CUDA context (on its current device); every call looks its
  *    device address up there (cudaGetSymbolAddress, which allocates
- *    nothing).  The first call in a context loads the module if it is not
- *    loaded yet; make that first call before any stream capture.
+ *    nothing).  The first call in a context loads the module there if it
+ *    is not loaded yet (work the CUDA runtime does, as for any first kernel
+ *    launch from a module).
  *  - It calls no cudaMalloc, cudaFree or other allocating routine.
  *  - Every call in a context shares the one array, and the array keeps the
  *    last call's contents.  Nothing in it needs to start at zero: the

@@ -186,8 +186,18 @@ int set_smem(const void* kern, int bytes) {
 template <int D, bool CAUSAL, bool SPARSE, bool O32 = false, bool VARLEN = false>
 int launch_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const attn::FwdParams& prm,
                int grid, cudaStream_t st) {
+  using C = attn::FwdCfg<D>;
   auto kern = attn::attn_fwd_kernel<D, CAUSAL, SPARSE, O32, VARLEN>;
-  constexpr int smem = attn::FwdCfg<D>::kSmemBytes;
+  constexpr int smem = C::kSmemBytes;
+  // The kernel moves registers between its warpgroups (setmaxnreg), which
+  // only adds up if every thread was launched with exactly kRegsLaunch.
+  cudaFuncAttributes fa;
+  const cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess)
+    return fail(ATTN_ERR_LAUNCH, "cudaFuncGetAttributes(forward): %s (%lld)", cudaGetErrorString(e), (long long)e);
+  if (fa.numRegs != int(C::kRegsLaunch))
+    return fail(ATTN_ERR_LAUNCH, "forward compiled to %d registers per thread, its warpgroup split needs %d",
+                fa.numRegs, int(C::kRegsLaunch));
   if (set_smem(reinterpret_cast<const void*>(kern), smem) != ATTN_OK) return ATTN_ERR_LAUNCH;
   kern<<<grid, attn::FwdCfg<D>::kThreads, smem, st>>>(q, k, v, prm);
   return launch_status();

@@ -8,7 +8,7 @@
 // kept, the partial output is rescaled by exp(m_old - m_new) when the max
 // grows, and only O and one statistic per row (LSE) are written out.
 //
-// B200 mapping: a persistent grid of at most one CTA per SM (320 threads).  A
+// B200 mapping: a persistent grid of at most one CTA per SM (384 threads).  A
 // work item is two 128-row query tiles of one head; items are ordered
 // heads-major, heaviest causal blocks first within a head (so that a head's
 // K/V stays in L2 while its items run), and dealt out in rounds of one item
@@ -21,13 +21,17 @@
 //               runs on across items.
 //   warp 8      MMA issuer (one thread): S_t = Q_t K_j^T and O_t += P_t V_j as
 //               tcgen05.mma with fp32 accumulators in tensor memory (TMEM).
+//   warps 10-11 idle: they complete warpgroup 2, whose registers go to the
+//               softmax warpgroups (setmaxnreg, see FwdCfg).
 //   warps 0-3   softmax for query tile 0, warps 4-7 for tile 1: each thread owns
 //               one query row (= one TMEM lane), so the row max and sum need no
 //               shuffles.  P is rounded to bf16 and written back into TMEM over
 //               the upper half of S, where the PV MMA reads it as its A operand.
-//               At the end of an item each thread writes its normalised O row
-//               (and LSE) straight to global memory, so that the Q slots are
-//               free for the next item as soon as its last QK^T is done.
+//               At the end of an item each thread reads its whole O row out of
+//               TMEM in one round trip, releases O_t to the next item's first
+//               PV, and writes the normalised row (and LSE) straight to global
+//               memory, so that the Q slots are free for the next item as soon
+//               as its last QK^T is done.
 // The issue order PV_t(j-1), S_t(j) lets the tensor core run one tile's GEMMs
 // while the other tile's softmax runs (ping-pong between the two tiles).
 //
@@ -98,9 +102,22 @@ struct FwdCfg {
   static constexpr int kBlockBytes = 128 * 128;          // one [128][64] bf16 column block
   static constexpr int kNumBlk = D / 64;
   static constexpr int kSlots = (D == 128) ? 4 : 8;      // K/V ring depth
-  static constexpr int kThreads = 320;
+  // Warps 0-7 softmax (two warpgroups), warpgroup 2 = MMA warp, TMA warp and
+  // two idle warps.  Registers are allocated per warpgroup slot, so a block
+  // of three warpgroups is launched with 168 per thread (3 * 168 <= 512 per
+  // SM sub-partition, which holds one warp of each warpgroup); warpgroup 2
+  // then gives registers back (setmaxnreg) and the softmax warpgroups take
+  // them: 2 * 176 + 152 = 3 * 168.  The issue warpgroup keeps 152 because its
+  // unrolled descriptor code spills below that in the packed-sequence
+  // instances; 176 lets the epilogue hold a whole O row without spilling.
+  // The host refuses to launch unless the kernel compiled to exactly
+  // kRegsLaunch, which the split assumes.
+  static constexpr int kThreads = 384;
   static constexpr int kWarpMma = 8;
   static constexpr int kWarpLoad = 9;
+  static constexpr uint32_t kRegsLaunch = 168;
+  static constexpr uint32_t kRegsIssue = 152;
+  static constexpr uint32_t kRegsSoftmax = 176;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColS0 = 0, kColS1 = 128;
   static constexpr uint32_t kColO0 = 256, kColO1 = 256 + D;
@@ -111,6 +128,7 @@ struct FwdCfg {
   static constexpr int kNumBars = 2 + 2 * kSlots + 2 + 2 + 2 + 2 + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;   // + slack for 1024-byte alignment
+  static_assert(2 * kRegsSoftmax + kRegsIssue <= 3 * kRegsLaunch, "register split");
 };
 
 // Work item -> (query head, first query row, key tiles that may be visible,
@@ -207,7 +225,7 @@ __device__ __forceinline__ void load_rows(const CUtensorMap* map, uint64_t* bar,
 // VARLEN: packed sequences of different lengths ([total][H][d] tensors, one
 // causal/non-causal attention per sequence; dense, bf16 output only).
 template <int D, bool CAUSAL, bool SPARSE, bool O32 = false, bool VARLEN = false>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
 attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, const FwdParams prm) {
   using C = FwdCfg<D>;
@@ -261,7 +279,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == C::kWarpLoad) {
+  if (warp >= C::kWarpMma) {
+   // warpgroup 2: one TMA thread, one MMA thread, two idle warps
+   regs_dec<C::kRegsIssue>();
+   if (warp == C::kWarpLoad) {
     // ------------------------------------------------------------------ TMA
     if (lane == 0) {
       int issued = 0;    // K/V tiles loaded (ring position)
@@ -302,7 +323,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mbar_wait(&kv_full[it % C::kSlots], (it / C::kSlots) & 1, abort_flag, false);
     }
     __syncwarp();
-  } else if (warp == C::kWarpMma) {
+   } else if (warp == C::kWarpMma) {
     // ------------------------------------------------------------------ MMA
     if (lane == 0) {
       constexpr uint32_t kIdescS = idesc_bf16(128, 128, false, false);
@@ -396,8 +417,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       mbar_wait(drain, 0, abort_flag, false);
     }
     __syncwarp();
+   }
   } else {
     // -------------------------------------------------------------- softmax
+    regs_inc<C::kRegsSoftmax>();
     const int t = warp >> 2;
     const int qw = warp & 3;
     const int r = qw * 32 + lane;           // row inside the tile = TMEM lane
@@ -537,15 +560,19 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       // l == 0 only for rows that see no key at all (block-sparse): O = 0, LSE = -inf.
       const float inv_l = (SPARSE && !(l > 0.f)) ? 0.f : 1.f / l;
       const size_t o_off = o_offset();
-#pragma unroll 1
+      // The whole row in one TMEM round trip (D/32 loads, one wait), so O_t is
+      // released to the next item's first PV before any of it is stored.
+      uint32_t orow[D / 32][32];
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) tmem_ld32(tO + cc * 32, orow[cc]);
+      tmem_ld_wait(orow[0]);
+#pragma unroll
+      for (int cc = 1; cc < D / 32; ++cc) reg_fence32(orow[cc]);
+      tc_fence_before();
+      mbar_arrive(&o_free[t]);                // O_t has been read: the next item may overwrite it
+#pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t o[32];
-        tmem_ld32(tO + cc * 32, o);
-        tmem_ld_wait(o);
-        if (cc == D / 32 - 1) {
-          tc_fence_before();
-          mbar_arrive(&o_free[t]);            // O_t has been read: the next item may overwrite it
-        }
+        const uint32_t (&o)[32] = orow[cc];
         if (i < n) {
           uint4* dst = reinterpret_cast<uint4*>(prm.o + o_off + cc * 32);
 #pragma unroll

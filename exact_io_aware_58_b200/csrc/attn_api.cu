@@ -773,8 +773,16 @@ namespace {
 template <bool CAUSAL>
 int launch_fp8(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const attn::Fp8Params& prm,
                int grid, cudaStream_t st) {
+  using C = attn::Fp8Cfg;
   auto kern = attn::attn_fwd_fp8_kernel<CAUSAL>;
-  constexpr int smem = attn::Fp8Cfg::kSmemBytes;
+  constexpr int smem = C::kSmemBytes;
+  cudaFuncAttributes fa;   // the setmaxnreg split needs exactly kRegsLaunch per thread at launch
+  const cudaError_t e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess)
+    return fail(ATTN_ERR_LAUNCH, "cudaFuncGetAttributes(FP8 forward): %s (%lld)", cudaGetErrorString(e), (long long)e);
+  if (fa.numRegs != int(C::kRegsLaunch))
+    return fail(ATTN_ERR_LAUNCH, "FP8 forward compiled to %d registers per thread, its warpgroup split needs %d",
+                fa.numRegs, int(C::kRegsLaunch));
   if (set_smem(reinterpret_cast<const void*>(kern), smem) != ATTN_OK) return ATTN_ERR_LAUNCH;
   kern<<<grid, attn::Fp8Cfg::kThreads, smem, st>>>(q, k, v, prm);
   return launch_status();

@@ -15,8 +15,8 @@
 //     not exact: each p changes by at most 2^-4 of itself or 2^-10 absolute.
 //
 // Layout and roles follow the bf16 forward (two 128-row query tiles per CTA,
-// warp 9 TMA, warp 8 MMA, warps 0-3 / 4-7 softmax of tile 0 / 1, S and O in
-// TMEM), with d = 128 only: one 128-byte swizzled row holds a full 128-wide
+// warp 9 TMA, warp 8 MMA, warps 0-3 / 4-7 softmax of tile 0 / 1, warps 10-11
+// idle, the same register split, S and O in TMEM), with d = 128 only: one 128-byte swizzled row holds a full 128-wide
 // E4M3 row, tiles are 16 KB, and the K/V ring has 8 slots.  The epilogue
 // stores each thread's O row straight to global memory.
 #pragma once
@@ -44,9 +44,17 @@ struct Fp8Params {
 struct Fp8Cfg {
   static constexpr int kTileBytes = 128 * 128;          // 128 rows x 128 E4M3
   static constexpr int kSlots = 8;
-  static constexpr int kThreads = 320;
+  // Warps 0-7 softmax, warpgroup 2 = MMA, TMA and two idle warps; launched
+  // with 168 registers per thread (three warpgroup slots), warpgroup 2 gives
+  // registers back and the softmax warpgroups take them (setmaxnreg):
+  // 2 * kRegsSoftmax + kRegsIssue = 3 * 168.  The host refuses to launch
+  // unless the kernel compiled to exactly kRegsLaunch.
+  static constexpr int kThreads = 384;
   static constexpr int kWarpMma = 8;
   static constexpr int kWarpLoad = 9;
+  static constexpr uint32_t kRegsLaunch = 168;
+  static constexpr uint32_t kRegsIssue = 152;
+  static constexpr uint32_t kRegsSoftmax = 176;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kColS0 = 0, kColS1 = 128;
   static constexpr uint32_t kColO0 = 256, kColO1 = 384;
@@ -57,6 +65,7 @@ struct Fp8Cfg {
   static constexpr int kNumBars = 2 + 2 * kSlots + 2 + 2 + 2 + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
+  static_assert(2 * kRegsSoftmax + kRegsIssue <= 3 * kRegsLaunch, "register split");
 };
 
 // Instruction descriptor, kind::f8f6f4 with E4M3 A and B (format code 0) and
@@ -103,7 +112,7 @@ __device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float
 }
 
 template <bool CAUSAL>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
 attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const Fp8Params prm) {
   using C = Fp8Cfg;
@@ -160,7 +169,10 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == C::kWarpLoad) {
+  if (warp >= C::kWarpMma) {
+   // warpgroup 2: one TMA thread, one MMA thread, two idle warps
+   regs_dec<C::kRegsIssue>();
+   if (warp == C::kWarpLoad) {
     // ------------------------------------------------------------------ TMA
     if (lane == 0) {
       for (int t = 0; t < 2; ++t) {
@@ -184,7 +196,7 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         mbar_wait(&kv_full[it % C::kSlots], (it / C::kSlots) & 1, abort_flag, false);
     }
     __syncwarp();
-  } else if (warp == C::kWarpMma) {
+   } else if (warp == C::kWarpMma) {
     // ------------------------------------------------------------------ MMA
     if (lane == 0) {
       constexpr uint32_t kIdescS = idesc_e4m3(128, 128, false, false);
@@ -263,8 +275,10 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
       mbar_wait(drain, 0, abort_flag, false);
     }
     __syncwarp();
+   }
   } else {
     // -------------------------------------------------------------- softmax
+    regs_inc<C::kRegsSoftmax>();
     const int t = warp >> 2;
     const int qw = warp & 3;
     const int r = qw * 32 + lane;
@@ -365,11 +379,15 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     if (ok) {
       tc_fence_after();
       const float f = prm.v_descale / l;
-#pragma unroll 1
+      uint32_t orow[D / 32][32];              // the whole row: one TMEM round trip
+#pragma unroll
+      for (int cc = 0; cc < D / 32; ++cc) tmem_ld32(tO + cc * 32, orow[cc]);
+      tmem_ld_wait(orow[0]);
+#pragma unroll
+      for (int cc = 1; cc < D / 32; ++cc) reg_fence32(orow[cc]);
+#pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t o[32];
-        tmem_ld32(tO + cc * 32, o);
-        tmem_ld_wait(o);
+        const uint32_t (&o)[32] = orow[cc];
         if (i < n) {
           uint4* dst = reinterpret_cast<uint4*>(prm.o + (size_t(bh) * size_t(n) + size_t(i)) * D + cc * 32);
 #pragma unroll

@@ -58,11 +58,14 @@ struct FusedCfg {
   // Registers per thread: launched with kRegsLaunch for every warp; warpgroup
   // 2 (MMA, TMA, two idle warps) gives back down to kRegsIssue and warpgroup 3
   // (the drain) takes up to kRegsDrain, enough to hold a whole 128-column
-  // partial.  2 * 128 + 80 + 176 = 4 * 128: the per-SM-subpartition register
-  // file is used exactly (each holds one warp of every warpgroup).
+  // partial.  2 * 128 + 72 + 184 = 2 * 128 + 80 + 176 = 4 * 128: the
+  // per-SM-subpartition register file is used exactly (each holds one warp of
+  // every warpgroup).  The split is the smallest drain share without spills
+  // at each D (at D = 128 the drain spills with 176, at D = 64 the issue
+  // warpgroup spills with 72).
   static constexpr uint32_t kRegsLaunch = 128;
-  static constexpr uint32_t kRegsIssue = 80;
-  static constexpr uint32_t kRegsDrain = 176;
+  static constexpr uint32_t kRegsIssue = (D == 128) ? 72 : 80;
+  static constexpr uint32_t kRegsDrain = (D == 128) ? 184 : 176;
   static_assert(2 * kRegsLaunch + kRegsIssue + kRegsDrain == 4 * kRegsLaunch, "register split");
   static constexpr uint32_t kTmemCols = 512;
   // Ring depths.  Q_i is read by S^T(i) (issued right after dV(i-1)) and,

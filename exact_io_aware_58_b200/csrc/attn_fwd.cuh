@@ -136,6 +136,8 @@ struct FwdCfg {
 // the same function on the same increasing item sequence.
 struct FwdItem {
   int bh, bkv, m0, kv_hi, nkv;
+  int nkv0;             // key tiles query tile 0 visits (causal: one fewer than nkv when the
+                        // item's last key tile lies wholly above tile 0's rows)
   int n;                // rows of this item's sequence (N, or the packed sequence's length)
   int head, head_kv;    // query / key-value head (packed sequences)
   int tok0;             // first token of the sequence in the packed tensors (0 otherwise)
@@ -205,6 +207,10 @@ __device__ __forceinline__ FwdItem fwd_item(const FwdParams& prm, int item, SeqC
     w.sel.r1 = (qt0 + 1 < prm.nt) ? w.sel.r0 + prm.nt : nullptr;
   }
   w.nkv = SPARSE ? w.sel.count(w.kv_hi) : w.kv_hi;
+  // Causal: key tile 2m+1 (the last one, when N does not cut it off) starts
+  // after the last row of query tile 0, so only tile 1 needs it.  (Not in the
+  // packed-sequence instances, whose issue warp would spill.)
+  w.nkv0 = (CAUSAL && !SPARSE && !VARLEN && w.kv_hi == (w.m0 >> 7) + 2) ? w.nkv - 1 : w.nkv;
   return w;
 }
 
@@ -360,17 +366,18 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
       bool ok = true;
       int qn = 0;        // items processed
-      int pc = 0;        // key tiles processed over all items (S/P barrier phases)
+      int pc[2] = {0, 0};   // key tiles query tile t processed over all items (S_t/P_t barrier phases)
       SeqCursor cur;
       for (int rr = 0, item = fwd_round_item(0, gridDim.x, prm.snake); rr * int(gridDim.x) < n_items && ok;
            item = fwd_round_item(++rr, gridDim.x, prm.snake)) {
         if (item >= n_items) continue;
-        const int nkv = fwd_item<CAUSAL, SPARSE, VARLEN>(prm, item, cur).nkv;
+        const FwdItem w = fwd_item<CAUSAL, SPARSE, VARLEN>(prm, item, cur);
+        const int nkv = w.nkv, nkv0 = w.nkv0;
         if (nkv == 0) continue;
         // PV of key tile jl (of this item) for query tile t; the item's first
         // PV overwrites O_t, which the previous item's epilogue must have read.
         auto pv = [&](int t, int jl, int vslot) -> bool {
-          if (!mbar_wait(&p_full[t], (pc + jl) & 1, abort_flag)) return false;
+          if (!mbar_wait(&p_full[t], (pc[t] + jl) & 1, abort_flag)) return false;
           if (jl == 0 && qn > 0 && !mbar_wait(&o_free[t], (qn - 1) & 1, abort_flag)) return false;
           tc_fence_after();
           issue_pv(t, vslot, jl > 0);
@@ -393,6 +400,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
           for (int t = 0; t < 2; ++t) {
             if (!(ok = pv(t, j - 1, vs))) break;
             if (t == 1) mma_commit(&kv_empty[vs]);
+            if (t == 0 && j >= nkv0) continue;       // key tile j is wholly masked for tile 0
             issue_s(t, ks);
             mma_commit(&s_full[t]);
           }
@@ -404,12 +412,14 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         int vs;
         if (!(ok = wait_kv(vs))) break;
         for (int t = 0; t < 2 && ok; ++t) {
-          if (!(ok = pv(t, nkv - 1, vs))) break;
-          mma_commit(&o_full[t]);
+          if (t == 1 || nkv - 1 < nkv0)
+            if (!(ok = pv(t, nkv - 1, vs))) break;
+          mma_commit(&o_full[t]);               // after the tile's last PV
         }
         if (!ok) break;
         mma_commit(&kv_empty[vs]);
-        pc += nkv;
+        pc[0] += nkv0;
+        pc[1] += nkv;
         ++qn;
       }
       // Every MMA issued so far must finish before tensor memory is released.
@@ -464,7 +474,8 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
       float m_ref = -INFINITY;
       float l = 0.f;
       int jsel = SPARSE ? w.sel.next(-1, w.kv_hi) : 0;
-      for (int jj = 0; jj < w.nkv; ++jj) {
+      const int nkv_t = (t == 0) ? w.nkv0 : w.nkv;   // key tiles this query tile visits
+      for (int jj = 0; jj < nkv_t; ++jj) {
         // jj counts visited tiles (barrier phases); j is the key tile itself
         const int j = SPARSE ? jsel : jj;
         const bool tile_on = SPARSE ? ((w.sel.flags(j) >> t) & 1u) != 0 : true;
@@ -592,7 +603,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
       }
       if (i < n) prm.lse[l_off] = (SPARSE && !(l > 0.f)) ? -INFINITY : (m_ref + __log2f(l)) * kLn2;
-      pc += w.nkv;
+      pc += nkv_t;
       ++qn;
     }
   }

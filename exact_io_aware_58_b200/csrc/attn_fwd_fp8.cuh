@@ -139,6 +139,9 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
   const int m0 = m_blk * 256;
   const int n_kv_total = (n + 127) >> 7;
   const int nkv = CAUSAL ? min(n_kv_total, (m0 >> 7) + 2) : n_kv_total;
+  // Causal: key tile 2m+1 (the last one, when N does not cut it off) starts
+  // after the last row of query tile 0, so only tile 1 visits it.
+  const int nkv0 = (CAUSAL && nkv == (m0 >> 7) + 2) ? nkv - 1 : nkv;
 
   if (threadIdx.x == 0) {
     for (int t = 0; t < 2; ++t) {
@@ -255,6 +258,7 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
           tc_fence_after();
           issue_pv(t, vs, j - 1 > 0);
           if (t == 1) mma_commit(&kv_empty[vs]);
+          if (t == 0 && j >= nkv0) continue;     // key tile j is wholly masked for tile 0
           issue_s(t, ks);
           mma_commit(&s_full[t]);
         }
@@ -264,10 +268,12 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         int vs;
         ok = wait_kv(vs);
         for (int t = 0; t < 2 && ok; ++t) {
-          if (!(ok = mbar_wait(&p_full[t], (nkv - 1) & 1, abort_flag))) break;
-          tc_fence_after();
-          issue_pv(t, vs, nkv - 1 > 0);
-          mma_commit(&o_full[t]);
+          if (t == 1 || nkv - 1 < nkv0) {
+            if (!(ok = mbar_wait(&p_full[t], (nkv - 1) & 1, abort_flag))) break;
+            tc_fence_after();
+            issue_pv(t, vs, nkv - 1 > 0);
+          }
+          mma_commit(&o_full[t]);                 // after the tile's last PV
         }
         if (ok) mma_commit(&kv_empty[vs]);
       }
@@ -292,7 +298,8 @@ attn_fwd_fp8_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     float l = 0.f;
     bool ok = true;
 
-    for (int j = 0; j < nkv; ++j) {
+    const int nkv_t = (t == 0) ? nkv0 : nkv;   // key tiles this query tile visits
+    for (int j = 0; j < nkv_t; ++j) {
       if (!(ok = mbar_wait_warp(&s_full[t], j & 1, abort_flag))) break;
       tc_fence_after();
       float s[128];

@@ -7,6 +7,7 @@
 // g_attn_status (a static __device__ variable).
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstdarg>
@@ -183,21 +184,38 @@ int set_smem(const void* kern, int bytes) {
               (long long)bytes);
 }
 
+// Kernels that move registers between their warpgroups (setmaxnreg) are only
+// correct when every thread was launched with exactly the count the split
+// assumes (otherwise a growing warpgroup would wait for registers that never
+// come), so each launch checks the compiled count.  It is a property of the
+// compiled kernel, queried once per kernel (a failed query is not cached).
+template <auto KERN>
+int check_launch_regs(int want, const char* what) {
+  static std::atomic<int> cached{0};
+  int regs = cached.load(std::memory_order_relaxed);
+  if (regs == 0) {
+    cudaFuncAttributes fa;
+    const cudaError_t e = cudaFuncGetAttributes(&fa, KERN);
+    if (e != cudaSuccess)
+      return fail(ATTN_ERR_LAUNCH, "cudaFuncGetAttributes(%s): %s (%lld)", what, cudaGetErrorString(e), (long long)e);
+    regs = fa.numRegs;
+    cached.store(regs, std::memory_order_relaxed);
+  }
+  if (regs != want)
+    return fail(ATTN_ERR_LAUNCH, "%s compiled to %d registers per thread, its warpgroup split needs %d", what, regs,
+                want);
+  return ATTN_OK;
+}
+
 template <int D, bool CAUSAL, bool SPARSE, bool O32 = false, bool VARLEN = false>
 int launch_fwd(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const attn::FwdParams& prm,
                int grid, cudaStream_t st) {
   using C = attn::FwdCfg<D>;
   auto kern = attn::attn_fwd_kernel<D, CAUSAL, SPARSE, O32, VARLEN>;
   constexpr int smem = C::kSmemBytes;
-  // The kernel moves registers between its warpgroups (setmaxnreg), which
-  // only adds up if every thread was launched with exactly kRegsLaunch.
-  cudaFuncAttributes fa;
-  const cudaError_t e = cudaFuncGetAttributes(&fa, kern);
-  if (e != cudaSuccess)
-    return fail(ATTN_ERR_LAUNCH, "cudaFuncGetAttributes(forward): %s (%lld)", cudaGetErrorString(e), (long long)e);
-  if (fa.numRegs != int(C::kRegsLaunch))
-    return fail(ATTN_ERR_LAUNCH, "forward compiled to %d registers per thread, its warpgroup split needs %d",
-                fa.numRegs, int(C::kRegsLaunch));
+  if (check_launch_regs<attn::attn_fwd_kernel<D, CAUSAL, SPARSE, O32, VARLEN>>(int(C::kRegsLaunch), "forward") !=
+      ATTN_OK)
+    return ATTN_ERR_LAUNCH;
   if (set_smem(reinterpret_cast<const void*>(kern), smem) != ATTN_OK) return ATTN_ERR_LAUNCH;
   kern<<<grid, attn::FwdCfg<D>::kThreads, smem, st>>>(q, k, v, prm);
   return launch_status();
@@ -246,17 +264,9 @@ int launch_fused(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& 
                  int grid, cudaStream_t st) {
   using C = attn::FusedCfg<D>;
   auto kern = attn::attn_bwd_fused_kernel<D, CAUSAL, SPARSE>;
-  // The kernel moves registers between its warpgroups (setmaxnreg); the split
-  // only adds up if every thread was launched with exactly kRegsLaunch of them
-  // (otherwise the growing warpgroup would wait for registers that never come).
-  cudaFuncAttributes fa;
-  const cudaError_t e = cudaFuncGetAttributes(&fa, kern);
-  if (e != cudaSuccess)
-    return fail(ATTN_ERR_LAUNCH, "cudaFuncGetAttributes(fused backward): %s (%lld)", cudaGetErrorString(e),
-                (long long)e);
-  if (fa.numRegs != int(C::kRegsLaunch))
-    return fail(ATTN_ERR_LAUNCH, "fused backward compiled to %d registers per thread, its warpgroup split needs %d",
-                fa.numRegs, int(C::kRegsLaunch));
+  if (check_launch_regs<attn::attn_bwd_fused_kernel<D, CAUSAL, SPARSE>>(int(C::kRegsLaunch), "fused backward") !=
+      ATTN_OK)
+    return ATTN_ERR_LAUNCH;
   if (set_smem(reinterpret_cast<const void*>(kern), C::kSmemBytes) != ATTN_OK) return ATTN_ERR_LAUNCH;
   kern<<<grid, C::kThreads, C::kSmemBytes, st>>>(q, k, v, dO, dk, dv, dqacc, prm);
   return launch_status();
@@ -776,13 +786,8 @@ int launch_fp8(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
   using C = attn::Fp8Cfg;
   auto kern = attn::attn_fwd_fp8_kernel<CAUSAL>;
   constexpr int smem = C::kSmemBytes;
-  cudaFuncAttributes fa;   // the setmaxnreg split needs exactly kRegsLaunch per thread at launch
-  const cudaError_t e = cudaFuncGetAttributes(&fa, kern);
-  if (e != cudaSuccess)
-    return fail(ATTN_ERR_LAUNCH, "cudaFuncGetAttributes(FP8 forward): %s (%lld)", cudaGetErrorString(e), (long long)e);
-  if (fa.numRegs != int(C::kRegsLaunch))
-    return fail(ATTN_ERR_LAUNCH, "FP8 forward compiled to %d registers per thread, its warpgroup split needs %d",
-                fa.numRegs, int(C::kRegsLaunch));
+  if (check_launch_regs<attn::attn_fwd_fp8_kernel<CAUSAL>>(int(C::kRegsLaunch), "FP8 forward") != ATTN_OK)
+    return ATTN_ERR_LAUNCH;
   if (set_smem(reinterpret_cast<const void*>(kern), smem) != ATTN_OK) return ATTN_ERR_LAUNCH;
   kern<<<grid, attn::Fp8Cfg::kThreads, smem, st>>>(q, k, v, prm);
   return launch_status();

@@ -513,7 +513,11 @@ def run_ours(args, rank, world, local_rank):
         fp8 = {"workload": "long_batch forward on E4M3 Q, K, V (per-tensor scales)", "ms_fwd": round(tf, 3),
                "fwd_tflops": round(fp8_tf, 2), "peak": round(2 * burst, 1),
                "peak_kind": f"2 x bf16_tflops ({peaks_src}), nominal E4M3:BF16 ratio",
-               "frac": round(fp8_tf / (2 * burst), 4), "steps": n_f, "traffic": traffic("fp8")}
+               "frac": round(fp8_tf / (2 * burst), 4),
+               # every exponential on MUFU: 2 x 128 x 128 ex2 per 128-key step at 16 per SM
+               # cycle (2048 cycles) against 1024 cycles of E4M3 products caps it at half the peak
+               "mufu_cap_frac": 0.5, "frac_of_mufu_cap": round(fp8_tf / (2 * burst) / 0.5, 4),
+               "steps": n_f, "traffic": traffic("fp8")}
         if not args.no_cpu_baseline and rank == 0:
             # the oracle on the causal prefix of head (0, 0): first 4096 rows and keys
             import numpy as np

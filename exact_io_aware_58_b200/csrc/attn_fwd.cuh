@@ -253,6 +253,10 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int n_items = VARLEN ? packed_items(prm) : prm.n_items;
+  // d = 64 dense instances give the softmax 192 (the issue warpgroup fits in
+  // 120 there); the others use FwdCfg's 176 / 152.
+  constexpr uint32_t kRegsSoftmaxI = (D == 64 && !VARLEN) ? 192u : C::kRegsSoftmax;
+  constexpr uint32_t kRegsIssueI = 3 * C::kRegsLaunch - 2 * kRegsSoftmaxI;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -287,7 +291,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
   if (warp >= C::kWarpMma) {
    // warpgroup 2: one TMA thread, one MMA thread, two idle warps
-   regs_dec<C::kRegsIssue>();
+   regs_dec<kRegsIssueI>();
    if (warp == C::kWarpLoad) {
     // ------------------------------------------------------------------ TMA
     if (lane == 0) {
@@ -430,7 +434,7 @@ attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
    }
   } else {
     // -------------------------------------------------------------- softmax
-    regs_inc<C::kRegsSoftmax>();
+    regs_inc<kRegsSoftmaxI>();
     const int t = warp >> 2;
     const int qw = warp & 3;
     const int r = qw * 32 + lane;           // row inside the tile = TMEM lane

@@ -139,8 +139,15 @@ def attn_last_error() -> str:
     return load_library().attn_last_error().decode()
 
 
+# The current stream's raw handle without building a torch.cuda.Stream object
+# (the public call costs a few microseconds per launch); None on builds without it.
+_raw_current_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
 def _stream_handle(stream) -> ctypes.c_void_p:
     if stream is None:
+        if _raw_current_stream is not None:
+            return ctypes.c_void_p(_raw_current_stream(torch.cuda.current_device()))
         stream = torch.cuda.current_stream()
     if isinstance(stream, torch.cuda.Stream):
         return ctypes.c_void_p(stream.cuda_stream)
@@ -154,7 +161,7 @@ def _ptr(t) -> ctypes.c_void_p:
 def _check_device(name: str, t: torch.Tensor):
     # The library launches on the calling thread's current device (and takes
     # its workspace and default stream from there): every tensor must live on it.
-    if t.is_cuda and t.device.index != torch.cuda.current_device():
+    if t.is_cuda and t.get_device() != torch.cuda.current_device():
         raise ValueError(f"{name} is on {t.device}, but the current CUDA device is "
                          f"cuda:{torch.cuda.current_device()}; call under torch.cuda.device({t.device})")
 
@@ -163,13 +170,13 @@ def _check_bhnd(name: str, t: torch.Tensor, shape=None):
     if not t.is_cuda or t.dtype != torch.bfloat16 or t.dim() != 4 or not t.is_contiguous():
         raise ValueError(f"{name} must be a contiguous CUDA bf16 tensor of shape (B, H, N, d)")
     _check_device(name, t)
-    if shape is not None and tuple(t.shape) != tuple(shape):
+    if shape is not None and t.shape != tuple(shape):
         raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
 
 
 def _check_lse(t: torch.Tensor, shape):
     B, H, N, _ = shape
-    if not t.is_cuda or t.dtype != torch.float32 or tuple(t.shape) != (B, H, N) or not t.is_contiguous():
+    if not t.is_cuda or t.dtype != torch.float32 or t.shape != (B, H, N) or not t.is_contiguous():
         raise ValueError("LSE must be a contiguous CUDA float32 tensor of shape (B, H, N)")
     _check_device("LSE", t)
 
